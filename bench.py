@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Throughput of the routed-expert MoE layer (Route -> Union -> int4 SwiGLU FFN -> combine) on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl colimoe|reference]
+
+One step = one pass of the whole layer (pre-norm/logits, route, union, expert
+FFN, combine) over one batch of seeded synthetic input already resident in
+HBM; for the 16-layer stack a step is one forward through all 16 layers.
+Inputs rotate over 8 batches and L2 is flushed (a 256 MiB write) before every
+step, outside the timed events.  Each step is timed with CUDA events on the
+launching stream; the total is the sum over K steps, max over ranks.  With
+N > 1 (torchrun) every rank runs its own batches on its own replica of the
+layer (the path has no exchange step): value = tokens of all ranks / time.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle on
+the host cores instead (rank 0 only) and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "routed-MoE layer tokens/s at 1 B200; int4 weight GB/s vs HBM peak (decode)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = synth.DECODE_B1.name
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["colimoe", "reference"], default="colimoe")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--batches", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="target length of the oracle sample")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = {"glm52_layer_decode_b1": 2000, "glm52_layer_decode_b64_zipf": 400,
+                   "glm52_layer_prefill_4096": 40, "glm52_stack16_decode_b4": 200}.get(a.workload, 20)
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc, self.path, self.index = None, None, index
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(index), "-lms", "100"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S")) + float("0." + f[0].split(".")[1])
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10], f[5]))
+            except (ValueError, IndexError):
+                continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.15 <= r[0] <= t1 + 0.15]
+        use = inside if inside else rows
+        if not use:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
+
+# ------------------------------------------------------------------ the oracle leg (CPU)
+
+def oracle_sample(shape: synth.LayerShape, seconds: float):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload.
+
+    Weights of the experts the sample touches are generated beforehand (not
+    timed); the timed call is oracle.moe_layer (logits, route, union, FFN,
+    combine).  Returns (tokens/s, cores, description)."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    li = synth.LayerInputs(shape, 0, 0)
+    rw = None if shape.logits_in else li.router_w()
+    bias = li.bias()
+    per_tok = 1 if shape.tokens == 1 else 4
+    layers_timed = 1
+    scale = shape.layers  # the stack: one layer is timed and the time is scaled by the layer count
+    tok_done, elapsed, batches = 0, 0.0, 0
+    with threadpool_limits(1):
+        while elapsed < seconds and batches < 8:
+            x = synth.activations(shape, 0, batches)[:per_tok]
+            lg = None
+            if shape.logits_in:
+                lg = synth.normal_f32(0, 1000 + batches, synth.LOGITS_IN, (shape.tokens, shape.n_experts), 1.0)[:per_tok]
+            # pre-generate the touched experts' codes/scales (untimed)
+            lpre = lg if lg is not None else oracle.router_logits(x if not shape.prenorm else oracle.rms_norm(x), rw)[1]
+            ids, _, _ = oracle.route(oracle.add_bias(lpre, bias), shape.top_k)
+            need = sorted(set(ids.ravel().tolist()) | set(range(shape.n_experts, shape.n_total)))
+            kinds = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
+            pre = {(k, e): (li.expert_codes(q, e), li.expert_scales(s, e)) for k, (q, s) in kinds.items() for e in need}
+            W = oracle.ExpertWeights(lambda k, e: pre[(k, e)][0], lambda k, e: pre[(k, e)][1])
+            xin = x
+            t0 = time.perf_counter()
+            if shape.prenorm:
+                xin = oracle.rms_norm(x)
+            oracle.moe_layer(W, xin, shape.n_experts, shape.top_k, shape.n_shared, router_w=rw, bias=bias,
+                             logits_in=lg, residual_bits=x if shape.prenorm else None)
+            elapsed += (time.perf_counter() - t0) * scale * layers_timed
+            tok_done += x.shape[0]
+            batches += 1
+    desc = (f"{batches} batches x {per_tok} token(s) of {shape.name}"
+            + (f"; one layer timed, x{shape.layers} for the stack" if shape.layers > 1 else "")
+            + "; numpy float64, BLAS limited to 1 thread; touched experts' weights generated untimed")
+    return tok_done / elapsed, 1, desc
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    shape = synth.WORKLOADS[a.workload]
+    v, cores, desc = oracle_sample(shape, max(5.0, a.cpu_seconds))
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": shape.tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden,
+                       "inter": shape.inter, "experts": shape.n_experts, "top_k": shape.top_k,
+                       "shared": shape.n_shared, "layers": shape.layers},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ the GPU leg
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    import int4_routed_expert_renorm_b200 as cm
+    import synth.gpu as sg
+
+    shape = synth.WORKLOADS[a.workload]
+    T, H, I, E, k, S = shape.tokens, shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared
+    dims = cm.dims_for(H, I, E, k, S)
+    layers = []
+    for l in range(shape.layers):
+        li = synth.LayerInputs(shape, 0, l)
+        rw = None if shape.logits_in else torch.from_numpy(li.router_w()).cuda()
+        b = li.bias()
+        layers.append(cm.MoELayer(dims, sg.expert_tensors(shape, 0, l), rw, None if b is None else torch.from_numpy(b).cuda()))
+    NB = a.batches
+    xs = [torch.from_numpy(synth.activations(shape, 0, rank * NB + b).view(np.int16)).cuda() for b in range(NB)]
+    lgs = [None] * NB
+    if shape.logits_in:
+        lgs = [torch.from_numpy(synth.normal_f32(0, 1000 + rank * NB + b, synth.LOGITS_IN, (T, E), 1.0)).cuda()
+               for b in range(NB)]
+    ws = layers[0].workspace(T)
+    outs = [torch.empty((T, H), dtype=torch.int16, device="cuda") for _ in range(2)]
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flags = cm._lib.COLI_LAYER_PRENORM if shape.prenorm else 0
+
+    def step(bi, x=None, out=None):
+        x = xs[bi] if x is None else x
+        if shape.layers == 1:
+            o = outs[0] if out is None else out
+            layers[0].forward(x, o, ws, logits_in=lgs[bi], flags=flags)
+            return o
+        h = x
+        for li_, lay in enumerate(layers):
+            o = outs[li_ % 2] if (out is None or li_ < len(layers) - 1) else out
+            lay.forward(h, o, ws, residual=h if shape.prenorm else None, flags=flags)
+            h = o
+        return h
+
+    # union size per batch (first layer), for the bytes-touched accounting
+    U = []
+    ids_buf = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    for bi in range(NB):
+        layers[0].forward(xs[bi], outs[0], ws, logits_in=lgs[bi], flags=flags, topk_ids_out=ids_buf)
+        U.append(int(torch.unique(ids_buf).numel()))
+    st, fl = cm.coli_moe_get_status()
+    if fl:
+        raise RuntimeError(f"device status flags {fl:#x} after the first pass")
+    u_stack = []
+    if shape.layers > 1:  # union size of every layer, batch 0 (one untimed forward)
+        h = xs[0]
+        for li_, lay in enumerate(layers):
+            o = outs[li_ % 2]
+            lay.forward(h, o, ws, residual=h, flags=flags, topk_ids_out=ids_buf)
+            u_stack.append(int(torch.unique(ids_buf).numel()))
+            h = o
+
+    for i in range(a.warmup):
+        step(i % NB)
+    torch.cuda.synchronize()
+
+    K = a.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    M = min(K, 64)
+    stage = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(M)]
+    for evs in stage:  # create the events (they exist once recorded)
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    cm.coli_moe_launch_count(reset=True)
+    t_wall0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record()
+        if i < M:
+            cm.coli_moe_set_stage_events(stage[i])
+        step(i % NB)
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    launches = cm.coli_moe_launch_count()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
+    st, fl = cm.coli_moe_get_status()
+    if fl:
+        raise RuntimeError(f"device status flags {fl:#x} in the timed region")
+
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * T * K / (total_ms / 1e3)
+
+    # dominant kernel: the gate/up expert FFN (stage 5 -> 6), timed live
+    gu_ms = [stage[i][5].elapsed_time(stage[i][6]) for i in range(M)]
+    dn_ms = [stage[i][6].elapsed_time(stage[i][7]) for i in range(M)]
+    gu_avg = statistics.mean(gu_ms)
+    hbm, tf_burst, tf_sus, src = peaks()
+    per_mat = H * I // 2 + (H * I // 32) * 2
+    P = T * k
+    u_step = [U[i % NB] for i in range(M)]  # the first layer of each step carries the stage events
+    if shape.name == synth.PREFILL_4096.name:
+        flops = 2 * 2 * H * I * (P + S * T)
+        achieved = flops / (gu_avg / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_sus, "unit": "TFLOP/s",
+                "frac": achieved / tf_sus, "traffic": None,
+                "kernel": "ffn_decode_kernel<0,256> (gate/up, mma.sync bf16)", "peak_kind": f"{src} sustained bf16"}
+    else:
+        gu_bytes = [(u + S) * 2 * per_mat + T * H * 2 + (P + S * T) * I * 2 for u in u_step]
+        achieved = statistics.mean(b / (ms / 1e3) / 1e9 for b, ms in zip(gu_bytes, gu_ms))
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": None, "kernel": "ffn_decode_kernel<0,256> (gate/up)", "peak_kind": f"{src} HBM copy"}
+
+    # int4 bytes touched per step (all three matrices of every unique + shared expert)
+    exp_bytes = shape.expert_bytes()
+    if shape.layers == 1:
+        bytes_step = statistics.mean((U[i % NB] + S) * exp_bytes for i in range(K))
+    else:
+        bytes_step = sum((u + S) * exp_bytes for u in u_stack)
+    int4_gbs = bytes_step / (statistics.mean(step_ms) / 1e3) / 1e9
+
+    # end to end through the public API with host buffers
+    xh = [torch.empty((T, H), dtype=torch.int16, pin_memory=True) for _ in range(NB)]
+    for bi in range(NB):
+        xh[bi].copy_(xs[bi].cpu())
+    lh = [None] * NB
+    if shape.logits_in:
+        lh = [lgs[bi].cpu().pin_memory() for bi in range(NB)]
+    oh = torch.empty((T, H), dtype=torch.int16, pin_memory=True)
+    xd = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    ld = torch.empty((T, E), dtype=torch.float32, device="cuda") if shape.logits_in else None
+    od = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    K2 = min(K, 500)
+    e2e_ms = []
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(K2)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(K2)]
+    for i in range(K2):
+        bi = i % NB
+        flush.zero_()
+        es[i].record()
+        xd.copy_(xh[bi], non_blocking=True)
+        if ld is not None:
+            ld.copy_(lh[bi], non_blocking=True)
+            lgs_save = lgs[bi]
+            lgs[bi] = ld
+        step(bi, x=xd, out=od)
+        if ld is not None:
+            lgs[bi] = lgs_save
+        oh.copy_(od, non_blocking=True)
+        ee[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(es[i].elapsed_time(ee[i]) for i in range(K2))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * T * K2 / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": T * H * 2 + (T * E * 4 if shape.logits_in else 0), "d2h_bytes_per_step": T * H * 2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, cores, desc = oracle_sample(shape, a.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": a.warmup,
+            "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": shape.name, "tokens": T, "hidden": H, "inter": I, "experts": E, "top_k": k,
+                       "shared": S, "layers": shape.layers, "union_per_batch": U,
+                       "union_per_layer": u_stack or None, "l2": "flushed (256 MiB write) before every step",
+                       "rotating_batches": NB},
+            "int4_bytes_per_step": bytes_step, "int4_gbs": int4_gbs, "int4_frac_of_hbm": int4_gbs / hbm,
+            "roofline": roof, "down_kernel_ms": statistics.mean(dn_ms), "gateup_kernel_ms": gu_avg,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * coli_moe.h -- C ABI of the B200 routed-expert MoE step
+ *               (Route -> Union -> int4 SwiGLU expert FFN -> combine).
+ *
+ * The per-token path this library computes is the one the Colibri README
+ * describes ("Come funziona", "Il percorso di ogni token": every layer of
+ * every token goes Route, then Union, before the expert matmuls) and the
+ * getting-started guide lists ("トークンごとの処理経路", steps 1 Route and
+ * 2 Union).  The pages fix that the router picks experts per token and per
+ * layer, that a batch reads each unique expert once (README, "Mai aspettare il
+ * disco due volte": batch-union), that routed experts are stored int4
+ * (README, "L'idea") and that placement never changes the router's decisions
+ * or the weights' precision.  Placement itself (VRAM/RAM/disk tiering) is not
+ * part of this library: every expert is resident in device memory (the
+ * README's full expert residence, "Una gerarchia di memoria").
+ *
+ * Numerics this library implements (the pages give no formula):
+ *   logits   l[t,e] = sum_h x[t,h] * W_r[e,h]           (fp32, x bf16)
+ *   bias     l'[t,e] = l[t,e] + bias[e]                 (one fp32 add; optional)
+ *   route    top-k of l' by (value desc, index asc); slot j = j-th in that order;
+ *            w_j = exp(l'_j - l'_max) / sum_{i<k} exp(l'_i - l'_max)
+ *   union    unique experts ascending; pairs p = t*k + j grouped by expert,
+ *            stable in p
+ *   expert   W = code * scale, code int4 in [-8,7], fp16 scale per 32 along K;
+ *            h = bf16( silu(W_gate x) * (W_up x) ),  y = W_down h   (fp32 accumulate)
+ *   combine  out[t] = bf16( sum_j w[t,j] * y_{id[t,j]} + sum_s y_{E+s} + residual[t] )
+ *
+ * Container format (row-major, K contiguous):
+ *   gate_q, up_q  uint8 [E+S][I][H/2]   down_q uint8 [E+S][H][I/2]
+ *   gate_s, up_s  fp16  [E+S][I][H/32]  down_s fp16  [E+S][H][I/32]
+ *   Element c of a row is nibble (c & 1) of byte c/2 (low nibble first); the
+ *   nibble n encodes code n - 16*(n >= 8).  Shared experts are ids E..E+S-1.
+ *
+ * Conventions for every call:
+ *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
+ *     The library allocates no memory, keeps no per-call state and does not
+ *     retain pointers after the call returns.
+ *   - bf16 / fp16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work on it: they never synchronise, never allocate, and can be
+ *     captured into a CUDA graph (except coli_moe_get_status).
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched.  Errors found on the device (non-finite logits, expert ids out
+ *     of range, a pipeline wait that timed out) set bits in a per-device
+ *     status word that coli_moe_get_status reads and clears; kernels never
+ *     trap.
+ *   - Supported shapes: group == 32, H % 256 == 0, I % 256 == 0 or I == 128,
+ *     1 <= k <= min(E, 32), E <= 1024, 0 <= S <= 4, T >= 0, T*k <= 2^24.
+ *     Anything else returns COLI_ERR_UNSUPPORTED.
+ *   - Thread safety: calls may be made concurrently from several host
+ *     threads on different streams; the device status word is shared by all
+ *     of them.
+ */
+#ifndef COLI_MOE_H
+#define COLI_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  COLI_OK = 0,
+  COLI_ERR_INVALID_ARG = 1,  /* NULL where a pointer is required, negative size, bad stride */
+  COLI_ERR_UNSUPPORTED = 2,  /* shape outside the supported set above */
+  COLI_ERR_WORKSPACE = 3,    /* ws_bytes smaller than coli_moe_workspace_bytes() */
+  COLI_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute, symbol) */
+  COLI_ERR_NONFINITE = 5,    /* returned by coli_moe_get_status only */
+  COLI_ERR_DEVICE = 6        /* returned by coli_moe_get_status: other device-side error bits */
+} coli_status;
+
+/* Device status bits (coli_moe_get_status). */
+#define COLI_FLAG_NONFINITE 0x1u  /* a logit was NaN or +inf, or a selected logit was -inf */
+#define COLI_FLAG_BAD_ID    0x2u  /* an expert id outside [0, E) reached the union */
+#define COLI_FLAG_TIMEOUT   0x4u  /* a bounded pipeline wait expired; outputs are undefined */
+
+/* Layer flags (coli_moe_layer / coli_moe_expert_ffn). */
+#define COLI_LAYER_PRENORM       0x1u  /* route and run the experts on n = bf16(x * rsqrt(mean(x^2) + 1e-6)) */
+#define COLI_PATH_DECODE         0x10u /* force the CUDA-core/mma.sync decode FFN form */
+#define COLI_PATH_PREFILL        0x20u /* force the tcgen05 grouped-GEMM FFN form */
+
+typedef struct {
+  int32_t hidden;     /* H */
+  int32_t inter;      /* I: expert intermediate size */
+  int32_t n_experts;  /* E: routed experts */
+  int32_t top_k;      /* k */
+  int32_t n_shared;   /* S: shared experts, always active with weight 1.0 */
+  int32_t group;      /* quantisation group along K; must be 32 */
+} coli_moe_dims;
+
+typedef struct {
+  const uint8_t *gate_q, *up_q, *down_q;     /* packed int4 codes, layout above */
+  const uint16_t *gate_s, *up_s, *down_s;    /* fp16 scale bits, layout above */
+  const float *router_w;                     /* fp32 [E][H]; may be NULL if logits are supplied */
+  const float *router_bias;                  /* fp32 [E] or NULL */
+} coli_moe_weights;
+
+/*
+ * Route: top-k selection and renormalised softmax weights per token.
+ *   logits   fp32 [T][E]   router logits (device)
+ *   bias     fp32 [E]      additive per-expert bias, or NULL
+ *   topk_ids int32 [T][k]  out: selected experts, slot order = selection order
+ *   topk_w   fp32 [T][k]   out: renormalised weights (sum to 1 per token)
+ * Ties go to the lowest expert index; -0.0 ties +0.0; a NaN logit ranks as
+ * -inf and sets COLI_FLAG_NONFINITE.  T == 0 is a no-op.
+ */
+coli_status coli_moe_route(const float *logits, const float *bias, int T, int E, int k,
+                           int32_t *topk_ids, float *topk_w, void *stream);
+
+/*
+ * Union: batch-union of the selected experts, without atomics.
+ *   topk_ids  int32 [T][k]        in
+ *   unique_ids int32 [min(E,T*k)] out: experts used by the batch, ascending
+ *   n_unique  int32 [1]           out: U (stays on the device)
+ *   seg_off   int32 [min(E,T*k)+1] out: pairs of unique_ids[u] are
+ *                                 perm[seg_off[u] .. seg_off[u+1])
+ *   perm      int32 [T*k]         out: pair indices p = t*k + j, sorted by
+ *                                 (expert, p)
+ *   pair_pos  int32 [T*k]         out: inverse of perm (-1 for a pair whose id
+ *                                 was out of range; COLI_FLAG_BAD_ID is set)
+ * Entries of unique_ids/seg_off past U are left unchanged.  One CTA; T*k <= 2^24.
+ */
+coli_status coli_moe_union(const int32_t *topk_ids, int T, int k, int E,
+                           int32_t *unique_ids, int32_t *n_unique, int32_t *seg_off,
+                           int32_t *perm, int32_t *pair_pos, void *stream);
+
+/*
+ * Expert FFN + combine for an already routed and unioned batch.
+ *   x         bf16 [T][H]   expert input
+ *   topk_ids, topk_w, unique_ids, n_unique, seg_off, perm, pair_pos:
+ *             as produced by coli_moe_route / coli_moe_union
+ *   residual  bf16 [T][H] or NULL (added once, in fp32, before rounding)
+ *   out       bf16 [T][H]   out (must not alias x; may alias residual)
+ *   ws        device scratch of at least coli_moe_workspace_bytes(dims, T) bytes,
+ *             256-byte aligned, owned by the caller; contents on entry are ignored
+ *   flags     COLI_PATH_* selects the FFN form (0 = automatic)
+ */
+coli_status coli_moe_expert_ffn(const coli_moe_dims *dims, const coli_moe_weights *w,
+                                const uint16_t *x, int T,
+                                const int32_t *topk_ids, const float *topk_w,
+                                const int32_t *unique_ids, const int32_t *n_unique,
+                                const int32_t *seg_off, const int32_t *perm,
+                                const int32_t *pair_pos, const uint16_t *residual,
+                                uint16_t *out, uint32_t flags, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/*
+ * One whole MoE layer: [pre-norm] -> logits -> Route -> Union -> FFN -> combine.
+ *   x          bf16 [T][H]
+ *   logits_in  fp32 [T][E] or NULL: when given, replaces x . W_r^T
+ *   residual   bf16 [T][H] or NULL
+ *   flags      COLI_LAYER_PRENORM and/or COLI_PATH_*
+ *   out        bf16 [T][H]   (must not alias x; may alias residual)
+ *   logits_out fp32 [T][E] or NULL: the logits used (before the bias)
+ *   topk_ids_out int32 [T][k] or NULL, topk_w_out fp32 [T][k] or NULL
+ *   ws / ws_bytes as for coli_moe_expert_ffn
+ */
+coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
+                           const uint16_t *x, int T, const float *logits_in,
+                           const uint16_t *residual, uint32_t flags, uint16_t *out,
+                           float *logits_out, int32_t *topk_ids_out, float *topk_w_out,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes needed by coli_moe_layer / coli_moe_expert_ffn for up to T_max
+ * tokens (0 for unsupported dims). Host only. */
+size_t coli_moe_workspace_bytes(const coli_moe_dims *dims, int T_max);
+
+/* Synchronises `stream`, then reads and clears the calling device's status
+ * word.  *flags (host pointer, may be NULL) receives the COLI_FLAG_* bits.
+ * Returns COLI_OK when no bit was set, COLI_ERR_NONFINITE when only the
+ * NONFINITE bit was set, COLI_ERR_DEVICE for any other bit, COLI_ERR_CUDA if
+ * the synchronisation failed.  Not capturable. */
+coli_status coli_moe_get_status(void *stream, uint32_t *flags);
+
+/* Static description of a status code. */
+const char *coli_status_str(coli_status s);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int coli_moe_version(void);
+
+/* Number of kernel launches made by the calling host thread since the last
+ * reset (reset != 0 clears it).  Counting only; no device work. */
+uint64_t coli_moe_launch_count(int reset);
+
+/* Timing hook (diagnostics, host only).  While set, the next coli_moe_layer or
+ * coli_moe_expert_ffn call made by this host thread records events[i]
+ * (cudaEvent_t handles owned by the caller, created on the call's device) on
+ * its stream at internal stage boundary i, for i < n:
+ *   0 start, 1 after pre-norm/fragment copy, 2 after logits, 3 after route,
+ *   4 after union, 5 after tile plan, 6 after gate/up FFN, 7 after down FFN,
+ *   8 after combine.
+ * Stages a call does not run record at the same point as the previous one.
+ * The setting is consumed by that one call; n = 0 or events = NULL clears it. */
+coli_status coli_moe_set_stage_events(void *const *events, int n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COLI_MOE_H */

@@ -1,0 +1,146 @@
+"""ctypes binding of libcolimoe (include/coli_moe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors that already live on the device (or None where the C call accepts
+NULL), passes their data pointers and the current CUDA stream, and raises
+``ColiError`` on a non-OK status.  No step of the layer runs in Python; if the
+library is missing the import fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libcolimoe.so")
+
+# COLI_* constants of include/coli_moe.h
+COLI_OK, COLI_ERR_INVALID_ARG, COLI_ERR_UNSUPPORTED, COLI_ERR_WORKSPACE = 0, 1, 2, 3
+COLI_ERR_CUDA, COLI_ERR_NONFINITE, COLI_ERR_DEVICE = 4, 5, 6
+COLI_FLAG_NONFINITE, COLI_FLAG_BAD_ID, COLI_FLAG_TIMEOUT = 0x1, 0x2, 0x4
+COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
+
+EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
+           "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
+           "coli_moe_launch_count", "coli_moe_set_stage_events")
+
+
+class ColiError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+        self.status = status
+
+
+class coli_moe_dims(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("group", ctypes.c_int32)]
+
+
+class coli_moe_weights(ctypes.Structure):
+    _fields_ = [("gate_q", ctypes.c_void_p), ("up_q", ctypes.c_void_p), ("down_q", ctypes.c_void_p),
+                ("gate_s", ctypes.c_void_p), ("up_s", ctypes.c_void_p), ("down_s", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p)]
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m int4_routed_expert_renorm_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, Z, U32, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_uint64
+    D, W = ctypes.POINTER(coli_moe_dims), ctypes.POINTER(coli_moe_weights)
+    sig = {
+        "coli_moe_route": (I, [P, P, I, I, I, P, P, P]),
+        "coli_moe_union": (I, [P, I, I, I, P, P, P, P, P, P]),
+        "coli_moe_expert_ffn": (I, [D, W, P, I, P, P, P, P, P, P, P, P, P, U32, P, Z, P]),
+        "coli_moe_layer": (I, [D, W, P, I, P, P, U32, P, P, P, P, P, Z, P]),
+        "coli_moe_workspace_bytes": (Z, [D, I]),
+        "coli_moe_get_status": (I, [P, ctypes.POINTER(U32)]),
+        "coli_status_str": (ctypes.c_char_p, [I]),
+        "coli_moe_version": (I, []),
+        "coli_moe_launch_count": (U64, [I]),
+        "coli_moe_set_stage_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    return lib
+
+
+_lib = load()
+
+
+def status_str(s: int) -> str:
+    return _lib.coli_status_str(s).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(st: int, where: str):
+    if st != COLI_OK:
+        raise ColiError(st, where)
+
+
+def coli_moe_version() -> int:
+    return _lib.coli_moe_version()
+
+
+def coli_moe_launch_count(reset: bool = False) -> int:
+    return _lib.coli_moe_launch_count(1 if reset else 0)
+
+
+def coli_moe_workspace_bytes(dims: coli_moe_dims, t_max: int) -> int:
+    return _lib.coli_moe_workspace_bytes(ctypes.byref(dims), t_max)
+
+
+def coli_moe_route(logits, bias, topk_ids, topk_w, stream=None):
+    T, E = logits.shape
+    k = topk_ids.shape[1]
+    _check(_lib.coli_moe_route(_ptr(logits), _ptr(bias), T, E, k, _ptr(topk_ids), _ptr(topk_w), _stream(stream)),
+           "coli_moe_route")
+
+
+def coli_moe_union(topk_ids, n_experts, unique_ids, n_unique, seg_off, perm, pair_pos, stream=None):
+    T, k = topk_ids.shape
+    _check(_lib.coli_moe_union(_ptr(topk_ids), T, k, n_experts, _ptr(unique_ids), _ptr(n_unique), _ptr(seg_off),
+                               _ptr(perm), _ptr(pair_pos), _stream(stream)), "coli_moe_union")
+
+
+def coli_moe_expert_ffn(dims, weights, x, topk_ids, topk_w, unique_ids, n_unique, seg_off, perm, pair_pos,
+                        residual, out, ws, flags=0, stream=None):
+    T = x.shape[0]
+    _check(_lib.coli_moe_expert_ffn(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(topk_ids),
+                                    _ptr(topk_w), _ptr(unique_ids), _ptr(n_unique), _ptr(seg_off), _ptr(perm),
+                                    _ptr(pair_pos), _ptr(residual), _ptr(out), flags, _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "coli_moe_expert_ffn")
+
+
+def coli_moe_layer(dims, weights, x, out, ws, logits_in=None, residual=None, flags=0, logits_out=None,
+                   topk_ids_out=None, topk_w_out=None, stream=None):
+    T = x.shape[0]
+    _check(_lib.coli_moe_layer(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
+                               _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
+                               _ptr(topk_w_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "coli_moe_layer")
+
+
+def coli_moe_set_stage_events(events):
+    """events: list of torch.cuda.Event (already recorded once, so they exist) or []."""
+    n = len(events)
+    arr = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in events])
+    _check(_lib.coli_moe_set_stage_events(arr if n else None, n), "coli_moe_set_stage_events")
+
+
+def coli_moe_get_status(stream=None):
+    """Returns (status, flags); synchronises the stream and clears the device word."""
+    f = ctypes.c_uint32(0)
+    st = _lib.coli_moe_get_status(_stream(stream), ctypes.byref(f))
+    return st, f.value

@@ -1,0 +1,454 @@
+// libcolimoe: host side of the C ABI declared in include/coli_moe.h.
+//
+// Argument checking, workspace layout, tensor-map encoding and the launch
+// sequence of one routed-expert MoE layer (Colibri README, "Il percorso di
+// ogni token": Route -> Union -> expert matmuls, every layer of every token).
+// All device work is enqueued on the caller's stream; nothing here allocates
+// or synchronises, except coli_moe_get_status.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "k_ffn_decode.cuh"
+#include "k_router.cuh"
+#include "k_union.cuh"
+
+using namespace coli;
+
+namespace {
+
+__device__ uint32_t g_status_word;
+
+thread_local uint64_t t_launches = 0;
+
+// Stage events of the timing hook (coli_moe_set_stage_events); consumed by one call.
+constexpr int kMaxStageEvents = 16;
+thread_local cudaEvent_t t_stage_ev[kMaxStageEvents];
+thread_local int t_stage_n = 0;
+
+struct StageRecorder {
+  cudaEvent_t ev[kMaxStageEvents];
+  int n;
+  cudaStream_t st;
+  explicit StageRecorder(cudaStream_t s) : n(t_stage_n), st(s) {
+    for (int i = 0; i < n; ++i) ev[i] = t_stage_ev[i];
+    t_stage_n = 0;
+  }
+  void mark(int i) const {
+    if (i < n) cudaEventRecord(ev[i], st);
+  }
+  void mark_through(int i0, int i1) const {
+    for (int i = i0; i <= i1; ++i) mark(i);
+  }
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t* g_status_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+bool g_attr_done[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+struct DevInfo {
+  uint32_t* status;
+  int sms;
+};
+
+coli_status dev_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return COLI_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return COLI_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return COLI_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    g_num_sms[dev] = sms;
+  }
+  if (!g_attr_done[dev]) {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(ffn_decode_kernel<0, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(FfnCfg<0, 256>::SMEM)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(ffn_decode_kernel<1, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(FfnCfg<1, 256>::SMEM)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(ffn_decode_kernel<1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(FfnCfg<1, 128>::SMEM)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kUnionWarps * 1024 * 4) == cudaSuccess;
+    if (!ok) return COLI_ERR_CUDA;
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return COLI_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    g_attr_done[dev] = true;
+  }
+  out->status = g_status_ptr[dev];
+  out->sms = g_num_sms[dev];
+  return COLI_OK;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline bool launched_ok() {
+  ++t_launches;
+  return cudaPeekAtLastError() == cudaSuccess;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+coli_status check_dims(const coli_moe_dims* d) {
+  if (!d) return COLI_ERR_INVALID_ARG;
+  if (d->group != 32) return COLI_ERR_UNSUPPORTED;
+  if (d->hidden <= 0 || d->hidden % 256 != 0) return COLI_ERR_UNSUPPORTED;
+  if (d->inter <= 0 || !(d->inter % 256 == 0 || d->inter == 128)) return COLI_ERR_UNSUPPORTED;
+  if (d->n_experts < 1 || d->n_experts > 1024) return COLI_ERR_UNSUPPORTED;
+  if (d->top_k < 1 || d->top_k > 32 || d->top_k > d->n_experts) return COLI_ERR_UNSUPPORTED;
+  if (d->n_shared < 0 || d->n_shared > 4) return COLI_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->n_experts + d->n_shared) * d->hidden > (int64_t(1) << 31)) return COLI_ERR_UNSUPPORTED;
+  return COLI_OK;
+}
+
+coli_status check_weights(const coli_moe_weights* w, bool need_router) {
+  if (!w || !w->gate_q || !w->up_q || !w->down_q || !w->gate_s || !w->up_s || !w->down_s)
+    return COLI_ERR_INVALID_ARG;
+  if (need_router && !w->router_w) return COLI_ERR_INVALID_ARG;
+  const void* ps[6] = {w->gate_q, w->up_q, w->down_q, w->gate_s, w->up_s, w->down_s};
+  for (const void* p : ps)
+    if (!aligned(p, 16)) return COLI_ERR_INVALID_ARG;
+  if (need_router && !aligned(w->router_w, 16)) return COLI_ERR_INVALID_ARG;
+  return COLI_OK;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace layout for T tokens (every region 256-byte aligned).
+struct Ws {
+  uint16_t* xq;      // [T][H] fragment-ordered expert input
+  uint16_t* xn;      // [T][H] normalised input (prenorm)
+  float* logits;     // [T][E]
+  int32_t* ids;      // [T*k]
+  float* w;          // [T*k]
+  int32_t* unique;   // [min(E,P)]
+  int32_t* n_unique; // [1]
+  int32_t* seg_off;  // [min(E,P)+1]
+  int32_t* perm;     // [P]
+  int32_t* pair_pos; // [P]
+  int32_t* plan;     // [min(E,P)+S+3]
+  uint16_t* hq;      // [P+S*T][I]
+  float* ypair;      // [P+S*T][H]
+  size_t bytes;
+};
+
+Ws layout(const coli_moe_dims* d, int T, void* base) {
+  Ws ws{};
+  const size_t H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
+  const size_t P = static_cast<size_t>(T) * k;
+  const size_t Umax = P < E ? P : E;
+  const size_t rows = P + S * static_cast<size_t>(T);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t o = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = b ? b + o : nullptr;
+    o += align256(bytes);
+    return p;
+  };
+  ws.xq = static_cast<uint16_t*>(take(T * H * 2));
+  ws.xn = static_cast<uint16_t*>(take(T * H * 2));
+  ws.logits = static_cast<float*>(take(T * E * 4));
+  ws.ids = static_cast<int32_t*>(take(P * 4));
+  ws.w = static_cast<float*>(take(P * 4));
+  ws.unique = static_cast<int32_t*>(take(Umax * 4));
+  ws.n_unique = static_cast<int32_t*>(take(4));
+  ws.seg_off = static_cast<int32_t*>(take((Umax + 1) * 4));
+  ws.perm = static_cast<int32_t*>(take(P * 4));
+  ws.pair_pos = static_cast<int32_t*>(take(P * 4));
+  ws.plan = static_cast<int32_t*>(take((Umax + S + 3) * 4));
+  ws.hq = static_cast<uint16_t*>(take(rows * I * 2));
+  ws.ypair = static_cast<float*>(take(rows * H * 4));
+  ws.bytes = o;
+  return ws;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of one matrix kind: codes [rows_total][K/2] bytes and scales
+// [rows_total][K/32] fp16, tiles of 128 rows x KC elements.
+bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, CUtensorMap* mq,
+                 CUtensorMap* ms) {
+  const CUtensorMapSwizzle swz = KC == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, KC / 2, kRowBlock, swz))
+    return false;
+  if (KC < K) {
+    if (!encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / 32, rows_total, (K / 32) * 2, KC / 32, kRowBlock,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  } else {
+    std::memset(ms, 0, sizeof(*ms));  // scales move by 1-D bulk copies when a stage spans K
+  }
+  return true;
+}
+
+template <int MODE, int KC>
+bool launch_ffn(const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& s0, const CUtensorMap& s1,
+                const FfnArgs& a, int grid, cudaStream_t st) {
+  ffn_decode_kernel<MODE, KC><<<grid, kFfnThreads, FfnCfg<MODE, KC>::SMEM, st>>>(q0, q1, s0, s1, a);
+  return launched_ok();
+}
+
+// The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer.
+coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
+                    const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
+                    const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
+                    cudaStream_t st, const StageRecorder& rec) {
+  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
+  const int P = T * k;
+  const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
+  const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
+
+  plan_kernel<<<1, 1024, 0, st>>>(n_unique, seg_off, T, S, ws.plan);
+  if (!launched_ok()) return COLI_ERR_CUDA;
+  rec.mark(5);
+
+  // upper bound on tiles: every segment contributes ceil(cnt/64) <= cnt/64 + 1 blocks
+  const int Umax = P < E ? P : E;
+  const long blocks_ub = static_cast<long>(Umax) + P / kTokBlock + static_cast<long>(S) * ((T + kTokBlock - 1) / kTokBlock);
+
+  CUtensorMap gq, uq, gs, us, dq, ds;
+  const int kc_dn = (I % 256 == 0) ? 256 : 128;
+  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, &gq, &gs) ||
+      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, &uq, &us) ||
+      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, &dq, &ds))
+    return COLI_ERR_CUDA;
+
+  FfnArgs a{};
+  a.unique_ids = unique;
+  a.n_unique = n_unique;
+  a.seg_off = seg_off;
+  a.perm = perm;
+  a.plan = ws.plan;
+  a.status = di.status;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.P = P;
+
+  // gate/up + SiLU*mul -> h
+  a.bsrc = ws.xq;
+  a.scales0 = w->gate_s;
+  a.scales1 = w->up_s;
+  a.hq = ws.hq;
+  a.ypair = nullptr;
+  a.K = H;
+  a.R = I;
+  {
+    const long tiles = blocks_ub * (I / kRowBlock);
+    const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
+    if (!launch_ffn<0, 256>(gq, uq, gs, us, a, grid, st)) return COLI_ERR_CUDA;
+  }
+  rec.mark(6);
+  // down -> y per (pair, row)
+  a.bsrc = ws.hq;
+  a.scales0 = w->down_s;
+  a.scales1 = w->down_s;
+  a.hq = nullptr;
+  a.ypair = ws.ypair;
+  a.K = I;
+  a.R = H;
+  {
+    const long tiles = blocks_ub * (H / kRowBlock);
+    const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
+    const bool ok = kc_dn == 256 ? launch_ffn<1, 256>(dq, dq, ds, ds, a, grid, st)
+                                 : launch_ffn<1, 128>(dq, dq, ds, ds, a, grid, st);
+    if (!ok) return COLI_ERR_CUDA;
+  }
+  rec.mark(7);
+  // combine
+  {
+    const long work = static_cast<long>(T) * (H / 4);
+    long blocks = (work + 255) / 256;
+    if (blocks > 4L * di.sms) blocks = 4L * di.sms;
+    combine_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(ws.ypair, pair_pos, topk_w, residual, T, k, S, H, out);
+    if (!launched_ok()) return COLI_ERR_CUDA;
+  }
+  rec.mark(8);
+  return COLI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int coli_moe_version(void) { return 100; }
+
+uint64_t coli_moe_launch_count(int reset) {
+  const uint64_t v = t_launches;
+  if (reset) t_launches = 0;
+  return v;
+}
+
+coli_status coli_moe_set_stage_events(void* const* events, int n) {
+  if (n < 0 || n > kMaxStageEvents || (n > 0 && !events)) return COLI_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) t_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
+  t_stage_n = events ? n : 0;
+  return COLI_OK;
+}
+
+const char* coli_status_str(coli_status s) {
+  switch (s) {
+    case COLI_OK: return "ok";
+    case COLI_ERR_INVALID_ARG: return "invalid argument";
+    case COLI_ERR_UNSUPPORTED: return "unsupported shape";
+    case COLI_ERR_WORKSPACE: return "workspace too small";
+    case COLI_ERR_CUDA: return "CUDA runtime error";
+    case COLI_ERR_NONFINITE: return "non-finite router logits";
+    case COLI_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+size_t coli_moe_workspace_bytes(const coli_moe_dims* dims, int T_max) {
+  if (check_dims(dims) != COLI_OK || T_max < 0) return 0;
+  return layout(dims, T_max, nullptr).bytes;
+}
+
+coli_status coli_moe_route(const float* logits, const float* bias, int T, int E, int k, int32_t* topk_ids,
+                           float* topk_w, void* stream) {
+  if (T < 0 || E < 1 || k < 1) return COLI_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || k > E) return COLI_ERR_UNSUPPORTED;
+  if (T == 0) return COLI_OK;
+  if (!logits || !topk_ids || !topk_w) return COLI_ERR_INVALID_ARG;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  route_kernel<<<(T + 7) / 8, 256, 0, as_stream(stream)>>>(logits, bias, T, E, k, topk_ids, topk_w, di.status);
+  return launched_ok() ? COLI_OK : COLI_ERR_CUDA;
+}
+
+coli_status coli_moe_union(const int32_t* topk_ids, int T, int k, int E, int32_t* unique_ids, int32_t* n_unique,
+                           int32_t* seg_off, int32_t* perm, int32_t* pair_pos, void* stream) {
+  if (T < 0 || k < 1 || E < 1) return COLI_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || static_cast<int64_t>(T) * k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  if (!n_unique || !seg_off) return COLI_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !unique_ids || !perm || !pair_pos)) return COLI_ERR_INVALID_ARG;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  union_kernel<<<1, kUnionThreads, kUnionWarps * E * 4, as_stream(stream)>>>(topk_ids, T * k, E, unique_ids, n_unique,
+                                                                             seg_off, perm, pair_pos, di.status);
+  return launched_ok() ? COLI_OK : COLI_ERR_CUDA;
+}
+
+coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
+                                const int32_t* topk_ids, const float* topk_w, const int32_t* unique_ids,
+                                const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm,
+                                const int32_t* pair_pos, const uint16_t* residual, uint16_t* out, uint32_t flags,
+                                void* ws, size_t ws_bytes, void* stream) {
+  coli_status st = check_dims(dims);
+  if (st != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  if ((st = check_weights(w, false)) != COLI_OK) return st;
+  if (T == 0) return COLI_OK;
+  if (!x || !topk_ids || !topk_w || !unique_ids || !n_unique || !seg_off || !perm || !pair_pos || !out || !ws)
+    return COLI_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
+    return COLI_ERR_INVALID_ARG;
+  if (x == out) return COLI_ERR_INVALID_ARG;
+  if (flags & COLI_PATH_PREFILL) return COLI_ERR_UNSUPPORTED;
+  const Ws lay = layout(dims, T, ws);
+  if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const StageRecorder rec(s);
+  rec.mark(0);
+  prep_kernel<<<T, 256, 0, s>>>(x, dims->hidden, 0, nullptr, lay.xq);
+  if (!launched_ok()) return COLI_ERR_CUDA;
+  rec.mark_through(1, 4);
+  return run_ffn(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di, s, rec);
+}
+
+coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
+                           const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
+                           float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  coli_status st = check_dims(dims);
+  if (st != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  if ((st = check_weights(w, logits_in == nullptr)) != COLI_OK) return st;
+  if (T == 0) return COLI_OK;
+  if (!x || !out || !ws) return COLI_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
+    return COLI_ERR_INVALID_ARG;
+  if (x == out) return COLI_ERR_INVALID_ARG;
+  if (flags & COLI_PATH_PREFILL) return COLI_ERR_UNSUPPORTED;
+  const Ws lay = layout(dims, T, ws);
+  if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int H = dims->hidden, E = dims->n_experts, k = dims->top_k;
+  const bool prenorm = (flags & COLI_LAYER_PRENORM) != 0;
+  const StageRecorder rec(s);
+  rec.mark(0);
+
+  prep_kernel<<<T, 256, 0, s>>>(x, H, prenorm ? 1 : 0, lay.xn, lay.xq);
+  if (!launched_ok()) return COLI_ERR_CUDA;
+  rec.mark(1);
+  const uint16_t* xr = prenorm ? lay.xn : x;
+
+  const float* lg = logits_in;
+  if (!lg) {
+    float* lo = logits_out ? logits_out : lay.logits;
+    logits_kernel<<<dim3(E, (T + 7) / 8), 256, 0, s>>>(xr, w->router_w, T, E, H, lo);
+    if (!launched_ok()) return COLI_ERR_CUDA;
+    lg = lo;
+  } else if (logits_out && logits_out != logits_in) {
+    if (cudaMemcpyAsync(logits_out, logits_in, static_cast<size_t>(T) * E * 4, cudaMemcpyDeviceToDevice, s) !=
+        cudaSuccess)
+      return COLI_ERR_CUDA;
+  }
+  rec.mark(2);
+  int32_t* ids = topk_ids_out ? topk_ids_out : lay.ids;
+  float* tw = topk_w_out ? topk_w_out : lay.w;
+  route_kernel<<<(T + 7) / 8, 256, 0, s>>>(lg, w->router_bias, T, E, k, ids, tw, di.status);
+  if (!launched_ok()) return COLI_ERR_CUDA;
+  rec.mark(3);
+  union_kernel<<<1, kUnionThreads, kUnionWarps * E * 4, s>>>(ids, T * k, E, lay.unique, lay.n_unique, lay.seg_off,
+                                                            lay.perm, lay.pair_pos, di.status);
+  if (!launched_ok()) return COLI_ERR_CUDA;
+  rec.mark(4);
+  return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
+                 di, s, rec);
+}
+
+coli_status coli_moe_get_status(void* stream, uint32_t* flags) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return COLI_ERR_CUDA;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, di.status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return COLI_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(di.status, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess) return COLI_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v == 0) return COLI_OK;
+  if (v == COLI_FLAG_NONFINITE) return COLI_ERR_NONFINITE;
+  return COLI_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+// Route step kernels: optional pre-norm + fragment-ordered copy of the
+// activations, router logits, and the top-k / renormalised-softmax router.
+//
+// Route is the first step of every layer of every token on the Colibri
+// README's per-token path ("Il percorso di ogni token"; getting-started
+// guide, "1. Route": the router decides which experts a token activates).
+#pragma once
+#include "common.cuh"
+
+namespace coli {
+
+constexpr float kRmsEps = 1e-6f;
+
+// One block per token.  Writes the fragment-ordered copy `xq` of the layer's
+// expert input and, with prenorm, the natural-order normalised copy `xn`:
+//   n = bf16( x * (1 / sqrt(mean(x^2) + 1e-6)) ), the sum of squares in fp32
+// in a fixed order.  H % 8 == 0.
+__global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int H, int prenorm,
+                                                   uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
+  const int t = blockIdx.x;
+  const uint16_t* xr = x + static_cast<size_t>(t) * H;
+  __shared__ float red[8];
+  float r = 1.0f;
+  if (prenorm) {
+    float ss = 0.f;
+    for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+      uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
+    r = 1.0f / sqrtf(tot / static_cast<float>(H) + kRmsEps);
+  }
+  for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+    uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+    uint16_t e[8];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      e[2 * q] = static_cast<uint16_t>(w[q] & 0xffffu);
+      e[2 * q + 1] = static_cast<uint16_t>(w[q] >> 16);
+    }
+    if (prenorm) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) e[q] = float_to_bf16_bits(bf16_bits_to_float(e[q]) * r);
+      uint4 o;
+      o.x = e[0] | (static_cast<uint32_t>(e[1]) << 16);
+      o.y = e[2] | (static_cast<uint32_t>(e[3]) << 16);
+      o.z = e[4] | (static_cast<uint32_t>(e[5]) << 16);
+      o.w = e[6] | (static_cast<uint32_t>(e[7]) << 16);
+      *reinterpret_cast<uint4*>(xn + static_cast<size_t>(t) * H + i) = o;
+    }
+    // fragment order x0 x4 x1 x5 x2 x6 x3 x7
+    uint4 o;
+    o.x = e[0] | (static_cast<uint32_t>(e[4]) << 16);
+    o.y = e[1] | (static_cast<uint32_t>(e[5]) << 16);
+    o.z = e[2] | (static_cast<uint32_t>(e[6]) << 16);
+    o.w = e[3] | (static_cast<uint32_t>(e[7]) << 16);
+    *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
+  }
+}
+
+// Router logits l[t,e] = sum_h x[t,h] * W_r[e,h] in fp32.
+// Block = 8 warps for one expert e and up to 8 tokens; warp w covers the
+// H/8 slice [w*H/8, (w+1)*H/8) with float4 loads of W_r; partial sums are
+// reduced in a fixed order (lane tree, then warps 0..7), so every token's
+// logit is computed the same way whatever the batch.  H % 256 == 0.
+__global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
+                                                     int T, int E, int H, float* __restrict__ logits) {
+  const int e = blockIdx.x;
+  const int t0 = blockIdx.y * 8;
+  const int nt = min(8, T - t0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hw = H >> 3;
+  const int h0 = warp * hw, h1 = h0 + hw;
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+  const float* wrow = wr + static_cast<size_t>(e) * H;
+  for (int h = h0 + lane * 4; h < h1; h += 128) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(wrow + h));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < nt) {
+        const uint2 xv = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t0 + q) * H + h);
+        float a = acc[q];
+        a = fmaf(__uint_as_float(xv.x << 16), w.x, a);
+        a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w.y, a);
+        a = fmaf(__uint_as_float(xv.y << 16), w.z, a);
+        a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w.w, a);
+        acc[q] = a;
+      }
+    }
+  }
+  __shared__ float part[8][8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float v = acc[q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) part[warp][q] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
+    logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = s;
+  }
+}
+
+// (value, index) order of the router: larger value first, then lower index.
+__device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+// One warp per token: top-k over E <= 1024 logits (+ bias) and the
+// renormalised softmax weights.  Lane l holds experts l, l+32, ...
+// NaN ranks as -inf; NaN or +inf anywhere, or -inf selected, sets
+// COLI_FLAG_NONFINITE.
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                    int T, int E, int k, int32_t* __restrict__ ids,
+                                                    float* __restrict__ wout, uint32_t* __restrict__ status) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float* lr = logits + static_cast<size_t>(t) * E;
+  float v[32];
+  uint32_t taken = 0;
+  bool bad = false;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const int e = lane + 32 * q;
+    float val = -INFINITY;
+    if (e < E) {
+      val = lr[e];
+      if (bias) val = val + bias[e];
+      if (isnan(val)) {
+        bad = true;
+        val = -INFINITY;
+      } else if (isinf(val) && val > 0.f) {
+        bad = true;
+      }
+    } else {
+      taken |= 1u << q;  // padding never selected
+    }
+    v[q] = val;
+  }
+  float l_max = 0.f, my_v = 0.f;
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = 0.f;
+    int bi = 0x7fffffff;
+    bool have = false;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      if (!(taken & (1u << q))) {
+        const int e = lane + 32 * q;
+        if (!have || route_better(v[q], e, bv, bi)) {
+          bv = v[q];
+          bi = e;
+          have = true;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || route_better(ov, oi, bv, bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (j == 0) l_max = bv;
+    if (lane == j) {
+      my_v = bv;
+      my_id = bi;
+    }
+    if (isinf(bv) && bv < 0.f) bad = true;
+  }
+  // weights: e_j = exp(l_j - l_max), summed in slot order, then normalised
+  const float ej = (lane < k) ? expf(my_v - l_max) : 0.f;
+  float sum = 0.f;
+  for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ej, j);
+  if (lane < k) {
+    ids[static_cast<size_t>(t) * k + lane] = my_id;
+    wout[static_cast<size_t>(t) * k + lane] = ej / sum;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_NONFINITE);
+}
+
+}  // namespace coli

@@ -1,0 +1,128 @@
+"""The C-ABI library loads, exports every symbol include/*.h declares, and its
+host-side argument checks answer before anything is launched.  CPU only: no
+call here reaches a kernel launch."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"\b(coli_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def colimoe():
+    from int4_routed_expert_renorm_b200.build import build
+    build()
+    import int4_routed_expert_renorm_b200 as m
+    return m
+
+
+def test_every_declared_symbol_is_exported(colimoe):
+    lib = ctypes.CDLL(colimoe._lib.LIB_PATH)
+    declared = _declared_functions()
+    assert {"coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer"} <= declared
+    missing = [n for n in sorted(declared) if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(colimoe._lib.EXPORTS) <= declared
+
+
+def test_version_and_status_strings(colimoe):
+    assert colimoe.coli_moe_version() >= 100
+    assert colimoe._lib.status_str(0) == "ok"
+    assert colimoe._lib.status_str(3) == "workspace too small"
+
+
+def _dims(m, **kw):
+    d = dict(hidden=6144, inter=2048, n_experts=256, top_k=8, n_shared=1, group=32)
+    d.update(kw)
+    return m.coli_moe_dims(**d)
+
+
+def test_workspace_bytes(colimoe):
+    m = colimoe
+    d = _dims(m)
+    n1 = m.coli_moe_workspace_bytes(d, 1)
+    n64 = m.coli_moe_workspace_bytes(d, 64)
+    assert 0 < n1 < n64
+    # ypair rows (T*k + S*T) x H fp32 dominate: at least that much
+    assert n64 >= (64 * 8 + 64) * 6144 * 4
+    assert m.coli_moe_workspace_bytes(_dims(m, group=64), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, hidden=6000), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, top_k=300), 4) == 0
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_route_and_union_argument_checks(colimoe):
+    lib = colimoe._lib._lib
+    f = _fake()
+    assert lib.coli_moe_route(f, None, 4, 2000, 8, f, f, None) == colimoe._lib.COLI_ERR_UNSUPPORTED
+    assert lib.coli_moe_route(f, None, 4, 16, 17, f, f, None) == colimoe._lib.COLI_ERR_UNSUPPORTED
+    assert lib.coli_moe_route(None, None, 4, 16, 2, f, f, None) == colimoe._lib.COLI_ERR_INVALID_ARG
+    assert lib.coli_moe_route(f, None, -1, 16, 2, f, f, None) == colimoe._lib.COLI_ERR_INVALID_ARG
+    assert lib.coli_moe_route(None, None, 0, 16, 2, None, None, None) == colimoe._lib.COLI_OK  # T = 0: no-op
+    assert lib.coli_moe_union(f, 4, 2, 2000, f, f, f, f, f, None) == colimoe._lib.COLI_ERR_UNSUPPORTED
+    assert lib.coli_moe_union(f, 1 << 22, 8, 256, f, f, f, f, f, None) == colimoe._lib.COLI_ERR_UNSUPPORTED
+    assert lib.coli_moe_union(f, 4, 2, 16, f, None, f, f, f, None) == colimoe._lib.COLI_ERR_INVALID_ARG
+
+
+def _weights(m, misalign=False):
+    a = 0x100000
+    ptrs = [a + i * 0x1000 for i in range(8)]
+    if misalign:
+        ptrs[0] += 2
+    return m.coli_moe_weights(*[ctypes.c_void_p(p) for p in ptrs])
+
+
+def test_layer_argument_checks(colimoe):
+    m = colimoe
+    lib = m._lib._lib
+    d, w = _dims(m), _weights(m)
+    x, out, ws = _fake(0x200000), _fake(0x300000), _fake(0x400000)
+    need = m.coli_moe_workspace_bytes(d, 4)
+    L = lambda d_, w_, x_, T, ws_, nbytes, flags=0: lib.coli_moe_layer(  # noqa: E731
+        ctypes.byref(d_), ctypes.byref(w_), x_, T, None, None, flags, out, None, None, None, ws_, nbytes, None)
+    assert L(d, w, x, 4, ws, need - 1) == m._lib.COLI_ERR_WORKSPACE
+    assert L(_dims(m, group=64), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, inter=384), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, n_shared=9), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(d, _weights(m, misalign=True), x, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG
+    assert L(d, w, None, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG
+    assert L(d, w, x, 4, _fake(0x400010), need) == m._lib.COLI_ERR_INVALID_ARG   # ws not 256-aligned
+    assert L(d, w, x, -2, ws, need) == m._lib.COLI_ERR_INVALID_ARG
+    assert L(d, w, x, 0, ws, 0) == m._lib.COLI_OK                                # T = 0: no-op
+    nw = m.coli_moe_weights(*[ctypes.c_void_p(0x100000 + i * 0x1000) for i in range(6)], None, None)
+    assert L(d, nw, x, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG              # no router, no logits_in
+
+
+def test_expert_ffn_argument_checks(colimoe):
+    m = colimoe
+    lib = m._lib._lib
+    d, w, f = _dims(m), _weights(m), _fake(0x500000)
+    need = m.coli_moe_workspace_bytes(d, 4)
+    F = lambda T, ws_bytes, x=f, out=_fake(0x600000): lib.coli_moe_expert_ffn(  # noqa: E731
+        ctypes.byref(d), ctypes.byref(w), x, T, f, f, f, f, f, f, f, None, out, 0, _fake(0x700000), ws_bytes, None)
+    assert F(4, need - 256) == m._lib.COLI_ERR_WORKSPACE
+    assert F(4, need, x=_fake(0x600000)) == m._lib.COLI_ERR_INVALID_ARG   # out aliases x
+    assert F(0, 0) == m._lib.COLI_OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from int4_routed_expert_renorm_b200 import _lib
+    with pytest.raises(ImportError):
+        _lib.load(str(tmp_path / "libcolimoe.so"))
