@@ -294,8 +294,10 @@ def main():
 
     # dominant kernel: the gate/up expert FFN (stage 5 -> 6), timed live
     gu_ms = [stage[i][5].elapsed_time(stage[i][6]) for i in range(M)]
-    dn_ms = [stage[i][6].elapsed_time(stage[i][7]) for i in range(M)]
     gu_avg = statistics.mean(gu_ms)
+    stage_names = ["prep", "logits", "route", "union", "plan", "gate_up", "down", "combine"]
+    stage_ms = {n: statistics.mean(stage[i][j].elapsed_time(stage[i][j + 1]) for i in range(M))
+                for j, n in enumerate(stage_names)}
     hbm, tf_burst, tf_sus, src = peaks()
     per_mat = H * I // 2 + (H * I // 32) * 2
     P = T * k
@@ -373,7 +375,7 @@ def main():
                        "union_per_layer": u_stack or None, "l2": "flushed (256 MiB write) before every step",
                        "rotating_batches": NB},
             "int4_bytes_per_step": bytes_step, "int4_gbs": int4_gbs, "int4_frac_of_hbm": int4_gbs / hbm,
-            "roofline": roof, "down_kernel_ms": statistics.mean(dn_ms), "gateup_kernel_ms": gu_avg,
+            "roofline": roof, "stage_ms": stage_ms,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

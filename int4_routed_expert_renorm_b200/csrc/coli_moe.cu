@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "k_ffn_decode.cuh"
@@ -71,14 +72,28 @@ coli_status dev_info(DevInfo* out) {
   }
   if (!g_attr_done[dev]) {
     bool ok = true;
-    ok &= cudaFuncSetAttribute(ffn_decode_kernel<0, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(FfnCfg<0, 256>::SMEM)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(ffn_decode_kernel<1, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(FfnCfg<1, 256>::SMEM)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(ffn_decode_kernel<1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(FfnCfg<1, 128>::SMEM)) == cudaSuccess;
+#define COLI_SET_SMEM(M, KC, NT, SG)                                                                   \
+  ok &= cudaFuncSetAttribute(ffn_decode_kernel<M, KC, NT, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(FfnCfg<M, KC, NT, SG>::SMEM)) == cudaSuccess;
+    COLI_SET_SMEM(0, 256, 1, true)
+    COLI_SET_SMEM(0, 256, 1, false)
+    COLI_SET_SMEM(0, 256, 4, false)
+    COLI_SET_SMEM(1, 256, 1, true)
+    COLI_SET_SMEM(1, 256, 1, false)
+    COLI_SET_SMEM(1, 256, 4, false)
+    COLI_SET_SMEM(1, 128, 1, true)
+    COLI_SET_SMEM(1, 128, 1, false)
+    COLI_SET_SMEM(1, 128, 4, false)
+#undef COLI_SET_SMEM
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
+    const int ru_smem = (kUnionWarps * 1024 + kFusedRouteMaxT * 32) * 4;
+    ok &= cudaFuncSetAttribute(route_union_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(route_union_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(route_union_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(route_union_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(route_union_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(route_union_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
     if (!ok) return COLI_ERR_CUDA;
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
@@ -97,9 +112,23 @@ coli_status dev_info(DevInfo* out) {
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-inline bool launched_ok() {
+// Every kernel is launched with programmatic stream serialization: its CTAs
+// may become resident while the previous kernel drains, and each kernel
+// executes griddepcontrol.wait before touching any input.
+template <typename... KArgs, typename... Args>
+bool launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   ++t_launches;
-  return cudaPeekAtLastError() == cudaSuccess;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess;
 }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -204,14 +233,59 @@ bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K
   return true;
 }
 
-template <int MODE, int KC>
+template <int MODE, int KC, int NT, bool SG>
 bool launch_ffn(const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& s0, const CUtensorMap& s1,
                 const FfnArgs& a, int grid, cudaStream_t st) {
-  ffn_decode_kernel<MODE, KC><<<grid, kFfnThreads, FfnCfg<MODE, KC>::SMEM, st>>>(q0, q1, s0, s1, a);
-  return launched_ok();
+  return launch(ffn_decode_kernel<MODE, KC, NT, SG>, dim3(grid), dim3(kFfnThreads), FfnCfg<MODE, KC, NT, SG>::SMEM,
+                st, q0, q1, s0, s1, a);
 }
 
-// The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer.
+// Decode-form variant for this batch: one token per tile when T == 1, 8-token
+// tiles while T <= 8, else 32-token tiles.
+template <int MODE, int KC>
+bool launch_ffn_for(int T, const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& s0,
+                    const CUtensorMap& s1, const FfnArgs& a, int grid, cudaStream_t st) {
+  if (T == 1) return launch_ffn<MODE, KC, 1, true>(q0, q1, s0, s1, a, grid, st);
+  if (T <= 8) return launch_ffn<MODE, KC, 1, false>(q0, q1, s0, s1, a, grid, st);
+  return launch_ffn<MODE, KC, 4, false>(q0, q1, s0, s1, a, grid, st);
+}
+
+inline int tok_block(int T) { return T <= 8 ? 8 : 32; }
+
+bool launch_route(const float* lg, const float* bias, int T, int E, int k, int32_t* ids, float* w, uint32_t* status,
+                  cudaStream_t st) {
+  const dim3 g((T + 7) / 8), b(256);
+  switch (route_nv(E)) {
+    case 1: return launch(route_kernel<1>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+    case 2: return launch(route_kernel<2>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+    case 4: return launch(route_kernel<4>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+    case 8: return launch(route_kernel<8>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+    case 16: return launch(route_kernel<16>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+    default: return launch(route_kernel<32>, g, b, 0, st, lg, bias, T, E, k, ids, w, status);
+  }
+}
+
+// Route + union + plan in one CTA (T <= kFusedRouteMaxT).
+bool launch_route_union(const float* lg, const float* bias, int T, int E, int k, int S, int tokb, int32_t* ids,
+                        float* w, const Ws& ws, uint32_t* status, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kUnionWarps * E + T * k) * 4;
+  const dim3 g(1), b(kUnionThreads);
+#define COLI_RU(NV)                                                                                            \
+  launch(route_union_kernel<NV>, g, b, smem, st, lg, bias, T, E, k, ids, w, ws.unique, ws.n_unique, ws.seg_off, \
+         ws.perm, ws.pair_pos, status, S, tokb, ws.plan)
+  switch (route_nv(E)) {
+    case 1: return COLI_RU(1);
+    case 2: return COLI_RU(2);
+    case 4: return COLI_RU(4);
+    case 8: return COLI_RU(8);
+    case 16: return COLI_RU(16);
+    default: return COLI_RU(32);
+  }
+#undef COLI_RU
+}
+
+// The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer;
+// the tile plan (ws.plan) must already be on the stream.
 coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
                     const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
                     const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
@@ -220,14 +294,11 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   const int P = T * k;
   const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
   const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
-
-  plan_kernel<<<1, 1024, 0, st>>>(n_unique, seg_off, T, S, ws.plan);
-  if (!launched_ok()) return COLI_ERR_CUDA;
-  rec.mark(5);
+  const int tokb = tok_block(T);
 
   // upper bound on tiles: every segment contributes ceil(cnt/64) <= cnt/64 + 1 blocks
   const int Umax = P < E ? P : E;
-  const long blocks_ub = static_cast<long>(Umax) + P / kTokBlock + static_cast<long>(S) * ((T + kTokBlock - 1) / kTokBlock);
+  const long blocks_ub = static_cast<long>(Umax) + P / tokb + static_cast<long>(S) * ((T + tokb - 1) / tokb);
 
   CUtensorMap gq, uq, gs, us, dq, ds;
   const int kc_dn = (I % 256 == 0) ? 256 : 128;
@@ -259,7 +330,7 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   {
     const long tiles = blocks_ub * (I / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    if (!launch_ffn<0, 256>(gq, uq, gs, us, a, grid, st)) return COLI_ERR_CUDA;
+    if (!launch_ffn_for<0, 256>(T, gq, uq, gs, us, a, grid, st)) return COLI_ERR_CUDA;
   }
   rec.mark(6);
   // down -> y per (pair, row)
@@ -273,8 +344,8 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   {
     const long tiles = blocks_ub * (H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    const bool ok = kc_dn == 256 ? launch_ffn<1, 256>(dq, dq, ds, ds, a, grid, st)
-                                 : launch_ffn<1, 128>(dq, dq, ds, ds, a, grid, st);
+    const bool ok = kc_dn == 256 ? launch_ffn_for<1, 256>(T, dq, dq, ds, ds, a, grid, st)
+                                 : launch_ffn_for<1, 128>(T, dq, dq, ds, ds, a, grid, st);
     if (!ok) return COLI_ERR_CUDA;
   }
   rec.mark(7);
@@ -283,8 +354,9 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
     const long work = static_cast<long>(T) * (H / 4);
     long blocks = (work + 255) / 256;
     if (blocks > 4L * di.sms) blocks = 4L * di.sms;
-    combine_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(ws.ypair, pair_pos, topk_w, residual, T, k, S, H, out);
-    if (!launched_ok()) return COLI_ERR_CUDA;
+    if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
+                pair_pos, topk_w, residual, T, k, S, H, out))
+      return COLI_ERR_CUDA;
   }
   rec.mark(8);
   return COLI_OK;
@@ -335,8 +407,8 @@ coli_status coli_moe_route(const float* logits, const float* bias, int T, int E,
   if (!logits || !topk_ids || !topk_w) return COLI_ERR_INVALID_ARG;
   DevInfo di;
   if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
-  route_kernel<<<(T + 7) / 8, 256, 0, as_stream(stream)>>>(logits, bias, T, E, k, topk_ids, topk_w, di.status);
-  return launched_ok() ? COLI_OK : COLI_ERR_CUDA;
+  return launch_route(logits, bias, T, E, k, topk_ids, topk_w, di.status, as_stream(stream)) ? COLI_OK
+                                                                                           : COLI_ERR_CUDA;
 }
 
 coli_status coli_moe_union(const int32_t* topk_ids, int T, int k, int E, int32_t* unique_ids, int32_t* n_unique,
@@ -347,9 +419,11 @@ coli_status coli_moe_union(const int32_t* topk_ids, int T, int k, int E, int32_t
   if (T > 0 && (!topk_ids || !unique_ids || !perm || !pair_pos)) return COLI_ERR_INVALID_ARG;
   DevInfo di;
   if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
-  union_kernel<<<1, kUnionThreads, kUnionWarps * E * 4, as_stream(stream)>>>(topk_ids, T * k, E, unique_ids, n_unique,
-                                                                             seg_off, perm, pair_pos, di.status);
-  return launched_ok() ? COLI_OK : COLI_ERR_CUDA;
+  return launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4,
+                as_stream(stream), topk_ids, T * k, E, unique_ids, n_unique, seg_off, perm, pair_pos, di.status, T, 0, 8,
+                static_cast<int32_t*>(nullptr))
+             ? COLI_OK
+             : COLI_ERR_CUDA;
 }
 
 coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
@@ -376,9 +450,12 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   cudaStream_t s = as_stream(stream);
   const StageRecorder rec(s);
   rec.mark(0);
-  prep_kernel<<<T, 256, 0, s>>>(x, dims->hidden, 0, nullptr, lay.xq);
-  if (!launched_ok()) return COLI_ERR_CUDA;
+  if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq))
+    return COLI_ERR_CUDA;
   rec.mark_through(1, 4);
+  if (!launch(plan_kernel, dim3(1), dim3(1024), 0, s, n_unique, seg_off, T, dims->n_shared, tok_block(T), lay.plan))
+    return COLI_ERR_CUDA;
+  rec.mark(5);
   return run_ffn(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di, s, rec);
 }
 
@@ -406,33 +483,51 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   const bool prenorm = (flags & COLI_LAYER_PRENORM) != 0;
   const StageRecorder rec(s);
   rec.mark(0);
+  const int S = dims->n_shared, tokb = tok_block(T);
 
-  prep_kernel<<<T, 256, 0, s>>>(x, H, prenorm ? 1 : 0, lay.xn, lay.xq);
-  if (!launched_ok()) return COLI_ERR_CUDA;
-  rec.mark(1);
-  const uint16_t* xr = prenorm ? lay.xn : x;
-
+  // 1. expert input (fragment order, optional pre-norm) and router logits
+  float* lo = logits_out ? logits_out : lay.logits;
   const float* lg = logits_in;
-  if (!lg) {
-    float* lo = logits_out ? logits_out : lay.logits;
-    logits_kernel<<<dim3(E, (T + 7) / 8), 256, 0, s>>>(xr, w->router_w, T, E, H, lo);
-    if (!launched_ok()) return COLI_ERR_CUDA;
-    lg = lo;
-  } else if (logits_out && logits_out != logits_in) {
+  const bool fused_front = T <= (prenorm ? 8 : 64);
+  if (fused_front) {
+    const float* wr = logits_in ? nullptr : w->router_w;
+    const int grid = logits_in ? T : E;
+    if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq))
+      return COLI_ERR_CUDA;
+    rec.mark_through(1, 2);
+    if (!logits_in) lg = lo;
+  } else {
+    if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, H, prenorm ? 1 : 0, lay.xn, lay.xq)) return COLI_ERR_CUDA;
+    rec.mark(1);
+    if (!logits_in) {
+      const uint16_t* xr = prenorm ? lay.xn : x;
+      if (!launch(logits_kernel, dim3(E, (T + 7) / 8), dim3(256), 0, s, xr, w->router_w, T, E, H, lo))
+        return COLI_ERR_CUDA;
+      lg = lo;
+    }
+    rec.mark(2);
+  }
+  if (logits_in && logits_out && logits_out != logits_in) {
     if (cudaMemcpyAsync(logits_out, logits_in, static_cast<size_t>(T) * E * 4, cudaMemcpyDeviceToDevice, s) !=
         cudaSuccess)
       return COLI_ERR_CUDA;
   }
-  rec.mark(2);
+  // 2. route, union and the FFN tile plan
   int32_t* ids = topk_ids_out ? topk_ids_out : lay.ids;
   float* tw = topk_w_out ? topk_w_out : lay.w;
-  route_kernel<<<(T + 7) / 8, 256, 0, s>>>(lg, w->router_bias, T, E, k, ids, tw, di.status);
-  if (!launched_ok()) return COLI_ERR_CUDA;
-  rec.mark(3);
-  union_kernel<<<1, kUnionThreads, kUnionWarps * E * 4, s>>>(ids, T * k, E, lay.unique, lay.n_unique, lay.seg_off,
-                                                            lay.perm, lay.pair_pos, di.status);
-  if (!launched_ok()) return COLI_ERR_CUDA;
-  rec.mark(4);
+  if (T <= kFusedRouteMaxT) {
+    if (!launch_route_union(lg, w->router_bias, T, E, k, S, tokb, ids, tw, lay, di.status, s)) return COLI_ERR_CUDA;
+    rec.mark_through(3, 5);
+  } else {
+    if (!launch_route(lg, w->router_bias, T, E, k, ids, tw, di.status, s)) return COLI_ERR_CUDA;
+    rec.mark(3);
+    if (!launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4, s,
+                static_cast<const int32_t*>(ids), T * k, E, lay.unique, lay.n_unique, lay.seg_off, lay.perm,
+                lay.pair_pos, di.status, T, S, tokb, lay.plan))
+      return COLI_ERR_CUDA;
+    rec.mark_through(4, 5);
+  }
+  // 3. expert FFN and combine
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
                  di, s, rec);
 }

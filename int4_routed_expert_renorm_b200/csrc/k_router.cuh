@@ -17,6 +17,8 @@ constexpr float kRmsEps = 1e-6f;
 // in a fixed order.  H % 8 == 0.
 __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int H, int prenorm,
                                                    uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const uint16_t* xr = x + static_cast<size_t>(t) * H;
   __shared__ float red[8];
@@ -77,6 +79,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
 // logit is computed the same way whatever the batch.  H % 256 == 0.
 __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                                                      int T, int E, int H, float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   const int t0 = blockIdx.y * 8;
   const int nt = min(8, T - t0);
@@ -119,27 +123,153 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
   }
 }
 
+// Small-batch front end (T <= 64): router logits as in logits_kernel, plus
+// the fragment-ordered copy of the expert input written by the blocks whose
+// index matches a token (block b writes tokens b, b + gridDim.x, ...).  With
+// prenorm every block normalises its tokens itself (n = bf16(x * r) with
+// r = 1/sqrt(mean(x^2) + 1e-6) summed in the same order as prep_kernel), so
+// the logits see exactly the normalised input the experts see.
+__device__ __forceinline__ float token_rms_scale(const uint16_t* __restrict__ xr, int H, float* red) {
+  float ss = 0.f;
+  for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
+      ss = fmaf(a, a, ss);
+      ss = fmaf(b, b, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+  return 1.0f / sqrtf(tot / static_cast<float>(H) + kRmsEps);
+}
+
+__global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
+                                                    int T, int E, int H, int prenorm, float* __restrict__ logits,
+                                                    uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[8];
+  __shared__ float rs[64];
+  const int e = blockIdx.x;
+  if (prenorm) {
+    for (int t = 0; t < T; ++t) {
+      const float r = token_rms_scale(x + static_cast<size_t>(t) * H, H, red);
+      if (threadIdx.x == 0) rs[t] = r;
+    }
+    __syncthreads();
+  }
+  // fragment-ordered (and normalised) copies of this block's tokens
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint16_t* xr = x + static_cast<size_t>(t) * H;
+    const float r = prenorm ? rs[t] : 1.0f;
+    for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+      uint16_t q8[8];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        q8[2 * q] = static_cast<uint16_t>(wv[q] & 0xffffu);
+        q8[2 * q + 1] = static_cast<uint16_t>(wv[q] >> 16);
+      }
+      if (prenorm) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) q8[q] = float_to_bf16_bits(bf16_bits_to_float(q8[q]) * r);
+        uint4 o;
+        o.x = q8[0] | (static_cast<uint32_t>(q8[1]) << 16);
+        o.y = q8[2] | (static_cast<uint32_t>(q8[3]) << 16);
+        o.z = q8[4] | (static_cast<uint32_t>(q8[5]) << 16);
+        o.w = q8[6] | (static_cast<uint32_t>(q8[7]) << 16);
+        *reinterpret_cast<uint4*>(xn + static_cast<size_t>(t) * H + i) = o;
+      }
+      uint4 o;
+      o.x = q8[0] | (static_cast<uint32_t>(q8[4]) << 16);
+      o.y = q8[1] | (static_cast<uint32_t>(q8[5]) << 16);
+      o.z = q8[2] | (static_cast<uint32_t>(q8[6]) << 16);
+      o.w = q8[3] | (static_cast<uint32_t>(q8[7]) << 16);
+      *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
+    }
+  }
+  if (!wr) return;
+  // logits of expert e for every token, 8 tokens at a time
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hw = H >> 3;
+  const int h0 = warp * hw, h1 = h0 + hw;
+  const float* wrow = wr + static_cast<size_t>(e) * H;
+  __shared__ float part[8][8];
+  for (int t0 = 0; t0 < T; t0 += 8) {
+    const int nt = min(8, T - t0);
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int h = h0 + lane * 4; h < h1; h += 128) {
+      const float4 w = __ldg(reinterpret_cast<const float4*>(wrow + h));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < nt) {
+          const uint2 xv = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t0 + q) * H + h);
+          float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+          float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+          if (prenorm) {
+            const float r = rs[t0 + q];
+            x0 = bf16_bits_to_float(float_to_bf16_bits(x0 * r));
+            x1 = bf16_bits_to_float(float_to_bf16_bits(x1 * r));
+            x2 = bf16_bits_to_float(float_to_bf16_bits(x2 * r));
+            x3 = bf16_bits_to_float(float_to_bf16_bits(x3 * r));
+          }
+          float a = acc[q];
+          a = fmaf(x0, w.x, a);
+          a = fmaf(x1, w.y, a);
+          a = fmaf(x2, w.z, a);
+          a = fmaf(x3, w.w, a);
+          acc[q] = a;
+        }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float v = acc[q];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) part[warp][q] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < nt) {
+      float sacc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sacc += part[w][threadIdx.x];
+      logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = sacc;
+    }
+  }
+}
+
 // (value, index) order of the router: larger value first, then lower index.
 __device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// One warp per token: top-k over E <= 1024 logits (+ bias) and the
-// renormalised softmax weights.  Lane l holds experts l, l+32, ...
-// NaN ranks as -inf; NaN or +inf anywhere, or -inf selected, sets
-// COLI_FLAG_NONFINITE.
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                                                    int T, int E, int k, int32_t* __restrict__ ids,
-                                                    float* __restrict__ wout, uint32_t* __restrict__ status) {
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  const float* lr = logits + static_cast<size_t>(t) * E;
-  float v[32];
+// Route one token with one warp: top-k over E <= 32*NV logits (+ bias) and
+// the renormalised softmax weights.  Lane l holds experts l, l+32, ...
+// Slot j receives the j-th expert in (value desc, index asc) order and
+// w_j = exp(l_j - l_max) / sum_{i<k} exp(l_i - l_max), summed in slot order.
+// NaN ranks as -inf; NaN or +inf anywhere, or a selected -inf, returns bad.
+// Lane j < k gets slot j in *id / *w.
+template <int NV>
+__device__ __forceinline__ bool route_token(const float* __restrict__ lr, const float* __restrict__ bias, int E,
+                                            int k, int lane, int* id, float* w) {
+  float v[NV];
   uint32_t taken = 0;
   bool bad = false;
 #pragma unroll
-  for (int q = 0; q < 32; ++q) {
+  for (int q = 0; q < NV; ++q) {
     const int e = lane + 32 * q;
     float val = -INFINITY;
     if (e < E) {
@@ -161,15 +291,13 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   for (int j = 0; j < k; ++j) {
     float bv = 0.f;
     int bi = 0x7fffffff;
-    bool have = false;
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
+    for (int q = 0; q < NV; ++q) {
       if (!(taken & (1u << q))) {
         const int e = lane + 32 * q;
-        if (!have || route_better(v[q], e, bv, bi)) {
+        if (bi == 0x7fffffff || route_better(v[q], e, bv, bi)) {
           bv = v[q];
           bi = e;
-          have = true;
         }
       }
     }
@@ -190,15 +318,38 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     }
     if (isinf(bv) && bv < 0.f) bad = true;
   }
-  // weights: e_j = exp(l_j - l_max), summed in slot order, then normalised
   const float ej = (lane < k) ? expf(my_v - l_max) : 0.f;
   float sum = 0.f;
   for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ej, j);
+  *id = my_id;
+  *w = ej / sum;
+  return __any_sync(0xffffffffu, bad);
+}
+
+// One warp per token over the whole batch (any T).
+template <int NV>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                    int T, int E, int k, int32_t* __restrict__ ids,
+                                                    float* __restrict__ wout, uint32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int id;
+  float w;
+  const bool bad = route_token<NV>(logits + static_cast<size_t>(t) * E, bias, E, k, lane, &id, &w);
   if (lane < k) {
-    ids[static_cast<size_t>(t) * k + lane] = my_id;
-    wout[static_cast<size_t>(t) * k + lane] = ej / sum;
+    ids[static_cast<size_t>(t) * k + lane] = id;
+    wout[static_cast<size_t>(t) * k + lane] = w;
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_NONFINITE);
+  if (bad && lane == 0) atomicOr(status, COLI_FLAG_NONFINITE);
+}
+
+// Values per lane needed for E experts (E <= 1024).
+inline int route_nv(int E) {
+  const int nv = (E + 31) / 32;
+  return nv <= 1 ? 1 : nv <= 2 ? 2 : nv <= 4 ? 4 : nv <= 8 ? 8 : nv <= 16 ? 16 : 32;
 }
 
 }  // namespace coli

@@ -165,7 +165,10 @@ DECODE_B1 = LayerShape("glm52_layer_decode_b1", 6144, 2048, 256, 8, 1, 1)
 DECODE_B64 = LayerShape("glm52_layer_decode_b64_zipf", 6144, 2048, 256, 8, 1, 64, zipf_bias=True)
 PREFILL_4096 = LayerShape("glm52_layer_prefill_4096", 6144, 2048, 256, 8, 1, 4096, logits_in=True)
 STACK16_B4 = LayerShape("glm52_stack16_decode_b4", 6144, 2048, 256, 8, 1, 4, layers=16, prenorm=True)
-WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4)}
+# Same per-step bytes as DECODE_B1 (8 routed + 1 shared expert, 191 MB > L2) with
+# only 16 routed experts resident: small enough for profiler captures.
+DECODE_B1_E16 = LayerShape("glm52_layer_decode_b1_e16", 6144, 2048, 16, 8, 1, 1)
+WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16)}
 
 
 class LayerInputs:
