@@ -72,18 +72,15 @@ coli_status dev_info(DevInfo* out) {
   }
   if (!g_attr_done[dev]) {
     bool ok = true;
-#define COLI_SET_SMEM(M, KC, NT, SG)                                                                   \
-  ok &= cudaFuncSetAttribute(ffn_decode_kernel<M, KC, NT, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(FfnCfg<M, KC, NT, SG>::SMEM)) == cudaSuccess;
-    COLI_SET_SMEM(0, 256, 1, true)
-    COLI_SET_SMEM(0, 256, 1, false)
-    COLI_SET_SMEM(0, 256, 4, false)
-    COLI_SET_SMEM(1, 256, 1, true)
-    COLI_SET_SMEM(1, 256, 1, false)
-    COLI_SET_SMEM(1, 256, 4, false)
-    COLI_SET_SMEM(1, 128, 1, true)
-    COLI_SET_SMEM(1, 128, 1, false)
-    COLI_SET_SMEM(1, 128, 4, false)
+#define COLI_SET_SMEM(NT, SG, KCD)                                                                   \
+  ok &= cudaFuncSetAttribute(ffn_fused_kernel<NT, SG, KCD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(FusedCfg<NT, KCD>::SMEM)) == cudaSuccess;
+    COLI_SET_SMEM(1, true, 256)
+    COLI_SET_SMEM(1, false, 256)
+    COLI_SET_SMEM(4, false, 256)
+    COLI_SET_SMEM(1, true, 128)
+    COLI_SET_SMEM(1, false, 128)
+    COLI_SET_SMEM(4, false, 128)
 #undef COLI_SET_SMEM
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
@@ -171,6 +168,8 @@ struct Ws {
   int32_t* perm;     // [P]
   int32_t* pair_pos; // [P]
   int32_t* plan;     // [min(E,P)+S+3]
+  int32_t* tb_done;  // [token blocks upper bound] gate/up completion per token block
+  int32_t* rb_done;  // [H/128] down completion per output row block
   uint16_t* hq;      // [P+S*T][I]
   float* ypair;      // [P+S*T][H]
   size_t bytes;
@@ -200,6 +199,12 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
   ws.perm = static_cast<int32_t*>(take(P * 4));
   ws.pair_pos = static_cast<int32_t*>(take(P * 4));
   ws.plan = static_cast<int32_t*>(take((Umax + S + 3) * 4));
+  {
+    const size_t tokb = T <= 8 ? 8 : 32;
+    const size_t blocks_ub = Umax + P / tokb + S * ((static_cast<size_t>(T) + tokb - 1) / tokb);
+    ws.tb_done = static_cast<int32_t*>(take(blocks_ub * 4));
+    ws.rb_done = static_cast<int32_t*>(take(H / 128 * 4));
+  }
   ws.hq = static_cast<uint16_t*>(take(rows * I * 2));
   ws.ypair = static_cast<float*>(take(rows * H * 4));
   ws.bytes = o;
@@ -233,21 +238,40 @@ bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K
   return true;
 }
 
-template <int MODE, int KC, int NT, bool SG>
-bool launch_ffn(const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& s0, const CUtensorMap& s1,
-                const FfnArgs& a, int grid, cudaStream_t st) {
-  return launch(ffn_decode_kernel<MODE, KC, NT, SG>, dim3(grid), dim3(kFfnThreads), FfnCfg<MODE, KC, NT, SG>::SMEM,
-                st, q0, q1, s0, s1, a);
+// The persistent FFN kernel is launched cooperatively (all CTAs resident, so
+// the counter waits of down tiles on gate/up tiles always make progress).
+template <int NT, bool SG, int KCD>
+bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFfnThreads);
+  cfg.dynamicSmemBytes = FusedCfg<NT, KCD>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  ++t_launches;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+  if (e != cudaSuccess) {
+    // without overlap with the previous kernel
+    cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+  }
+  return e == cudaSuccess;
 }
 
 // Decode-form variant for this batch: one token per tile when T == 1, 8-token
 // tiles while T <= 8, else 32-token tiles.
-template <int MODE, int KC>
-bool launch_ffn_for(int T, const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& s0,
-                    const CUtensorMap& s1, const FfnArgs& a, int grid, cudaStream_t st) {
-  if (T == 1) return launch_ffn<MODE, KC, 1, true>(q0, q1, s0, s1, a, grid, st);
-  if (T <= 8) return launch_ffn<MODE, KC, 1, false>(q0, q1, s0, s1, a, grid, st);
-  return launch_ffn<MODE, KC, 4, false>(q0, q1, s0, s1, a, grid, st);
+template <int KCD>
+bool launch_ffn_for(int T, const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
+  if (T == 1) return launch_ffn_fused<1, true, KCD>(m, a, grid, st);
+  if (T <= 8) return launch_ffn_fused<1, false, KCD>(m, a, grid, st);
+  return launch_ffn_fused<4, false, KCD>(m, a, grid, st);
 }
 
 inline int tok_block(int T) { return T <= 8 ? 8 : 32; }
@@ -266,13 +290,13 @@ bool launch_route(const float* lg, const float* bias, int T, int E, int k, int32
 }
 
 // Route + union + plan in one CTA (T <= kFusedRouteMaxT).
-bool launch_route_union(const float* lg, const float* bias, int T, int E, int k, int S, int tokb, int32_t* ids,
-                        float* w, const Ws& ws, uint32_t* status, cudaStream_t st) {
+bool launch_route_union(const float* lg, const float* bias, int T, int E, int k, int S, int tokb, int n_rb,
+                        int32_t* ids, float* w, const Ws& ws, uint32_t* status, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kUnionWarps * E + T * k) * 4;
   const dim3 g(1), b(kUnionThreads);
 #define COLI_RU(NV)                                                                                            \
   launch(route_union_kernel<NV>, g, b, smem, st, lg, bias, T, E, k, ids, w, ws.unique, ws.n_unique, ws.seg_off, \
-         ws.perm, ws.pair_pos, status, S, tokb, ws.plan)
+         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb)
   switch (route_nv(E)) {
     case 1: return COLI_RU(1);
     case 2: return COLI_RU(2);
@@ -300,57 +324,47 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   const int Umax = P < E ? P : E;
   const long blocks_ub = static_cast<long>(Umax) + P / tokb + static_cast<long>(S) * ((T + tokb - 1) / tokb);
 
-  CUtensorMap gq, uq, gs, us, dq, ds;
+  CUtensorMap maps[6];   // gate q, up q, gate s, up s, down q, down s
   const int kc_dn = (I % 256 == 0) ? 256 : 128;
-  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, &gq, &gs) ||
-      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, &uq, &us) ||
-      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, &dq, &ds))
+  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, &maps[0], &maps[2]) ||
+      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, &maps[1], &maps[3]) ||
+      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, &maps[4], &maps[5]))
     return COLI_ERR_CUDA;
 
   FfnArgs a{};
+  a.xq = ws.xq;
+  a.hq = ws.hq;
+  a.ypair = ws.ypair;
+  a.gate_s = w->gate_s;
+  a.up_s = w->up_s;
+  a.down_s = w->down_s;
   a.unique_ids = unique;
   a.n_unique = n_unique;
   a.seg_off = seg_off;
   a.perm = perm;
   a.plan = ws.plan;
+  a.tb_done = ws.tb_done;
+  a.rb_done = ws.rb_done;
+  a.pair_pos = pair_pos;
+  a.topk_w = topk_w;
+  a.residual = residual;
+  a.out = out;
   a.status = di.status;
+  a.H = H;
+  a.I = I;
   a.T = T;
   a.k = k;
   a.E = E;
+  a.S = S;
   a.P = P;
-
-  // gate/up + SiLU*mul -> h
-  a.bsrc = ws.xq;
-  a.scales0 = w->gate_s;
-  a.scales1 = w->up_s;
-  a.hq = ws.hq;
-  a.ypair = nullptr;
-  a.K = H;
-  a.R = I;
   {
-    const long tiles = blocks_ub * (I / kRowBlock);
+    const long tiles = blocks_ub * (I / kRowBlock + H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    if (!launch_ffn_for<0, 256>(T, gq, uq, gs, us, a, grid, st)) return COLI_ERR_CUDA;
-  }
-  rec.mark(6);
-  // down -> y per (pair, row)
-  a.bsrc = ws.hq;
-  a.scales0 = w->down_s;
-  a.scales1 = w->down_s;
-  a.hq = nullptr;
-  a.ypair = ws.ypair;
-  a.K = I;
-  a.R = H;
-  {
-    const long tiles = blocks_ub * (H / kRowBlock);
-    const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    const bool ok = kc_dn == 256 ? launch_ffn_for<1, 256>(T, dq, dq, ds, ds, a, grid, st)
-                                 : launch_ffn_for<1, 128>(T, dq, dq, ds, ds, a, grid, st);
+    const bool ok = kc_dn == 256 ? launch_ffn_for<256>(T, maps, a, grid, st) : launch_ffn_for<128>(T, maps, a, grid, st);
     if (!ok) return COLI_ERR_CUDA;
   }
-  rec.mark(7);
-  // combine
-  {
+  rec.mark_through(6, 7);
+  if (T > kFusedCombineMaxT) {
     const long work = static_cast<long>(T) * (H / 4);
     long blocks = (work + 255) / 256;
     if (blocks > 4L * di.sms) blocks = 4L * di.sms;
@@ -421,7 +435,7 @@ coli_status coli_moe_union(const int32_t* topk_ids, int T, int k, int E, int32_t
   if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
   return launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4,
                 as_stream(stream), topk_ids, T * k, E, unique_ids, n_unique, seg_off, perm, pair_pos, di.status, T, 0, 8,
-                static_cast<int32_t*>(nullptr))
+                static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr), 0)
              ? COLI_OK
              : COLI_ERR_CUDA;
 }
@@ -453,7 +467,8 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq))
     return COLI_ERR_CUDA;
   rec.mark_through(1, 4);
-  if (!launch(plan_kernel, dim3(1), dim3(1024), 0, s, n_unique, seg_off, T, dims->n_shared, tok_block(T), lay.plan))
+  if (!launch(plan_kernel, dim3(1), dim3(1024), 0, s, n_unique, seg_off, T, dims->n_shared, tok_block(T), lay.plan,
+              lay.tb_done, lay.rb_done, dims->hidden / kRowBlock))
     return COLI_ERR_CUDA;
   rec.mark(5);
   return run_ffn(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di, s, rec);
@@ -516,14 +531,15 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   int32_t* ids = topk_ids_out ? topk_ids_out : lay.ids;
   float* tw = topk_w_out ? topk_w_out : lay.w;
   if (T <= kFusedRouteMaxT) {
-    if (!launch_route_union(lg, w->router_bias, T, E, k, S, tokb, ids, tw, lay, di.status, s)) return COLI_ERR_CUDA;
+    if (!launch_route_union(lg, w->router_bias, T, E, k, S, tokb, H / kRowBlock, ids, tw, lay, di.status, s))
+      return COLI_ERR_CUDA;
     rec.mark_through(3, 5);
   } else {
     if (!launch_route(lg, w->router_bias, T, E, k, ids, tw, di.status, s)) return COLI_ERR_CUDA;
     rec.mark(3);
     if (!launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4, s,
                 static_cast<const int32_t*>(ids), T * k, E, lay.unique, lay.n_unique, lay.seg_off, lay.perm,
-                lay.pair_pos, di.status, T, S, tokb, lay.plan))
+                lay.pair_pos, di.status, T, S, tokb, lay.plan, lay.tb_done, lay.rb_done, H / kRowBlock))
       return COLI_ERR_CUDA;
     rec.mark_through(4, 5);
   }

@@ -3,26 +3,34 @@
 // The routed experts are int4 (Colibri README, "L'idea": ~19 MB per expert in
 // the int4 container; an expert's three matrices are the gate, up and down
 // projections of a SwiGLU FFN).  With few tokens per expert the step is bound
-// by reading the int4 weights, so this form streams them once at HBM rate:
-//   * a persistent CTA per SM walks (segment, token block, 128-row block)
-//     tiles of the device-side plan; one producer warp moves, per stage,
-//     128 rows x 256 K of codes (2-D tensor-map copies, 128B swizzle), their
-//     fp16 scales, and the stage's slice of each token's activation row
-//     (1-D bulk copies) into a ring of shared-memory stages;
+// by reading the int4 weights, so this form streams them once at HBM rate in
+// ONE persistent, cooperatively launched kernel (one CTA per SM):
+//   * tiles are (segment, token block, 128-row block); every CTA first walks
+//     its gate/up tiles, then its down tiles, so all CTAs stream weights
+//     without a gap between the two projections;
+//   * one producer warp moves, per stage, 128 rows x 256 K of codes (2-D
+//     tensor-map copies, 128B swizzle), their fp16 scales and the stage's
+//     slice of each token's activation row (1-D bulk copies) into a ring of
+//     shared-memory stages;
+//   * a down tile needs h of its token block from all gate/up row blocks: the
+//     gate/up epilogue publishes each finished (token block, row block) with
+//     a fence and an atomic increment; the down producer issues its weight
+//     copies at once and waits (bounded) on that counter only before copying
+//     the h rows;
 //   * 16 consumer warps: warps w and w+8 own the same 16 rows and split every
-//     stage's 32-wide groups between them (first and second half), so each SM
-//     sub-partition has four warps to hide latency; they sum their partial
-//     accumulators once per tile, in a fixed order;
+//     stage's 32-wide groups between them; they add their partials once per
+//     tile, in a fixed order;
 //   * dequantisation of a pair of codes is one mask-and-magic LOP3 (nibble n
-//     of two's-complement code q becomes the bf16 value 128 + (n ^ 8) =
-//     136 + q) and one exact bf16x2 subtract of 136 (on the FMA pipe, which
-//     the rest of the loop leaves idle); m16n8k16 bf16 mma.sync multiplies the
-//     codes with up to 8 tokens per n-tile; each 32-wide group's fp32 partial
-//     is multiplied by its fp16 scale and accumulated in fp32.
-// Mode 0 runs gate and up together and writes h = bf16(silu(g) * u); mode 1
-// runs down and writes y (fp32) per (pair, row).  combine_kernel then sums each
-// token's k routed y's with its routing weights, its shared experts and its
-// residual in a fixed order and rounds once to bf16.
+//     of the two's-complement code q becomes the bf16 value 128 + (n ^ 8) =
+//     136 + q) and one exact bf16x2 subtract of 136; m16n8k16 bf16 mma.sync
+//     multiplies the codes with up to 8 tokens per n-tile; each 32-wide
+//     group's fp32 partial is multiplied by its fp16 scale and accumulated in
+//     fp32.
+// Gate/up writes h = bf16(silu(g) * u); down writes y (fp32) per (pair, row).
+// The combine (each token's k routed y's with its routing weights, its shared
+// experts and its residual, summed in a fixed order and rounded once to bf16)
+// is done by the last down warp to finish a row block when T <= 4, and by
+// combine_kernel otherwise.
 #pragma once
 #include "common.cuh"
 #include "k_union.cuh"
@@ -33,50 +41,61 @@ constexpr int kRowWarps = 8;                         // 16-row slices per tile
 constexpr int kFfnConsumerWarps = 2 * kRowWarps;     // two K-halves per slice
 constexpr int kFfnThreads = (kFfnConsumerWarps + 1) * 32;
 constexpr int kRowBlock = 16 * kRowWarps;            // 128 rows per tile
+constexpr int kMaxSeg = 1024 + 8;                    // unique routed + shared segments
+constexpr int kFusedCombineMaxT = 4;
 
 struct FfnArgs {
-  const uint16_t* bsrc;      // mode 0: fragment-ordered x [T][K]; mode 1: h [P+S*T][K]
-  const uint16_t* scales0;   // 1-D scale copies when a stage spans all of K
-  const uint16_t* scales1;
+  const uint16_t* xq;        // fragment-ordered expert input [T][H]
+  uint16_t* hq;              // h, fragment-ordered [P+S*T][I]
+  float* ypair;              // y [P+S*T][H]
+  const uint16_t* gate_s;    // scales for 1-D copies when a stage spans all of K
+  const uint16_t* up_s;
+  const uint16_t* down_s;
   const int32_t* unique_ids;
   const int32_t* n_unique;
   const int32_t* seg_off;
   const int32_t* perm;
   const int32_t* plan;       // [n_seg, total_blocks, tile_off[0..n_seg]]
-  uint16_t* hq;              // mode 0 output, fragment-ordered [P+S*T][R]
-  float* ypair;              // mode 1 output [P+S*T][R]
+  int32_t* tb_done;          // [total_blocks] gate/up warps finished per token block
+  int32_t* rb_done;          // [H/128] down warps finished per row block (fused combine)
+  const int32_t* pair_pos;   // for the fused combine
+  const float* topk_w;
+  const uint16_t* residual;
+  uint16_t* out;
   uint32_t* status;
-  int K, R, T, k, E, P;
+  int H, I, T, k, E, S, P;
 };
 
-// MODE 0 gate/up, 1 down; KC elements of K per stage; NT n-tiles of 8 tokens
-// per tile; SINGLE: every tile holds exactly one token (T == 1).
-template <int MODE, int KC, int NT, bool SINGLE>
-struct FfnCfg {
-  static constexpr int NMAT = MODE == 0 ? 2 : 1;
-  static constexpr int TOKB = 8 * NT;                 // tokens per tile
-  static constexpr int GPS = KC / 32;                 // groups per stage
-  static constexpr int GPW = GPS / 2;                 // groups per warp per stage
-  static constexpr int ROWB = KC / 2;                 // code bytes per row per stage
-  static constexpr int SROWB = KC / 16;               // scale bytes per row per stage
+// Shared-memory layout constants.  KC elements of K per stage; NT n-tiles of 8
+// tokens per tile; NMAT matrices per stage (2 = gate+up, 1 = down).
+template <int KC, int NT, int NMAT>
+struct StageCfg {
+  static constexpr int TOKB = 8 * NT;
+  static constexpr int GPW = KC / 64;                 // groups per warp per stage (two K-halves)
+  static constexpr int ROWB = KC / 2;                 // code bytes per row
+  static constexpr int SROWB = KC / 16;               // scale bytes per row
   static constexpr int CODE_BYTES = kRowBlock * ROWB;
   static constexpr int SC_BYTES = kRowBlock * SROWB;
-  static constexpr int W_BYTES = NMAT * (CODE_BYTES + SC_BYTES);   // weights of one stage
-  // activation rows of the tile's tokens for this stage: KC bf16 + 64 B pad, so
-  // the 16-byte fragment loads of 8 tokens x 4 lanes fall in distinct banks
-  static constexpr int XROW = KC * 2 + 64;
-  static constexpr int X_BYTES = TOKB * XROW;
-  static constexpr int STAGE = ((W_BYTES + X_BYTES) + 1023) / 1024 * 1024;
-  static constexpr int RED_BYTES = kRowWarps * 32 * NT * 4 * NMAT * 4;   // K-half partials
-  static constexpr int NS_RAW = (225 * 1024 - RED_BYTES - 2048) / STAGE;
-  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
+  static constexpr int W_BYTES = NMAT * (CODE_BYTES + SC_BYTES);
+  static constexpr int XROW = KC * 2 + 64;            // padded activation row (bank-conflict free)
+  static constexpr int STAGE_USED = W_BYTES + TOKB * XROW;
   static constexpr bool SWZ = (KC == 256);
-  static constexpr size_t SMEM =
-      static_cast<size_t>(NS) * STAGE + RED_BYTES + 1024 + (2 * NS + 2 * kRowWarps) * 8 + 16;
   static_assert(CODE_BYTES % 1024 == 0 && SC_BYTES % 1024 == 0, "stage regions must stay 1 KiB aligned");
-  static_assert(NS >= 2, "pipeline depth");
+};
+
+template <int NT, int KCD>
+struct FusedCfg {
+  using GU = StageCfg<256, NT, 2>;
+  using DN = StageCfg<KCD, NT, 1>;
+  static constexpr int STAGE = ((GU::STAGE_USED > DN::STAGE_USED ? GU::STAGE_USED : DN::STAGE_USED) + 1023) / 1024 * 1024;
+  static constexpr int RED_BYTES = kRowWarps * 32 * NT * 4 * 2 * 4;   // K-half partials (2 matrices)
+  static constexpr int META_BYTES = (3 * kMaxSeg + 4) * 4;            // cached plan / unique / seg_off
+  static constexpr int FIXED = RED_BYTES + META_BYTES + 1024 + 64 * 8 + 64;
+  static constexpr int NS_RAW = (227 * 1024 - FIXED) / STAGE;
+  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
+  static constexpr size_t SMEM = static_cast<size_t>(NS) * STAGE + FIXED;
+  static_assert(NS >= 3, "pipeline depth");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(!SINGLE || NT == 1, "single-token tiles use one n-tile");
 };
 
 // Two code nibbles (e_i, e_{i+4}) of word w -> exact bf16x2 (q_i, q_{i+4}).
@@ -90,51 +109,17 @@ __device__ __forceinline__ uint32_t dq_pair(uint32_t w, int sh) {
   return q;
 }
 
+__device__ __forceinline__ void dq_word_pair(uint32_t (&p)[8], uint32_t w0, uint32_t w1) {
+  p[0] = dq_pair(w0, 0); p[1] = dq_pair(w0, 4); p[2] = dq_pair(w0, 8); p[3] = dq_pair(w0, 12);
+  p[4] = dq_pair(w1, 0); p[5] = dq_pair(w1, 4); p[6] = dq_pair(w1, 8); p[7] = dq_pair(w1, 12);
+}
+
 __device__ __forceinline__ void mma_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ __half2 u32_as_half2(uint32_t v) {
-  __half2 h;
-  memcpy(&h, &v, 4);
-  return h;
-}
-
-struct TileInfo {
-  int u, tb, rb, e, base, cnt;
-  bool routed;
-};
-
-// Tile -> (segment, token block, row block).  Segments 0..S-1 are the shared
-// experts (every token), then the U unique routed experts (plan order).
-__device__ __forceinline__ TileInfo decode_tile(const FfnArgs& a, int tile, int nrb, int n_seg, int U) {
-  TileInfo ti;
-  const int tbg = tile / nrb;
-  ti.rb = tile - tbg * nrb;
-  int lo = 0, hi = n_seg - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.plan + 2 + mid) <= tbg) lo = mid; else hi = mid - 1;
-  }
-  ti.u = lo;
-  ti.tb = tbg - __ldg(a.plan + 2 + lo);
-  const int S = n_seg - U;
-  if (lo >= S) {
-    ti.routed = true;
-    ti.e = __ldg(a.unique_ids + (lo - S));
-    ti.base = __ldg(a.seg_off + (lo - S));
-    ti.cnt = __ldg(a.seg_off + (lo - S) + 1) - ti.base;
-  } else {
-    ti.routed = false;
-    ti.e = a.E + lo;
-    ti.base = a.P + lo * a.T;
-    ti.cnt = a.T;
-  }
-  return ti;
 }
 
 // Accumulate one 32-wide group of one matrix for one n-tile: p[0..3] are the
@@ -153,119 +138,228 @@ __device__ __forceinline__ void group_acc(float (&acc)[4], const uint32_t (&p)[8
   }
 }
 
-__device__ __forceinline__ void dq_word_pair(uint32_t (&p)[8], uint32_t w0, uint32_t w1) {
-  p[0] = dq_pair(w0, 0); p[1] = dq_pair(w0, 4); p[2] = dq_pair(w0, 8); p[3] = dq_pair(w0, 12);
-  p[4] = dq_pair(w1, 0); p[5] = dq_pair(w1, 4); p[6] = dq_pair(w1, 8); p[7] = dq_pair(w1, 12);
+__device__ __forceinline__ __half2 u32_as_half2(uint32_t v) {
+  __half2 h;
+  memcpy(&h, &v, 4);
+  return h;
 }
 
-template <int MODE, int KC, int NT, bool SINGLE>
-__global__ void __launch_bounds__(kFfnThreads, 1)
-    ffn_decode_kernel(const __grid_constant__ CUtensorMap mapq0, const __grid_constant__ CUtensorMap mapq1,
-                      const __grid_constant__ CUtensorMap maps0, const __grid_constant__ CUtensorMap maps1,
-                      const FfnArgs a) {
-  using C = FfnCfg<MODE, KC, NT, SINGLE>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(smem + C::NS * C::STAGE);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NS * C::STAGE + C::RED_BYTES);
-  uint64_t* empty = full + C::NS;
-  uint64_t* red_full = empty + C::NS;       // [kRowWarps]: K-half 1 partials written
-  uint64_t* red_empty = red_full + kRowWarps;  // [kRowWarps]: K-half 0 has read them
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_empty + kRowWarps);
+__device__ __forceinline__ float half2_pick(const __half2& h, int hi) {
+  return hi ? __high2float(h) : __low2float(h);
+}
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kFfnConsumerWarps);
-    }
-    for (int r = 0; r < kRowWarps; ++r) {
-      mbar_init(&red_full[r], 32);
-      mbar_init(&red_empty[r], 32);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Tile geometry shared by producer and consumers.
+struct Meta {
+  const int32_t* plan;      // shared copy: [n_seg, total_blocks, tile_off...]
+  const int32_t* unique;    // shared copy
+  const int32_t* seg_off;   // shared copy
+  int n_seg, U, S, total_blocks, nrb_gu, nrb_dn, tiles_gu, tiles_all;
+};
+
+struct TileInfo {
+  int tbg, rb, e, base, cnt, i0, ntok;
+  bool routed, down;
+};
+
+template <int TOKB>
+__device__ __forceinline__ TileInfo decode_tile(const FfnArgs& a, const Meta& m, int tile) {
+  TileInfo ti;
+  ti.down = tile >= m.tiles_gu;
+  const int t = ti.down ? tile - m.tiles_gu : tile;
+  const int nrb = ti.down ? m.nrb_dn : m.nrb_gu;
+  ti.tbg = t / nrb;
+  ti.rb = t - ti.tbg * nrb;
+  int lo = 0, hi = m.n_seg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.plan[2 + mid] <= ti.tbg) lo = mid; else hi = mid - 1;
   }
-  __syncthreads();
-  pdl_wait();
-  pdl_trigger();
+  const int tb = ti.tbg - m.plan[2 + lo];
+  if (lo >= m.S) {
+    const int u = lo - m.S;
+    ti.routed = true;
+    ti.e = m.unique[u];
+    ti.base = m.seg_off[u];
+    ti.cnt = m.seg_off[u + 1] - ti.base;
+  } else {
+    ti.routed = false;
+    ti.e = a.E + lo;
+    ti.base = a.P + lo * a.T;
+    ti.cnt = a.T;
+  }
+  ti.i0 = tb * TOKB;
+  ti.ntok = min(TOKB, ti.cnt - ti.i0);
+  return ti;
+}
 
-  const int n_seg = __ldg(a.plan + 0);
-  const int nrb = a.R / kRowBlock;
-  const int n_tiles = __ldg(a.plan + 1) * nrb;
-  const int U = __ldg(a.n_unique);
-  const int nkc = a.K / KC;
-
-  if (warp == kFfnConsumerWarps) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      prefetch_tensormap(&mapq0);
-      if (C::NMAT == 2) prefetch_tensormap(&mapq1);
-      if (KC != a.K) {
-        prefetch_tensormap(&maps0);
-        if (C::NMAT == 2) prefetch_tensormap(&maps1);
+// Bounded wait of the producer lane for a token block's h to be complete.
+__device__ __forceinline__ bool wait_h_ready(const FfnArgs& a, int tbg, int target, volatile int* abort_flag) {
+  const int32_t* cnt = a.tb_done + tbg;
+  bool ok = true;
+  if (ld_acquire_gpu(cnt) < target) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+      if (ld_acquire_gpu(cnt) >= target) break;
+      if ((it & 63u) == 0 && (*abort_flag || globaltimer() - t0 > kWaitLimitNs)) {
+        if (!*abort_flag) atomicOr(a.status, COLI_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        ok = false;
+        break;
       }
+      __nanosleep(64);
     }
-    int s = 0;
-    uint32_t ph = 0;
-    long issued = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(a, tile, nrb, n_seg, U);
-      const int row0 = ti.e * a.R + ti.rb * kRowBlock;
-      const int i0 = ti.tb * C::TOKB;
-      const int ntok = min(C::TOKB, ti.cnt - i0);
-      int brow = 0;  // activation row of the token this lane copies (lane < ntok)
-      if (lane < ntok) {
-        const int i = i0 + lane;
-        if (MODE == 0) brow = ti.routed ? __ldg(a.perm + ti.base + i) / a.k : i;
-        else brow = ti.base + i;
-      }
-      const uint16_t* bsrc_row = a.bsrc + static_cast<size_t>(brow) * a.K;
-      for (int kc = 0; kc < nkc; ++kc) {
-        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status);
+  }
+  // h was written through the generic proxy; the bulk copies read it through the async proxy
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return ok;
+}
+
+// Producer: fills the stages of one tile.  For a down tile the weight copies
+// go out immediately; the h rows wait (bounded) for the tile's token block to
+// be complete in gate/up.  Returns false on a timeout.
+template <int KC, int NT, int NMAT, int NS, int STAGE>
+__device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& ti, const CUtensorMap* mq0,
+                                             const CUtensorMap* mq1, const CUtensorMap* ms0, const CUtensorMap* ms1,
+                                             const uint16_t* s0_1d, const uint16_t* s1_1d, int K, int R, int nrb_gu,
+                                             uint8_t* smem, uint64_t* full, uint64_t* empty, int& s, uint32_t& ph,
+                                             long& issued, volatile int* abort_flag, int lane) {
+  using C = StageCfg<KC, NT, NMAT>;
+  const int row0 = ti.e * R + ti.rb * kRowBlock;
+  const int nkc = K / KC;
+  const uint16_t* bsrc = a.xq;
+  if (lane < ti.ntok) {
+    const int i = ti.i0 + lane;
+    if (!ti.down) {
+      const int tok = ti.routed ? __ldg(a.perm + ti.base + i) / a.k : i;
+      bsrc = a.xq + static_cast<size_t>(tok) * K;
+    } else {
+      bsrc = a.hq + static_cast<size_t>(ti.base + i) * K;
+    }
+  }
+  const int target = nrb_gu * kRowWarps;
+  bool b_ready = !ti.down;
+  int pend_s[8], pend_kc[8];
+  int npend = 0;
+  for (int kc = 0; kc < nkc; ++kc) {
+    // a slot still in use would only free up once the consumers have the
+    // pending h rows: resolve them before blocking on it
+    if (!b_ready && npend > 0) {
+      bool free_now = false;
+      if (lane == 0) free_now = mbar_try_wait(&empty[s], ph ^ 1u);
+      free_now = __shfl_sync(0xffffffffu, free_now, 0);
+      if (!free_now || npend == 8) {
+        bool ok = true;
+        if (lane == 0) ok = wait_h_ready(a, ti.tbg, target, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        uint8_t* st = smem + s * C::STAGE;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], C::W_BYTES + ntok * KC * 2);
-          tma_load_2d(st, &mapq0, &full[s], kc * C::ROWB, row0);
-          if (C::NMAT == 2) tma_load_2d(st + C::CODE_BYTES, &mapq1, &full[s], kc * C::ROWB, row0);
-          uint8_t* sc = st + C::NMAT * C::CODE_BYTES;
-          if (KC == a.K) {
-            bulk_load(sc, a.scales0 + static_cast<size_t>(row0) * (a.K / 32), C::SC_BYTES, &full[s]);
-            if (C::NMAT == 2)
-              bulk_load(sc + C::SC_BYTES, a.scales1 + static_cast<size_t>(row0) * (a.K / 32), C::SC_BYTES,
-                        &full[s]);
-          } else {
-            tma_load_2d(sc, &maps0, &full[s], kc * (KC / 32), row0);
-            if (C::NMAT == 2) tma_load_2d(sc + C::SC_BYTES, &maps1, &full[s], kc * (KC / 32), row0);
-          }
-        }
+        if (!ok) return false;
+        b_ready = true;
         __syncwarp();
-        if (lane < ntok) bulk_load(st + C::W_BYTES + lane * C::XROW, bsrc_row + kc * KC, KC * 2, &full[s]);
-        ++issued;
-        if (++s == C::NS) {
-          s = 0;
-          ph ^= 1u;
-        }
+        for (int q = 0; q < npend; ++q)
+          if (lane < ti.ntok)
+            bulk_load(smem + pend_s[q] * STAGE + C::W_BYTES + lane * C::XROW, bsrc + pend_kc[q] * KC, KC * 2,
+                      &full[pend_s[q]]);
+        npend = 0;
       }
     }
-    if (!ok && lane == 0) {
-      // Wait (bounded, ignoring the abort flag) for the copies still in flight
-      // so none lands after this CTA has exited.
-      int dummy = 0;
-      const long n = issued < C::NS ? issued : C::NS;
-      for (long q = 0; q < n; ++q) {
-        const long idx = issued - 1 - q;
-        mbar_wait(&full[static_cast<int>(idx % C::NS)], static_cast<uint32_t>((idx / C::NS) & 1),
-                  reinterpret_cast<volatile int*>(&dummy), a.status);
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) return false;
+    uint8_t* st = smem + s * STAGE;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&full[s], C::W_BYTES + ti.ntok * KC * 2);
+      tma_load_2d(st, mq0, &full[s], kc * C::ROWB, row0);
+      if (NMAT == 2) tma_load_2d(st + C::CODE_BYTES, mq1, &full[s], kc * C::ROWB, row0);
+      uint8_t* sc = st + NMAT * C::CODE_BYTES;
+      if (KC == K) {
+        bulk_load(sc, s0_1d + static_cast<size_t>(row0) * (K / 32), C::SC_BYTES, &full[s]);
+        if (NMAT == 2) bulk_load(sc + C::SC_BYTES, s1_1d + static_cast<size_t>(row0) * (K / 32), C::SC_BYTES, &full[s]);
+      } else {
+        tma_load_2d(sc, ms0, &full[s], kc * (KC / 32), row0);
+        if (NMAT == 2) tma_load_2d(sc + C::SC_BYTES, ms1, &full[s], kc * (KC / 32), row0);
       }
     }
-    return;
+    __syncwarp();
+    if (b_ready) {
+      if (lane < ti.ntok) bulk_load(st + C::W_BYTES + lane * C::XROW, bsrc + kc * KC, KC * 2, &full[s]);
+    } else {
+      pend_s[npend] = s;
+      pend_kc[npend] = kc;
+      ++npend;
+    }
+    ++issued;
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
   }
+  if (npend > 0) {
+    // every stage of the tile is out: wait for h and send the pending rows
+    bool ok = true;
+    if (lane == 0) ok = wait_h_ready(a, ti.tbg, target, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) return false;
+    __syncwarp();
+    for (int q = 0; q < npend; ++q)
+      if (lane < ti.ntok)
+        bulk_load(smem + pend_s[q] * STAGE + C::W_BYTES + lane * C::XROW, bsrc + pend_kc[q] * KC, KC * 2,
+                  &full[pend_s[q]]);
+  }
+  return true;
+}
 
-  // ---------------- consumers ----------------
+// Combine of one 128-row block for all T tokens by one warp (T <= 4):
+// out[t, r] = bf16( sum_j w[t,j] * y[pair_pos[t*k+j], r] + sum_s y[P+s*T+t, r] + residual[t, r] ).
+__device__ __forceinline__ void warp_combine_rows(const FfnArgs& a, int rb, int lane) {
+  for (int t = 0; t < a.T; ++t) {
+    const int r = rb * kRowBlock + lane * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < a.k; ++j) {
+      const int pp = a.pair_pos[t * a.k + j];
+      if (pp >= 0) {
+        const float wt = a.topk_w[t * a.k + j];
+        const float4 y = __ldcg(reinterpret_cast<const float4*>(a.ypair + static_cast<size_t>(pp) * a.H + r));
+        acc.x = fmaf(wt, y.x, acc.x);
+        acc.y = fmaf(wt, y.y, acc.y);
+        acc.z = fmaf(wt, y.z, acc.z);
+        acc.w = fmaf(wt, y.w, acc.w);
+      }
+    }
+    for (int s = 0; s < a.S; ++s) {
+      const float4 y =
+          __ldcg(reinterpret_cast<const float4*>(a.ypair + static_cast<size_t>(a.P + s * a.T + t) * a.H + r));
+      acc.x += y.x;
+      acc.y += y.y;
+      acc.z += y.z;
+      acc.w += y.w;
+    }
+    if (a.residual) {
+      const uint2 rv = *reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r);
+      acc.x += __uint_as_float(rv.x << 16);
+      acc.y += __uint_as_float(rv.x & 0xffff0000u);
+      acc.z += __uint_as_float(rv.y << 16);
+      acc.w += __uint_as_float(rv.y & 0xffff0000u);
+    }
+    uint2 o;
+    o.x = float_to_bf16_bits(acc.x) | (static_cast<uint32_t>(float_to_bf16_bits(acc.y)) << 16);
+    o.y = float_to_bf16_bits(acc.z) | (static_cast<uint32_t>(float_to_bf16_bits(acc.w)) << 16);
+    *reinterpret_cast<uint2*>(a.out + static_cast<size_t>(t) * a.H + r) = o;
+  }
+}
+
+// Consumers: one tile.  Returns false on a timeout.
+template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE>
+__device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, const TileInfo& ti, int K, int R,
+                                             uint8_t* smem, float* red, uint64_t* full, uint64_t* empty,
+                                             uint64_t* red_full, uint64_t* red_empty, int& s, uint32_t& ph,
+                                             uint32_t& rph, volatile int* abort_flag, int warp, int lane) {
+  using C = StageCfg<KC, NT, NMAT>;
   const int rw = warp & (kRowWarps - 1);   // 16-row slice
   const int half = warp / kRowWarps;       // which half of each stage's groups
   const int g = lane >> 2, c = lane & 3;
@@ -277,130 +371,255 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   const uint32_t cbase = rl0 * C::ROWB + (C::SWZ ? (g << 4) : 0) + 4 * c;
   const uint32_t sbase = rl0 * C::SROWB + half * C::GPW * 2;
   const uint32_t xbase = C::W_BYTES + g * C::XROW + (half * C::GPW * 32 + 8 * c) * 2;
+  const int nnt = (ti.ntok + 7) >> 3;
+  const int nkc = K / KC;
+  float acc0[NT][4], acc1[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc0[nt][q] = 0.f;
+      acc1[nt][q] = 0.f;
+    }
+
+  for (int kc = 0; kc < nkc; ++kc) {
+    if (!mbar_wait(&full[s], ph, abort_flag, a.status)) return false;
+    const uint8_t* st = smem + s * STAGE;
+    const uint8_t* sc = st + NMAT * C::CODE_BYTES + sbase;
+    // this warp's fp16 scales for its GPW groups (rows rl0 and rl0 + 8, both matrices)
+    __half2 sh0[2], sh1[2], th0[2], th1[2];
+    if (C::GPW == 4) {
+      const uint2 v0 = *reinterpret_cast<const uint2*>(sc);
+      const uint2 v1 = *reinterpret_cast<const uint2*>(sc + 8 * C::SROWB);
+      sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
+      sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y);
+      if (NMAT == 2) {
+        const uint2 u0 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES);
+        const uint2 u1 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES + 8 * C::SROWB);
+        th0[0] = u32_as_half2(u0.x); th0[1] = u32_as_half2(u0.y);
+        th1[0] = u32_as_half2(u1.x); th1[1] = u32_as_half2(u1.y);
+      }
+    } else {
+      sh0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc));
+      sh1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + 8 * C::SROWB));
+      sh0[1] = sh0[0];
+      sh1[1] = sh1[0];
+      if (NMAT == 2) {
+        th0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES));
+        th1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES + 8 * C::SROWB));
+        th0[1] = th0[0];
+        th1[1] = th1[0];
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < C::GPW; ++jj) {
+      const int j = half * C::GPW + jj;                       // group within the stage
+      const uint8_t* ca = st + (cbase ^ static_cast<uint32_t>(j << 4));
+      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
+      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::ROWB);
+      const float s0 = half2_pick(sh0[jj >> 1], jj & 1);
+      const float s1 = half2_pick(sh1[jj >> 1], jj & 1);
+      uint32_t pg[8], pu[8];
+      dq_word_pair(pg, w0, w1);
+      float t0 = 0.f, t1 = 0.f;
+      if (NMAT == 2) {
+        const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
+        const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::ROWB);
+        t0 = half2_pick(th0[jj >> 1], jj & 1);
+        t1 = half2_pick(th1[jj >> 1], jj & 1);
+        dq_word_pair(pu, v0, v1);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (NT == 1 || nt < nnt) {
+          uint4 b = make_uint4(0u, 0u, 0u, 0u);
+          if (nt * 8 + g < ti.ntok) b = *reinterpret_cast<const uint4*>(st + xbase + nt * 8 * C::XROW + jj * 64);
+          group_acc<SINGLE>(acc0[nt], pg, b, s0, s1);
+          if (NMAT == 2) group_acc<SINGLE>(acc1[nt], pu, b, t0, t1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+
+  // Add the two K-halves of each 16-row slice (fixed order: half 0 + half 1),
+  // handing the partials over through shared memory under bounded waits.
+  float* rp = red + (rw * 32 + lane) * (NT * 4 * 2);
+  if (half == 1) {
+    if (!mbar_wait(&red_empty[rw], rph ^ 1u, abort_flag, a.status)) return false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        rp[nt * 4 + q] = acc0[nt][q];
+        if (NMAT == 2) rp[NT * 4 + nt * 4 + q] = acc1[nt][q];
+      }
+    mbar_arrive(&red_full[rw]);
+    rph ^= 1u;
+    return true;
+  }
+  if (!mbar_wait(&red_full[rw], rph, abort_flag, a.status)) return false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc0[nt][q] += rp[nt * 4 + q];
+      if (NMAT == 2) acc1[nt][q] += rp[NT * 4 + nt * 4 + q];
+    }
+  mbar_arrive(&red_empty[rw]);
+  rph ^= 1u;
+  // epilogue: d0 (row g, col 2c), d1 (row g, col 2c+1), d2 (row g+8, col 2c), d3 (row g+8, col 2c+1)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    if (nt < nnt) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = ti.i0 + nt * 8 + 2 * c + (q & 1);
+        if (i < ti.cnt && !(SINGLE && (q & 1))) {
+          const size_t orow = static_cast<size_t>(ti.base + i);
+          const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
+          if (NMAT == 2) {
+            const float gv = acc0[nt][q], uv = acc1[nt][q];
+            const float hv = gv / (1.0f + expf(-gv)) * uv;
+            a.hq[orow * R + frag_pos(r)] = float_to_bf16_bits(hv);
+          } else {
+            a.ypair[orow * R + r] = acc0[nt][q];
+          }
+        }
+      }
+    }
+  }
+  // publish: every lane's stores, then one increment per warp
+  __threadfence();
+  __syncwarp();
+  if (NMAT == 2) {
+    if (lane == 0) atomicAdd(a.tb_done + ti.tbg, 1);
+  } else if (a.T <= kFusedCombineMaxT) {
+    int old = 0;
+    if (lane == 0) old = atomicAdd(a.rb_done + ti.rb, 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old + 1 == m.total_blocks * kRowWarps) {   // last warp of this row block
+      __threadfence();
+      warp_combine_rows(a, ti.rb, lane);
+    }
+  }
+  return true;
+}
+
+// The persistent FFN kernel (gate/up tiles, then down tiles).  Launched
+// cooperatively so that every CTA is resident: a down tile only waits for
+// gate/up tiles, which every CTA processes before any of its down tiles.
+template <int NT, bool SINGLE, int KCD>
+__global__ void __launch_bounds__(kFfnThreads, 1)
+    ffn_fused_kernel(const __grid_constant__ CUtensorMap gq, const __grid_constant__ CUtensorMap uq,
+                     const __grid_constant__ CUtensorMap gs, const __grid_constant__ CUtensorMap us,
+                     const __grid_constant__ CUtensorMap dq, const __grid_constant__ CUtensorMap ds,
+                     const FfnArgs a) {
+  using F = FusedCfg<NT, KCD>;
+  constexpr int NS = F::NS, STAGE = F::STAGE;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(smem + NS * STAGE);
+  int32_t* meta = reinterpret_cast<int32_t*>(smem + NS * STAGE + F::RED_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE + F::RED_BYTES + F::META_BYTES);
+  uint64_t* empty = full + NS;
+  uint64_t* red_full = empty + NS;
+  uint64_t* red_empty = red_full + kRowWarps;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_empty + kRowWarps);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < NS; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kFfnConsumerWarps);
+    }
+    for (int r = 0; r < kRowWarps; ++r) {
+      mbar_init(&red_full[r], 32);
+      mbar_init(&red_empty[r], 32);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kFfnConsumerWarps && lane == 0) {
+    prefetch_tensormap(&gq);
+    prefetch_tensormap(&uq);
+    prefetch_tensormap(&dq);
+  }
+  pdl_wait();
+  pdl_trigger();
+  // cache the plan, the unique experts and their segment offsets
+  Meta m;
+  {
+    const int n_seg = __ldg(a.plan);
+    const int U = __ldg(a.n_unique);
+    int32_t* mplan = meta;
+    int32_t* muniq = meta + kMaxSeg + 2;
+    int32_t* mseg = muniq + kMaxSeg;
+    for (int i = threadIdx.x; i < n_seg + 3; i += blockDim.x) mplan[i] = __ldg(a.plan + i);
+    for (int i = threadIdx.x; i < U; i += blockDim.x) muniq[i] = __ldg(a.unique_ids + i);
+    for (int i = threadIdx.x; i <= U; i += blockDim.x) mseg[i] = __ldg(a.seg_off + i);
+    m.plan = mplan;
+    m.unique = muniq;
+    m.seg_off = mseg;
+    m.n_seg = n_seg;
+    m.U = U;
+    m.S = n_seg - U;
+    m.total_blocks = __ldg(a.plan + 1);
+    m.nrb_gu = a.I / kRowBlock;
+    m.nrb_dn = a.H / kRowBlock;
+    m.tiles_gu = m.total_blocks * m.nrb_gu;
+    m.tiles_all = m.tiles_gu + m.total_blocks * m.nrb_dn;
+  }
+  __syncthreads();
+  constexpr int TOKB = 8 * NT;
+
+  if (warp == kFfnConsumerWarps) {
+    // ---------------- producer ----------------
+    int s = 0;
+    uint32_t ph = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < m.tiles_all; tile += gridDim.x) {
+      const TileInfo ti = decode_tile<TOKB>(a, m, tile);
+      if (!ti.down)
+        ok = produce_tile<256, NT, 2, NS, STAGE>(a, ti, &gq, &uq, &gs, &us, a.gate_s, a.up_s, a.H, a.I, m.nrb_gu,
+                                                 smem, full, empty, s, ph, issued, abort_flag, lane);
+      else
+        ok = produce_tile<KCD, NT, 1, NS, STAGE>(a, ti, &dq, &dq, &ds, &ds, a.down_s, a.down_s, a.I, a.H, m.nrb_gu,
+                                                 smem, full, empty, s, ph, issued, abort_flag, lane);
+    }
+    if (!ok && lane == 0) {
+      // Wait (bounded, ignoring the abort flag) for the copies still in flight
+      // so none lands after this CTA has exited.
+      int dummy = 0;
+      const long n = issued < NS ? issued : NS;
+      for (long q = 0; q < n; ++q) {
+        const long idx = issued - 1 - q;
+        mbar_wait(&full[static_cast<int>(idx % NS)], static_cast<uint32_t>((idx / NS) & 1),
+                  reinterpret_cast<volatile int*>(&dummy), a.status);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
   int s = 0;
   uint32_t ph = 0, rph = 0;
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, rph ^= 1u) {
-    const TileInfo ti = decode_tile(a, tile, nrb, n_seg, U);
-    const int i0 = ti.tb * C::TOKB;
-    const int ntok = min(C::TOKB, ti.cnt - i0);
-    const int nnt = (ntok + 7) >> 3;
-    float acc0[NT][4], acc1[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc0[nt][q] = 0.f;
-        acc1[nt][q] = 0.f;
-      }
-
-    for (int kc = 0; kc < nkc; ++kc) {
-      if (!mbar_wait(&full[s], ph, abort_flag, a.status)) return;
-      const uint8_t* st = smem + s * C::STAGE;
-      const uint8_t* sc = st + C::NMAT * C::CODE_BYTES + sbase;
-      // this warp's fp16 scales for its GPW groups (rows rl0 and rl0 + 8, both matrices)
-      __half2 sh0[2], sh1[2], th0[2], th1[2];
-      if (C::GPW == 4) {
-        const uint2 v0 = *reinterpret_cast<const uint2*>(sc);
-        const uint2 v1 = *reinterpret_cast<const uint2*>(sc + 8 * C::SROWB);
-        sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
-        sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y);
-        if (C::NMAT == 2) {
-          const uint2 u0 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES);
-          const uint2 u1 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES + 8 * C::SROWB);
-          th0[0] = u32_as_half2(u0.x); th0[1] = u32_as_half2(u0.y);
-          th1[0] = u32_as_half2(u1.x); th1[1] = u32_as_half2(u1.y);
-        }
-      } else {
-        sh0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc));
-        sh1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + 8 * C::SROWB));
-        sh0[1] = sh1[1] = sh0[0];
-        if (C::NMAT == 2) {
-          th0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES));
-          th1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES + 8 * C::SROWB));
-          th0[1] = th1[1] = th0[0];
-        }
-      }
-#pragma unroll
-      for (int jj = 0; jj < C::GPW; ++jj) {
-        const int j = half * C::GPW + jj;                       // group within the stage
-        const uint8_t* ca = st + (cbase ^ static_cast<uint32_t>(j << 4));
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::ROWB);
-        const float s0 = (jj & 1) ? __high2float(sh0[jj >> 1]) : __low2float(sh0[jj >> 1]);
-        const float s1 = (jj & 1) ? __high2float(sh1[jj >> 1]) : __low2float(sh1[jj >> 1]);
-        uint32_t pg[8], pu[8];
-        dq_word_pair(pg, w0, w1);
-        float t0 = 0.f, t1 = 0.f;
-        if (C::NMAT == 2) {
-          const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
-          const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::ROWB);
-          t0 = (jj & 1) ? __high2float(th0[jj >> 1]) : __low2float(th0[jj >> 1]);
-          t1 = (jj & 1) ? __high2float(th1[jj >> 1]) : __low2float(th1[jj >> 1]);
-          dq_word_pair(pu, v0, v1);
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if (NT == 1 || nt < nnt) {
-            uint4 b = make_uint4(0u, 0u, 0u, 0u);
-            if (nt * 8 + g < ntok) b = *reinterpret_cast<const uint4*>(st + xbase + nt * 8 * C::XROW + jj * 64);
-            group_acc<SINGLE>(acc0[nt], pg, b, s0, s1);
-            if (C::NMAT == 2) group_acc<SINGLE>(acc1[nt], pu, b, t0, t1);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == C::NS) {
-        s = 0;
-        ph ^= 1u;
-      }
-    }
-
-    // Combine the two K-halves of each 16-row slice (fixed order: half 0 + half 1),
-    // handing the partials over through shared memory under bounded waits.
-    float* rp = red + (rw * 32 + lane) * (NT * 4 * C::NMAT);
-    if (half == 1) {
-      if (!mbar_wait(&red_empty[rw], rph ^ 1u, abort_flag, a.status)) return;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          rp[nt * 4 + q] = acc0[nt][q];
-          if (C::NMAT == 2) rp[NT * 4 + nt * 4 + q] = acc1[nt][q];
-        }
-      mbar_arrive(&red_full[rw]);
-      continue;
-    }
-    if (!mbar_wait(&red_full[rw], rph, abort_flag, a.status)) return;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc0[nt][q] += rp[nt * 4 + q];
-        if (C::NMAT == 2) acc1[nt][q] += rp[NT * 4 + nt * 4 + q];
-      }
-    mbar_arrive(&red_empty[rw]);
-    // epilogue: d0 (row g, col 2c), d1 (row g, col 2c+1), d2 (row g+8, col 2c), d3 (row g+8, col 2c+1)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      if (nt < nnt) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = i0 + nt * 8 + 2 * c + (q & 1);
-          if (i < ti.cnt && !(SINGLE && (q & 1))) {
-            const size_t orow = static_cast<size_t>(ti.base + i);
-            const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
-            if (MODE == 0) {
-              const float gv = acc0[nt][q], uv = acc1[nt][q];
-              const float hv = gv / (1.0f + expf(-gv)) * uv;
-              a.hq[orow * a.R + frag_pos(r)] = float_to_bf16_bits(hv);
-            } else {
-              a.ypair[orow * a.R + r] = acc0[nt][q];
-            }
-          }
-        }
-      }
-    }
+  for (int tile = blockIdx.x; tile < m.tiles_all; tile += gridDim.x) {
+    const TileInfo ti = decode_tile<TOKB>(a, m, tile);
+    bool ok;
+    if (!ti.down)
+      ok = consume_tile<256, NT, 2, SINGLE, NS, STAGE>(a, m, ti, a.H, a.I, smem, red, full, empty, red_full,
+                                                        red_empty, s, ph, rph, abort_flag, warp, lane);
+    else
+      ok = consume_tile<KCD, NT, 1, SINGLE, NS, STAGE>(a, m, ti, a.I, a.H, smem, red, full, empty, red_full,
+                                                        red_empty, s, ph, rph, abort_flag, warp, lane);
+    if (!ok) return;
   }
 }
 

@@ -126,8 +126,11 @@ __device__ __forceinline__ int block_union(const int32_t* ids, int P, int E, int
 // blocks of `tokb` tokens; plan = [n_seg, total_blocks, tile_off[0..n_seg]]
 // with tile_off the exclusive prefix of the blocks per segment.  Shared
 // segments come first so their tiles do not depend on the routing.
+// Also zeroes the FFN's completion counters (tb_done per token block,
+// rb_done per output row block) for this call.
 __device__ __forceinline__ void block_plan(int U, const int* seg_cnt, int T, int S, int tokb, int* scratch,
-                                           int32_t* __restrict__ plan) {
+                                           int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
+                                           int32_t* __restrict__ rb_done, int n_rb) {
   __shared__ int carry;
   const int n_seg = U + S;
   if (threadIdx.x == 0) carry = 0;
@@ -150,6 +153,10 @@ __device__ __forceinline__ void block_plan(int U, const int* seg_cnt, int T, int
     plan[1] = carry;
     plan[2 + n_seg] = carry;
   }
+  if (tb_done)
+    for (int i = threadIdx.x; i < carry; i += blockDim.x) tb_done[i] = 0;
+  if (rb_done)
+    for (int i = threadIdx.x; i < n_rb; i += blockDim.x) rb_done[i] = 0;
 }
 
 // Union of a routed batch (any size) and, if `plan` is given, the FFN tile plan.
@@ -158,20 +165,22 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
     union_kernel(const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ unique_ids,
                  int32_t* __restrict__ n_unique, int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
                  int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status, int T, int S, int tokb,
-                 int32_t* __restrict__ plan) {
+                 int32_t* __restrict__ plan, int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done,
+                 int n_rb) {
   extern __shared__ int hist[];
   __shared__ int scratch[33];
   __shared__ int seg_cnt[1024];
   pdl_wait();
   pdl_trigger();
   const int U = block_union(ids, P, E, hist, scratch, seg_cnt, unique_ids, n_unique, seg_off, perm, pair_pos, status);
-  if (plan) block_plan(U, seg_cnt, T, S, tokb, scratch, plan);
+  if (plan) block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
 }
 
 // Plan from an existing union (coli_moe_expert_ffn), one CTA.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ n_unique,
                                                     const int32_t* __restrict__ seg_off, int T, int S, int tokb,
-                                                    int32_t* __restrict__ plan) {
+                                                    int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
+                                                    int32_t* __restrict__ rb_done, int n_rb) {
   __shared__ int scratch[33];
   __shared__ int seg_cnt[1024];
   pdl_wait();
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   const int U = *n_unique;
   for (int u = threadIdx.x; u < U; u += blockDim.x) seg_cnt[u] = seg_off[u + 1] - seg_off[u];
   __syncthreads();
-  block_plan(U, seg_cnt, T, S, tokb, scratch, plan);
+  block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
 }
 
 // Small batches (T <= kFusedRouteMaxT): Route, Union and the tile plan in one
@@ -192,7 +201,8 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
                        int32_t* __restrict__ ids_out, float* __restrict__ w_out, int32_t* __restrict__ unique_ids,
                        int32_t* __restrict__ n_unique, int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
                        int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status, int S, int tokb,
-                       int32_t* __restrict__ plan) {
+                       int32_t* __restrict__ plan, int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done,
+                       int n_rb) {
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   int* ids_s = smem_i + kUnionWarps * E;
@@ -215,7 +225,7 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
   __syncthreads();
   const int U = block_union(ids_s, T * k, E, hist, scratch, seg_cnt, unique_ids, n_unique, seg_off, perm, pair_pos,
                             status);
-  block_plan(U, seg_cnt, T, S, tokb, scratch, plan);
+  block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
 }
 
 }  // namespace coli
