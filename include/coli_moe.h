@@ -163,6 +163,35 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
                            float *logits_out, int32_t *topk_ids_out, float *topk_w_out,
                            void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * coli_moe_layer without a caller-provided workspace.  The pages describe no
+ * such call; it exists for callers that cannot allocate device memory when
+ * they run the layer: code embedded in a host runtime that owns every device
+ * allocation (a plugin or custom operator inside another inference engine),
+ * real-time loops whose memory is fixed up front, or callers that simply have
+ * no allocator at hand.  Instead of `ws`, it uses a scratch array of
+ * COLI_NOALLOC_SCRATCH_BYTES bytes that the library itself places in device
+ * memory as a file-scope variable: every GPU that loads the library holds
+ * that much memory until the process exits.
+ *   - Arguments and results are those of coli_moe_layer, without ws/ws_bytes.
+ *   - Batches whose coli_moe_workspace_bytes(dims, T) exceeds
+ *     COLI_NOALLOC_SCRATCH_BYTES are rejected with COLI_ERR_WORKSPACE before
+ *     anything is launched (up to 29 tokens for H=6144, I=2048, E=256, k=8, S=1).
+ *   - The first call on a device looks up the array's device address (one
+ *     cudaGetSymbolAddress with that device current); make that first call
+ *     before capturing a stream.  No call allocates or frees device memory.
+ *   - Every call on a device uses the same array, which keeps whatever the
+ *     last call left in it (the layer needs nothing in it to start at zero).
+ *     Calls that can overlap on the GPU (different streams without ordering
+ *     between them) race on the array and give undefined results: order them.
+ */
+#define COLI_NOALLOC_SCRATCH_BYTES (8u << 20)
+coli_status coli_moe_layer_noalloc(const coli_moe_dims *dims, const coli_moe_weights *w,
+                                   const uint16_t *x, int T, const float *logits_in,
+                                   const uint16_t *residual, uint32_t flags, uint16_t *out,
+                                   float *logits_out, int32_t *topk_ids_out, float *topk_w_out,
+                                   void *stream);
+
 /* Workspace bytes needed by coli_moe_layer / coli_moe_expert_ffn for up to T_max
  * tokens (0 for unsupported dims). Host only. */
 size_t coli_moe_workspace_bytes(const coli_moe_dims *dims, int T_max);

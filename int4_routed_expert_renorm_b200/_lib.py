@@ -22,7 +22,8 @@ COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
 
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
-           "coli_moe_launch_count", "coli_moe_set_stage_events")
+           "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc")
+COLI_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class ColiError(RuntimeError):
@@ -59,6 +60,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_version": (I, []),
         "coli_moe_launch_count": (U64, [I]),
         "coli_moe_set_stage_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
+        "coli_moe_layer_noalloc": (I, [D, W, P, I, P, P, U32, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -130,6 +132,16 @@ def coli_moe_layer(dims, weights, x, out, ws, logits_in=None, residual=None, fla
                                _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
                                _ptr(topk_w_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "coli_moe_layer")
+
+
+def coli_moe_layer_noalloc(dims, weights, x, out, logits_in=None, residual=None, flags=0, logits_out=None,
+                           topk_ids_out=None, topk_w_out=None, stream=None):
+    """coli_moe_layer with the library's own scratch instead of a workspace
+    tensor, for callers that cannot allocate device memory (see the header)."""
+    T = x.shape[0]
+    _check(_lib.coli_moe_layer_noalloc(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
+                                       _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
+                                       _ptr(topk_w_out), _stream(stream)), "coli_moe_layer_noalloc")
 
 
 def coli_moe_set_stage_events(events):

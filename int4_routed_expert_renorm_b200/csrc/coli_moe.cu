@@ -19,6 +19,12 @@
 
 using namespace coli;
 
+// Scratch of coli_moe_layer_noalloc (see include/coli_moe.h): device memory
+// owned by the library for callers that cannot allocate.  Host code must not
+// use this name as a pointer; its device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[COLI_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 __device__ uint32_t g_status_word;
@@ -546,6 +552,31 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   // 3. expert FFN and combine
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
                  di, s, rec);
+}
+
+coli_status coli_moe_layer_noalloc(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
+                                   const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
+                                   float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* stream) {
+  static std::mutex mu;
+  static void* scratch_ptr[kMaxDevices] = {};
+  const coli_status st = check_dims(dims);
+  if (st != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (coli_moe_workspace_bytes(dims, T) > COLI_NOALLOC_SCRATCH_BYTES) return COLI_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return COLI_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!scratch_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return COLI_ERR_CUDA;
+      scratch_ptr[dev] = p;
+    }
+    ptr = scratch_ptr[dev];
+  }
+  return coli_moe_layer(dims, w, x, T, logits_in, residual, flags, out, logits_out, topk_ids_out, topk_w_out, ptr,
+                        COLI_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 coli_status coli_moe_get_status(void* stream, uint32_t* flags) {
