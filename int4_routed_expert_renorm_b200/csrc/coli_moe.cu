@@ -295,9 +295,25 @@ bool launch_route(const float* lg, const float* bias, int T, int E, int k, int32
   }
 }
 
-// Route + union + plan in one CTA (T <= kFusedRouteMaxT).
+// Route + union + plan in one CTA (T <= kFusedRouteMaxT); one warp does the
+// union when T*k <= kWarpUnionMaxP.
 bool launch_route_union(const float* lg, const float* bias, int T, int E, int k, int S, int tokb, int n_rb,
                         int32_t* ids, float* w, const Ws& ws, uint32_t* status, cudaStream_t st) {
+  if (T * k <= kWarpUnionMaxP) {
+    const dim3 g(1), b(32 * (T < 8 ? T : 8));
+#define COLI_RUS(NV)                                                                                             \
+  launch(route_union_small_kernel<NV>, g, b, 0, st, lg, bias, T, E, k, ids, w, ws.unique, ws.n_unique, ws.seg_off, \
+         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb)
+    switch (route_nv(E)) {
+      case 1: return COLI_RUS(1);
+      case 2: return COLI_RUS(2);
+      case 4: return COLI_RUS(4);
+      case 8: return COLI_RUS(8);
+      case 16: return COLI_RUS(16);
+      default: return COLI_RUS(32);
+    }
+#undef COLI_RUS
+  }
   const size_t smem = static_cast<size_t>(kUnionWarps * E + T * k) * 4;
   const dim3 g(1), b(kUnionThreads);
 #define COLI_RU(NV)                                                                                            \

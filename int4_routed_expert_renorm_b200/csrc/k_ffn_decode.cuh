@@ -317,18 +317,32 @@ __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& t
 // Combine of one 128-row block for all T tokens by one warp (T <= 4):
 // out[t, r] = bf16( sum_j w[t,j] * y[pair_pos[t*k+j], r] + sum_s y[P+s*T+t, r] + residual[t, r] ).
 __device__ __forceinline__ void warp_combine_rows(const FfnArgs& a, int rb, int lane) {
+  const int r = rb * kRowBlock + lane * 4;
   for (int t = 0; t < a.T; ++t) {
-    const int r = rb * kRowBlock + lane * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < a.k; ++j) {
-      const int pp = a.pair_pos[t * a.k + j];
-      if (pp >= 0) {
-        const float wt = a.topk_w[t * a.k + j];
-        const float4 y = __ldcg(reinterpret_cast<const float4*>(a.ypair + static_cast<size_t>(pp) * a.H + r));
-        acc.x = fmaf(wt, y.x, acc.x);
-        acc.y = fmaf(wt, y.y, acc.y);
-        acc.z = fmaf(wt, y.z, acc.z);
-        acc.w = fmaf(wt, y.w, acc.w);
+    // issue the loads of up to 8 routed slots at once, then add them in slot order
+    for (int j0 = 0; j0 < a.k; j0 += 8) {
+      int pp[8];
+      float wt[8];
+      float4 y[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int j = j0 + q;
+        pp[q] = j < a.k ? a.pair_pos[t * a.k + j] : -1;
+        wt[q] = j < a.k ? a.topk_w[t * a.k + j] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        y[q] = pp[q] >= 0 ? __ldcg(reinterpret_cast<const float4*>(a.ypair + static_cast<size_t>(pp[q]) * a.H + r))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (pp[q] >= 0) {
+          acc.x = fmaf(wt[q], y[q].x, acc.x);
+          acc.y = fmaf(wt[q], y[q].y, acc.y);
+          acc.z = fmaf(wt[q], y[q].z, acc.z);
+          acc.w = fmaf(wt[q], y[q].w, acc.w);
+        }
       }
     }
     for (int s = 0; s < a.S; ++s) {
@@ -640,15 +654,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     const int t = static_cast<int>(idx / per_tok);
     const int n = static_cast<int>(idx - static_cast<long>(t) * per_tok) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const int pp = __ldg(pair_pos + t * k + j);
-      if (pp >= 0) {
-        const float wt = __ldg(w + t * k + j);
-        const float4 y = __ldg(reinterpret_cast<const float4*>(ypair + static_cast<size_t>(pp) * H + n));
-        acc.x = fmaf(wt, y.x, acc.x);
-        acc.y = fmaf(wt, y.y, acc.y);
-        acc.z = fmaf(wt, y.z, acc.z);
-        acc.w = fmaf(wt, y.w, acc.w);
+    // issue the loads of up to 8 routed slots at once, then add them in slot order
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int pp[8];
+      float wt[8];
+      float4 y[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int j = j0 + q;
+        pp[q] = j < k ? __ldg(pair_pos + t * k + j) : -1;
+        wt[q] = j < k ? __ldg(w + t * k + j) : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        y[q] = pp[q] >= 0 ? __ldg(reinterpret_cast<const float4*>(ypair + static_cast<size_t>(pp[q]) * H + n))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (pp[q] >= 0) {
+          acc.x = fmaf(wt[q], y[q].x, acc.x);
+          acc.y = fmaf(wt[q], y[q].y, acc.y);
+          acc.z = fmaf(wt[q], y[q].z, acc.z);
+          acc.w = fmaf(wt[q], y[q].w, acc.w);
+        }
       }
     }
     for (int s = 0; s < S; ++s) {

@@ -198,37 +198,51 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
     }
   }
   if (!wr) return;
-  // logits of expert e for every token, 8 tokens at a time
+  // logits of expert e for every token, 8 tokens at a time.  Each lane issues
+  // all its W_r loads (and a token's x loads) before any arithmetic, so the
+  // DRAM round trips overlap instead of following one another.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hw = H >> 3;
   const int h0 = warp * hw, h1 = h0 + hw;
   const float* wrow = wr + static_cast<size_t>(e) * H;
   __shared__ float part[8][8];
+  constexpr int kIt = 8;                       // float4 per lane per pass (1024 elements per warp)
   for (int t0 = 0; t0 < T; t0 += 8) {
     const int nt = min(8, T - t0);
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int h = h0 + lane * 4; h < h1; h += 128) {
-      const float4 w = __ldg(reinterpret_cast<const float4*>(wrow + h));
+    for (int hb = h0 + lane * 4; hb < h1; hb += 128 * kIt) {
+      float4 w[kIt];
+#pragma unroll
+      for (int it = 0; it < kIt; ++it)
+        w[it] = (hb + it * 128 < h1) ? __ldg(reinterpret_cast<const float4*>(wrow + hb + it * 128))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (q < nt) {
-          const uint2 xv = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t0 + q) * H + h);
-          float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
-          float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
-          if (prenorm) {
-            const float r = rs[t0 + q];
-            x0 = bf16_bits_to_float(float_to_bf16_bits(x0 * r));
-            x1 = bf16_bits_to_float(float_to_bf16_bits(x1 * r));
-            x2 = bf16_bits_to_float(float_to_bf16_bits(x2 * r));
-            x3 = bf16_bits_to_float(float_to_bf16_bits(x3 * r));
-          }
+          const uint16_t* xr = x + static_cast<size_t>(t0 + q) * H;
+          uint2 xv[kIt];
+#pragma unroll
+          for (int it = 0; it < kIt; ++it)
+            xv[it] = (hb + it * 128 < h1) ? *reinterpret_cast<const uint2*>(xr + hb + it * 128) : make_uint2(0u, 0u);
           float a = acc[q];
-          a = fmaf(x0, w.x, a);
-          a = fmaf(x1, w.y, a);
-          a = fmaf(x2, w.z, a);
-          a = fmaf(x3, w.w, a);
+#pragma unroll
+          for (int it = 0; it < kIt; ++it) {
+            float x0 = __uint_as_float(xv[it].x << 16), x1 = __uint_as_float(xv[it].x & 0xffff0000u);
+            float x2 = __uint_as_float(xv[it].y << 16), x3 = __uint_as_float(xv[it].y & 0xffff0000u);
+            if (prenorm) {
+              const float r = rs[t0 + q];
+              x0 = bf16_bits_to_float(float_to_bf16_bits(x0 * r));
+              x1 = bf16_bits_to_float(float_to_bf16_bits(x1 * r));
+              x2 = bf16_bits_to_float(float_to_bf16_bits(x2 * r));
+              x3 = bf16_bits_to_float(float_to_bf16_bits(x3 * r));
+            }
+            a = fmaf(x0, w[it].x, a);
+            a = fmaf(x1, w[it].y, a);
+            a = fmaf(x2, w[it].z, a);
+            a = fmaf(x3, w[it].w, a);
+          }
           acc[q] = a;
         }
       }
@@ -245,7 +259,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
     if (threadIdx.x < nt) {
       float sacc = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) sacc += part[w][threadIdx.x];
+      for (int w8 = 0; w8 < 8; ++w8) sacc += part[w8][threadIdx.x];
       logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = sacc;
     }
   }

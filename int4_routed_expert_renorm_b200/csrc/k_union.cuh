@@ -228,4 +228,190 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
   block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
 }
 
+// ---------------------------------------------------------------------------
+// Small batches (T*k <= 128): the union in ONE warp, without block barriers.
+// The 128 keys (expert << 8 | pair) live four per lane (key i in lane i/4,
+// slot i%4; unused keys are INT_MAX) and are put in order by a bitonic
+// network: partners within a lane swap in registers, partners in other lanes
+// are exchanged with __shfl_xor_sync.  Sorting by (expert, pair) is exactly
+// the stable grouping of pairs by expert.
+constexpr int kWarpUnionMaxP = 128;
+
+// The stage loops are kept rolled (only the four in-lane slots are unrolled):
+// this kernel runs once per layer right after the expert FFN has streamed the
+// weights through L2, so its code is fetched cold every time and a small code
+// footprint matters more than loop overhead.
+__device__ __forceinline__ void warp_bitonic_sort128(int (&key)[4], int lane) {
+#pragma unroll 1
+  for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll 1
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 4) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = lane * 4 + r;
+          const int other = __shfl_xor_sync(0xffffffffu, key[r], j >> 2);
+          const bool up = (i & k) == 0, lower = (i & j) == 0;
+          const int lo = min(key[r], other), hi = max(key[r], other);
+          key[r] = (lower == up) ? lo : hi;
+        }
+      } else {
+        // in-lane pairs (r, r ^ j), each updated once from its lower slot
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = lane * 4 + r;
+          const bool up = (i & k) == 0, lower = (i & j) == 0;
+          if (lower) {
+            const int rr = r ^ j;
+            int a = key[r], b = j == 1 ? key[r ^ 1] : key[r ^ 2];
+            const int lo = min(a, b), hi = max(a, b);
+            a = up ? lo : hi;
+            b = up ? hi : lo;
+            key[r] = a;
+            if (rr == (r ^ 1) && j == 1) key[r ^ 1] = b;
+            else key[r ^ 2] = b;
+          }
+        }
+      }
+    }
+  }
+}
+
+// ids: T*k routed experts (shared memory); writes the union outputs, the plan
+// and zeroes the FFN counters, like block_union + block_plan.  Called by warp 0.
+__device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, int T, int S, int tokb,
+                                                int32_t* __restrict__ unique_ids, int32_t* __restrict__ n_unique,
+                                                int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
+                                                int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status,
+                                                int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
+                                                int32_t* __restrict__ rb_done, int n_rb, int lane) {
+  int key[4];
+  bool bad = false;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int p = lane * 4 + r;
+    key[r] = 0x7fffffff;
+    if (p < P) {
+      const int e = ids[p];
+      if (e < 0 || e >= E) bad = true;
+      else key[r] = (e << 8) | p;
+      pair_pos[p] = -1;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+  warp_bitonic_sort128(key, lane);
+  // segment starts: a valid key whose expert differs from the previous key's
+  const int prev_last = __shfl_up_sync(0xffffffffu, key[3], 1);
+  int flags = 0, nvalid = 0;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const bool valid = key[r] != 0x7fffffff;
+    const int prev = (r == 0) ? (lane == 0 ? -1 : prev_last) : key[r - 1];
+    const bool start = valid && (prev == -1 || (prev >> 8) != (key[r] >> 8));
+    flags |= (start ? 1 : 0) << r;
+    nvalid += valid ? 1 : 0;
+  }
+  int cnt = __popc(flags), incl = cnt, vincl = nvalid;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, incl, o), b = __shfl_up_sync(0xffffffffu, vincl, o);
+    if (lane >= o) {
+      incl += a;
+      vincl += b;
+    }
+  }
+  const int U = __shfl_sync(0xffffffffu, incl, 31);
+  const int Pv = __shfl_sync(0xffffffffu, vincl, 31);
+  int u = incl - cnt;
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = lane * 4 + r;
+    if (key[r] != 0x7fffffff) {
+      const int p = key[r] & 0xff;
+      perm[i] = p;
+      pair_pos[p] = i;
+      if (flags & (1 << r)) {
+        unique_ids[u] = key[r] >> 8;
+        seg_off[u] = i;
+        ++u;
+      }
+    }
+  }
+  if (lane == 0) {
+    *n_unique = U;
+    seg_off[U] = Pv;
+  }
+  __syncwarp();
+  // plan over S shared segments then U routed ones (U <= 128, S <= 4)
+  int nb[5], lsum = 0;
+#pragma unroll
+  for (int q = 0; q < 5; ++q) {
+    const int sidx = lane * 5 + q;
+    int v = 0;
+    if (sidx < S) {
+      v = (T + tokb - 1) / tokb;
+    } else if (sidx < S + U) {
+      const int uu = sidx - S;
+      const int c = ((uu + 1 < U) ? seg_off[uu + 1] : Pv) - seg_off[uu];
+      v = (c + tokb - 1) / tokb;
+    }
+    nb[q] = v;
+    lsum += v;
+  }
+  int lincl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, lincl, o);
+    if (lane >= o) lincl += a;
+  }
+  const int total = __shfl_sync(0xffffffffu, lincl, 31);
+  int run = lincl - lsum;
+  const int n_seg = U + S;
+#pragma unroll
+  for (int q = 0; q < 5; ++q) {
+    const int sidx = lane * 5 + q;
+    if (sidx < n_seg) plan[2 + sidx] = run;
+    run += nb[q];
+  }
+  if (lane == 0) {
+    plan[0] = n_seg;
+    plan[1] = total;
+    plan[2 + n_seg] = total;
+  }
+  for (int i = lane; i < total; i += 32) tb_done[i] = 0;
+  for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
+}
+
+// Route + union + plan for T*k <= 128: warp w routes tokens w, w + nwarps, ...;
+// then warp 0 alone builds the union and the plan.
+template <int NV>
+__global__ void __launch_bounds__(256) route_union_small_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    int32_t* __restrict__ ids_out, float* __restrict__ w_out, int32_t* __restrict__ unique_ids,
+    int32_t* __restrict__ n_unique, int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
+    int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status, int S, int tokb, int32_t* __restrict__ plan,
+    int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done, int n_rb) {
+  __shared__ int ids_s[kWarpUnionMaxP];
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int t = warp; t < T; t += nwarps) {
+    int id;
+    float w;
+    const bool bad = route_token<NV>(logits + static_cast<size_t>(t) * E, bias, E, k, lane, &id, &w);
+    if (lane < k) {
+      ids_s[t * k + lane] = id;
+      ids_out[static_cast<size_t>(t) * k + lane] = id;
+      w_out[static_cast<size_t>(t) * k + lane] = w;
+    }
+    if (bad && lane == 0) atomicOr(status, COLI_FLAG_NONFINITE);
+  }
+  if (nwarps > 1) __syncthreads();
+  else __syncwarp();
+  if (warp == 0)
+    warp_union_plan(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan, tb_done,
+                    rb_done, n_rb, lane);
+}
+
 }  // namespace coli
