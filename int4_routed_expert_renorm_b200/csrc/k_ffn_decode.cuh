@@ -73,14 +73,18 @@ struct StageCfg {
   static constexpr int TOKB = 8 * NT;
   static constexpr int GPW = KC / 64;                 // groups per warp per stage (two K-halves)
   static constexpr int ROWB = KC / 2;                 // code bytes per row
+  static constexpr int SUBS = KC >= 512 ? KC / 256 : 1;   // 128-byte-wide code sub-tiles per stage
+  static constexpr int RSTR = ROWB / SUBS;            // row stride inside a code sub-tile
+  static constexpr int SUB_BYTES = kRowBlock * RSTR;
   static constexpr int SROWB = KC / 16;               // scale bytes per row
   static constexpr int CODE_BYTES = kRowBlock * ROWB;
   static constexpr int SC_BYTES = kRowBlock * SROWB;
   static constexpr int W_BYTES = NMAT * (CODE_BYTES + SC_BYTES);
   static constexpr int XROW = KC * 2 + 64;            // padded activation row (bank-conflict free)
   static constexpr int STAGE_USED = W_BYTES + TOKB * XROW;
-  static constexpr bool SWZ = (KC == 256);
+  static constexpr bool SWZ = (KC >= 256);
   static_assert(CODE_BYTES % 1024 == 0 && SC_BYTES % 1024 == 0, "stage regions must stay 1 KiB aligned");
+  static_assert(NMAT == 1 || KC <= 256, "wide stages are for the down projection only");
 };
 
 template <int NT, int KCD>
@@ -274,7 +278,9 @@ __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& t
     uint8_t* st = smem + s * STAGE;
     if (lane == 0) {
       mbar_arrive_expect_tx(&full[s], C::W_BYTES + ti.ntok * KC * 2);
-      tma_load_2d(st, mq0, &full[s], kc * C::ROWB, row0);
+#pragma unroll
+      for (int sb = 0; sb < C::SUBS; ++sb)
+        tma_load_2d(st + sb * C::SUB_BYTES, mq0, &full[s], kc * C::ROWB + sb * C::RSTR, row0);
       if (NMAT == 2) tma_load_2d(st + C::CODE_BYTES, mq1, &full[s], kc * C::ROWB, row0);
       uint8_t* sc = st + NMAT * C::CODE_BYTES;
       if (KC == K) {
@@ -382,7 +388,7 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   // 128B swizzle the 16-byte chunk j of row r sits at chunk j ^ (r & 7), and
   // rl0 & 7 == (rl0 + 8) & 7 == g; bits 4..6 of cbase hold g, so chunk j is
   // cbase ^ (j << 4).
-  const uint32_t cbase = rl0 * C::ROWB + (C::SWZ ? (g << 4) : 0) + 4 * c;
+  const uint32_t cbase = rl0 * C::RSTR + (C::SWZ ? (g << 4) : 0) + 4 * c;
   const uint32_t sbase = rl0 * C::SROWB + half * C::GPW * 2;
   const uint32_t xbase = C::W_BYTES + g * C::XROW + (half * C::GPW * 32 + 8 * c) * 2;
   const int nnt = (ti.ntok + 7) >> 3;
@@ -401,8 +407,13 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
     const uint8_t* st = smem + s * STAGE;
     const uint8_t* sc = st + NMAT * C::CODE_BYTES + sbase;
     // this warp's fp16 scales for its GPW groups (rows rl0 and rl0 + 8, both matrices)
-    __half2 sh0[2], sh1[2], th0[2], th1[2];
-    if (C::GPW == 4) {
+    __half2 sh0[4], sh1[4], th0[4], th1[4];
+    if (C::GPW == 8) {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(sc);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(sc + 8 * C::SROWB);
+      sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y); sh0[2] = u32_as_half2(v0.z); sh0[3] = u32_as_half2(v0.w);
+      sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y); sh1[2] = u32_as_half2(v1.z); sh1[3] = u32_as_half2(v1.w);
+    } else if (C::GPW == 4) {
       const uint2 v0 = *reinterpret_cast<const uint2*>(sc);
       const uint2 v1 = *reinterpret_cast<const uint2*>(sc + 8 * C::SROWB);
       sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
@@ -428,9 +439,10 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
 #pragma unroll
     for (int jj = 0; jj < C::GPW; ++jj) {
       const int j = half * C::GPW + jj;                       // group within the stage
-      const uint8_t* ca = st + (cbase ^ static_cast<uint32_t>(j << 4));
+      const int jc = C::SUBS == 1 ? j : (j & 7);              // 16-byte chunk within the sub-tile row
+      const uint8_t* ca = st + (C::SUBS == 1 ? 0 : (j >> 3) * C::SUB_BYTES) + (cbase ^ static_cast<uint32_t>(jc << 4));
       const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
-      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::ROWB);
+      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::RSTR);
       const float s0 = half2_pick(sh0[jj >> 1], jj & 1);
       const float s1 = half2_pick(sh1[jj >> 1], jj & 1);
       uint32_t pg[8], pu[8];
@@ -438,7 +450,7 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
       float t0 = 0.f, t1 = 0.f;
       if (NMAT == 2) {
         const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
-        const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::ROWB);
+        const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::RSTR);
         t0 = half2_pick(th0[jj >> 1], jj & 1);
         t1 = half2_pick(th1[jj >> 1], jj & 1);
         dq_word_pair(pu, v0, v1);
