@@ -78,8 +78,11 @@ typedef enum {
 
 /* Layer flags (coli_moe_layer / coli_moe_expert_ffn). */
 #define COLI_LAYER_PRENORM       0x1u  /* route and run the experts on n = bf16(x * rsqrt(mean(x^2) + 1e-6)) */
-#define COLI_PATH_DECODE         0x10u /* force the CUDA-core/mma.sync decode FFN form */
-#define COLI_PATH_PREFILL        0x20u /* force the tcgen05 grouped-GEMM FFN form */
+#define COLI_PATH_DECODE         0x10u /* force the decode FFN form (weights streamed once, mma.sync) */
+#define COLI_PATH_PREFILL        0x20u /* force the prefill FFN form (tcgen05 grouped GEMM) */
+/* With neither flag the prefill form is taken when T >= 32 and T*k >= 32*min(E, T*k)
+ * (at least 32 tokens per expert on average), else the decode form.  Both flags
+ * together return COLI_ERR_INVALID_ARG. */
 
 typedef struct {
   int32_t hidden;     /* H */
@@ -176,7 +179,7 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
  *   - Arguments and results are those of coli_moe_layer, without ws/ws_bytes.
  *   - Batches whose coli_moe_workspace_bytes(dims, T) exceeds
  *     COLI_NOALLOC_SCRATCH_BYTES are rejected with COLI_ERR_WORKSPACE before
- *     anything is launched (up to 29 tokens for H=6144, I=2048, E=256, k=8, S=1).
+ *     anything is launched (up to 21 tokens for H=6144, I=2048, E=256, k=8, S=1).
  *   - The first call on a device looks up the array's device address (one
  *     cudaGetSymbolAddress with that device current); make that first call
  *     before capturing a stream.  No call allocates or frees device memory.

@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "k_ffn_decode.cuh"
+#include "k_ffn_prefill.cuh"
 #include "k_router.cuh"
 #include "k_union.cuh"
 
@@ -87,7 +88,13 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_SMEM(1, true, 128)
     COLI_SET_SMEM(1, false, 128)
     COLI_SET_SMEM(4, false, 128)
+    COLI_SET_SMEM(1, true, 512)
+    COLI_SET_SMEM(1, false, 512)
 #undef COLI_SET_SMEM
+    ok &= cudaFuncSetAttribute(ffn_prefill_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PfCfg<2>::SMEM)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(ffn_prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PfCfg<1>::SMEM)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
     const int ru_smem = (kUnionWarps * 1024 + kFusedRouteMaxT * 32) * 4;
@@ -163,6 +170,7 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout for T tokens (every region 256-byte aligned).
 struct Ws {
+  uint16_t* xg;      // [P][H] expert input gathered into pair order (prefill form), directly followed by xq
   uint16_t* xq;      // [T][H] fragment-ordered expert input
   uint16_t* xn;      // [T][H] normalised input (prenorm)
   float* logits;     // [T][E]
@@ -194,7 +202,8 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
     o += align256(bytes);
     return p;
   };
-  ws.xq = static_cast<uint16_t*>(take(T * H * 2));
+  ws.xg = static_cast<uint16_t*>(take((P + static_cast<size_t>(T)) * H * 2));
+  ws.xq = ws.xg ? ws.xg + P * H : nullptr;
   ws.xn = static_cast<uint16_t*>(take(T * H * 2));
   ws.logits = static_cast<float*>(take(T * E * 4));
   ws.ids = static_cast<int32_t*>(take(P * 4));
@@ -231,8 +240,10 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 // [rows_total][K/32] fp16, tiles of 128 rows x KC elements.
 bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, CUtensorMap* mq,
                  CUtensorMap* ms) {
-  const CUtensorMapSwizzle swz = KC == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, KC / 2, kRowBlock, swz))
+  // stages of 512 K move their codes as two 128-byte-wide boxes
+  const CUtensorMapSwizzle swz = KC >= 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, KC >= 256 ? 128 : KC / 2, kRowBlock,
+                 swz))
     return false;
   if (KC < K) {
     if (!encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / 32, rows_total, (K / 32) * 2, KC / 32, kRowBlock,
@@ -330,6 +341,127 @@ bool launch_route_union(const float* lg, const float* bias, int T, int E, int k,
 #undef COLI_RU
 }
 
+// FFN form for this call: the tcgen05 grouped GEMM when forced, or by default
+// once the batch averages >= 32 tokens per expert of the union's upper bound.
+enum class Form { kDecode, kPrefill, kInvalid };
+
+Form choose_form(uint32_t flags, int T, int E, int k) {
+  const bool fd = (flags & COLI_PATH_DECODE) != 0, fp = (flags & COLI_PATH_PREFILL) != 0;
+  if (fd && fp) return Form::kInvalid;
+  if (fd) return Form::kDecode;
+  if (fp) return Form::kPrefill;
+  const long P = static_cast<long>(T) * k;
+  const long U = P < E ? P : E;
+  return (T >= kPfAutoMinT && P >= 32 * U) ? Form::kPrefill : Form::kDecode;
+}
+
+// Tensor maps of the prefill form: codes [rows][K/2] bytes in boxes of 128
+// rows x cps*32 bytes (128B / 64B swizzle), scales [rows][K/32] fp16 in boxes
+// of 128 rows x cps*2 (unless one stage spans K), token rows [rows][K] bf16 in
+// boxes of 16 rows x 64 elements (128B swizzle).
+bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, CUtensorMap* mq,
+                    CUtensorMap* ms) {
+  const int cps = (K % 256 == 0) ? 4 : 2;
+  const CUtensorMapSwizzle swz = cps == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, cps * 32, kRowBlock, swz))
+    return false;
+  if (K == cps * 64) {
+    std::memset(ms, 0, sizeof(*ms));
+    return true;
+  }
+  return encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / 32, rows_total, (K / 32) * 2, cps * 2, kRowBlock,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int NMAT>
+bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = PfCfg<NMAT>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ++t_launches;
+  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT>, m[0], m[1], m[2], m[3], m[4], a) == cudaSuccess;
+}
+
+// Prefill form: gather the expert input into pair order, plan the token
+// blocks, gate/up GEMM (h), down GEMM (y), combine.
+coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
+                            const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm,
+                            const int32_t* pair_pos, const float* topk_w, const uint16_t* residual, uint16_t* out,
+                            const Ws& ws, const DevInfo& di, cudaStream_t st, const StageRecorder& rec) {
+  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
+  const int P = T * k;
+  const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
+  const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
+  CUtensorMap mg[5], md[5];   // q0, q1, s0, s1, token rows
+  if (!pf_weight_maps(w->gate_q, w->gate_s, rows_gu, H, &mg[0], &mg[2]) ||
+      !pf_weight_maps(w->up_q, w->up_s, rows_gu, H, &mg[1], &mg[3]) ||
+      !encode_2d(&mg[4], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.xg, H, static_cast<uint64_t>(P) + T,
+                 static_cast<uint64_t>(H) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !pf_weight_maps(w->down_q, w->down_s, rows_dn, I, &md[0], &md[2]) ||
+      !encode_2d(&md[4], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.hq, I, static_cast<uint64_t>(P) + static_cast<uint64_t>(S) * T,
+                 static_cast<uint64_t>(I) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return COLI_ERR_CUDA;
+  md[1] = md[0];
+  md[3] = md[2];
+
+  {
+    long blocks = (P + 7) / 8;
+    if (blocks > 8L * di.sms) blocks = 8L * di.sms;
+    if (!launch(gather_rows_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st,
+                static_cast<const uint16_t*>(ws.xq), perm, k, P, H, ws.xg))
+      return COLI_ERR_CUDA;
+  }
+  if (!launch(pf_plan_kernel, dim3(1), dim3(1024), 0, st, n_unique, seg_off, T, S, ws.plan)) return COLI_ERR_CUDA;
+  rec.mark(5);
+
+  PfArgs a{};
+  a.plan = ws.plan;
+  a.unique_ids = unique;
+  a.n_unique = n_unique;
+  a.seg_off = seg_off;
+  a.hq = ws.hq;
+  a.ypair = ws.ypair;
+  a.status = di.status;
+  a.H = H;
+  a.I = I;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.S = S;
+  a.P = P;
+  const int Umax = P < E ? P : E;
+  const long blocks_ub = static_cast<long>(Umax) + P / kPfMaxN + static_cast<long>(S) * (T / kPfMaxN + 1);
+  auto grid_for = [&](int mb) {
+    const long tiles = blocks_ub * mb;
+    return static_cast<int>(tiles < di.sms ? tiles : di.sms);
+  };
+  a.s0 = w->gate_s;
+  a.s1 = w->up_s;
+  if (!launch_prefill<2>(mg, a, grid_for(I / kRowBlock), st)) return COLI_ERR_CUDA;
+  rec.mark(6);
+  a.s0 = w->down_s;
+  a.s1 = w->down_s;
+  if (!launch_prefill<1>(md, a, grid_for(H / kRowBlock), st)) return COLI_ERR_CUDA;
+  rec.mark(7);
+  {
+    const long work = static_cast<long>(T) * (H / 4);
+    long blocks = (work + 255) / 256;
+    if (blocks > 4L * di.sms) blocks = 4L * di.sms;
+    if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
+                pair_pos, topk_w, residual, T, k, S, H, out))
+      return COLI_ERR_CUDA;
+  }
+  rec.mark(8);
+  return COLI_OK;
+}
+
 // The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer;
 // the tile plan (ws.plan) must already be on the stream.
 coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
@@ -347,7 +479,9 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   const long blocks_ub = static_cast<long>(Umax) + P / tokb + static_cast<long>(S) * ((T + tokb - 1) / tokb);
 
   CUtensorMap maps[6];   // gate q, up q, gate s, up s, down q, down s
-  const int kc_dn = (I % 256 == 0) ? 256 : 128;
+  // down stages: 512 K (two 128-byte code boxes) for the one-n-tile forms,
+  // whose activation slice per stage stays small
+  const int kc_dn = (I % 512 == 0 && T <= 8) ? 512 : (I % 256 == 0) ? 256 : 128;
   if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, &maps[0], &maps[2]) ||
       !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, &maps[1], &maps[3]) ||
       !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, &maps[4], &maps[5]))
@@ -382,7 +516,11 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   {
     const long tiles = blocks_ub * (I / kRowBlock + H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    const bool ok = kc_dn == 256 ? launch_ffn_for<256>(T, maps, a, grid, st) : launch_ffn_for<128>(T, maps, a, grid, st);
+    bool ok;
+    if (kc_dn == 512)
+      ok = T == 1 ? launch_ffn_fused<1, true, 512>(maps, a, grid, st) : launch_ffn_fused<1, false, 512>(maps, a, grid, st);
+    else
+      ok = kc_dn == 256 ? launch_ffn_for<256>(T, maps, a, grid, st) : launch_ffn_for<128>(T, maps, a, grid, st);
     if (!ok) return COLI_ERR_CUDA;
   }
   rec.mark_through(6, 7);
@@ -478,7 +616,8 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
     return COLI_ERR_INVALID_ARG;
   if (x == out) return COLI_ERR_INVALID_ARG;
-  if (flags & COLI_PATH_PREFILL) return COLI_ERR_UNSUPPORTED;
+  const Form form = choose_form(flags, T, dims->n_experts, dims->top_k);
+  if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
   DevInfo di;
@@ -489,6 +628,9 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq))
     return COLI_ERR_CUDA;
   rec.mark_through(1, 4);
+  if (form == Form::kPrefill)
+    return run_ffn_prefill(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di,
+                           s, rec);
   if (!launch(plan_kernel, dim3(1), dim3(1024), 0, s, n_unique, seg_off, T, dims->n_shared, tok_block(T), lay.plan,
               lay.tb_done, lay.rb_done, dims->hidden / kRowBlock))
     return COLI_ERR_CUDA;
@@ -510,7 +652,8 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
     return COLI_ERR_INVALID_ARG;
   if (x == out) return COLI_ERR_INVALID_ARG;
-  if (flags & COLI_PATH_PREFILL) return COLI_ERR_UNSUPPORTED;
+  const Form form = choose_form(flags, T, dims->n_experts, dims->top_k);
+  if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
   DevInfo di;
@@ -566,6 +709,9 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
     rec.mark_through(4, 5);
   }
   // 3. expert FFN and combine
+  if (form == Form::kPrefill)
+    return run_ffn_prefill(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual,
+                           out, lay, di, s, rec);
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
                  di, s, rec);
 }

@@ -168,7 +168,11 @@ STACK16_B4 = LayerShape("glm52_stack16_decode_b4", 6144, 2048, 256, 8, 1, 4, lay
 # Same per-step bytes as DECODE_B1 (8 routed + 1 shared expert, 191 MB > L2) with
 # only 16 routed experts resident: small enough for profiler captures.
 DECODE_B1_E16 = LayerShape("glm52_layer_decode_b1_e16", 6144, 2048, 16, 8, 1, 1)
-WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16)}
+# Prefill tiles of the same shape as PREFILL_4096 (~128 tokens on every expert;
+# 32 routed + 1 shared expert resident, 0.7 GB): for profiler captures.
+PREFILL_512_E32 = LayerShape("glm52_layer_prefill_512_e32", 6144, 2048, 32, 8, 1, 512, logits_in=True)
+WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16,
+                                 PREFILL_512_E32)}
 
 
 class LayerInputs:
