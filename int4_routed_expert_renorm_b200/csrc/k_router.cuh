@@ -266,10 +266,6 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
 }
 
 // (value, index) order of the router: larger value first, then lower index.
-__device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
-}
-
 // Route one token with one warp: top-k over E <= 32*NV logits (+ bias) and
 // the renormalised softmax weights.  Lane l holds experts l, l+32, ...
 // Slot j receives the j-th expert in (value desc, index asc) order and
@@ -295,35 +291,37 @@ __device__ __forceinline__ bool route_token(const float* __restrict__ lr, const 
       } else if (isinf(val) && val > 0.f) {
         bad = true;
       }
+      if (val == 0.f) val = 0.f;   // -0.0 ties +0.0
     } else {
       taken |= 1u << q;  // padding never selected
     }
     v[q] = val;
   }
+  // Each round: every lane offers its best untaken value as an order-preserving
+  // integer (larger value -> larger key; -0.0 was folded into +0.0 above),
+  // the warp takes the maximum key and, among lanes holding it, the lowest
+  // expert index -- two redux.sync reductions instead of a shuffle tree.
+  uint32_t ord[NV];
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const uint32_t u = __float_as_uint(v[q]);
+    ord[q] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
   float l_max = 0.f, my_v = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = 0.f;
-    int bi = 0x7fffffff;
+    uint32_t lo = 0u;            // below every real key (-inf maps to 0x007FFFFF)
+    int le = 0x7fffffff;
 #pragma unroll
-    for (int q = 0; q < NV; ++q) {
-      if (!(taken & (1u << q))) {
-        const int e = lane + 32 * q;
-        if (bi == 0x7fffffff || route_better(v[q], e, bv, bi)) {
-          bv = v[q];
-          bi = e;
-        }
+    for (int q = 0; q < NV; ++q)
+      if (!(taken & (1u << q)) && ord[q] > lo) {   // strict: the lower index wins ties inside a lane
+        lo = ord[q];
+        le = lane + 32 * q;
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || route_better(ov, oi, bv, bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lo);
+    const int bi = __reduce_min_sync(0xffffffffu, lo == m ? le : 0x7fffffff);
+    const uint32_t bu = (m & 0x80000000u) ? (m & 0x7fffffffu) : ~m;
+    const float bv = __uint_as_float(bu);
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (j == 0) l_max = bv;
     if (lane == j) {

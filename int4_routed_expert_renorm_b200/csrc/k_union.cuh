@@ -383,6 +383,78 @@ __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, in
   for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
 }
 
+// The same for T*k <= 32, one key per lane: a 32-wide bitonic sort (15
+// shuffle stages), segment starts by ballot, and the plan's per-segment block
+// counts from the distance to the next segment start -- no global reads back.
+__device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, int T, int S, int tokb,
+                                                  int32_t* __restrict__ unique_ids, int32_t* __restrict__ n_unique,
+                                                  int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
+                                                  int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status,
+                                                  int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
+                                                  int32_t* __restrict__ rb_done, int n_rb, int lane) {
+  int key = 0x7fffffff;
+  bool bad = false;
+  if (lane < P) {
+    const int e = ids[lane];
+    if (e < 0 || e >= E) bad = true;
+    else key = (e << 8) | lane;
+    pair_pos[lane] = -1;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int other = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+      key = (lower == up) ? min(key, other) : max(key, other);
+    }
+  }
+  const bool valid = key != 0x7fffffff;
+  const int prev = __shfl_up_sync(0xffffffffu, key, 1);
+  const bool start = valid && (lane == 0 || (prev >> 8) != (key >> 8));
+  const uint32_t smask = __ballot_sync(0xffffffffu, start);
+  const int Pv = __popc(__ballot_sync(0xffffffffu, valid));
+  const int U = __popc(smask);
+  const int u = __popc(smask & ((1u << lane) - 1u));
+  // pairs of the segment starting here: up to the next start (or the end)
+  const uint32_t later = lane == 31 ? 0u : (smask & ~((2u << lane) - 1u));
+  const int cnt = start ? (later ? __ffs(later) - 1 : Pv) - lane : 0;
+  __syncwarp();   // the -1 stores above come before the pair_pos stores below
+  if (valid) {
+    const int p = key & 0xff;
+    perm[lane] = p;
+    pair_pos[p] = lane;
+    if (start) {
+      unique_ids[u] = key >> 8;
+      seg_off[u] = lane;
+    }
+  }
+  // plan: S shared segments of T tokens, then the U routed ones in order
+  const int nb_shared = (T + tokb - 1) / tokb;
+  int nb = start ? (cnt + tokb - 1) / tokb : 0;
+  int incl = nb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += a;
+  }
+  const int routed_total = __shfl_sync(0xffffffffu, incl, 31);
+  const int total = S * nb_shared + routed_total;
+  const int n_seg = U + S;
+  if (start) plan[2 + S + u] = S * nb_shared + incl - nb;
+  if (lane < S) plan[2 + lane] = lane * nb_shared;
+  if (lane == 0) {
+    *n_unique = U;
+    seg_off[U] = Pv;
+    plan[0] = n_seg;
+    plan[1] = total;
+    plan[2 + n_seg] = total;
+  }
+  for (int i = lane; i < total; i += 32) tb_done[i] = 0;
+  for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
+}
+
 // Route + union + plan for T*k <= 128: warp w routes tokens w, w + nwarps, ...;
 // then warp 0 alone builds the union and the plan.
 template <int NV>
@@ -409,9 +481,14 @@ __global__ void __launch_bounds__(256) route_union_small_kernel(
   }
   if (nwarps > 1) __syncthreads();
   else __syncwarp();
-  if (warp == 0)
-    warp_union_plan(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan, tb_done,
-                    rb_done, n_rb, lane);
+  if (warp == 0) {
+    if (T * k <= 32)
+      warp_union_plan32(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan,
+                        tb_done, rb_done, n_rb, lane);
+    else
+      warp_union_plan(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan,
+                      tb_done, rb_done, n_rb, lane);
+  }
 }
 
 }  // namespace coli
