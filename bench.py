@@ -63,6 +63,14 @@ def parse():
     return a
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture
+# of the same kernel build: (workload, FFN form) -> bytes.  The batch-1 capture
+# ran on the 16-expert variant of the layer, which moves the same 9 experts per
+# step (profiles/ffn_fused_kernel_glm52_layer_decode_b1_e16.md).
+TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.752704e6 + 4.751616e6,
+           ("glm52_layer_decode_b1_e16", "decode"): 191.752704e6 + 4.751616e6}
+
+
 def prefill_form(shape) -> bool:
     """The library takes the prefill (tcgen05) form once a batch averages >= 32
     tokens per expert; the prefill workloads are the ones that do."""
@@ -360,6 +368,8 @@ def main():
                 "algorithmic": "int4 codes + fp16 scales of every unique and shared expert (3 matrices) "
                                "+ x read + h write/read + y write" + (" + y read + out write" if fused_combine else ""),
                 "peak_kind": f"{src} HBM copy"}
+
+    roof["traffic"] = TRAFFIC.get((shape.name, form))
 
     # int4 bytes touched per step (all three matrices of every unique + shared expert)
     exp_bytes = shape.expert_bytes()

@@ -358,7 +358,7 @@ Form choose_form(uint32_t flags, int T, int E, int k) {
 // Tensor maps of the prefill form: codes [rows][K/2] bytes in boxes of 128
 // rows x cps*32 bytes (128B / 64B swizzle), scales [rows][K/32] fp16 in boxes
 // of 128 rows x cps*2 (unless one stage spans K), token rows [rows][K] bf16 in
-// boxes of 16 rows x 64 elements (128B swizzle).
+// boxes of 128/64/32/16 rows x 64 elements (128B swizzle).
 bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, CUtensorMap* mq,
                     CUtensorMap* ms) {
   const int cps = (K % 256 == 0) ? 4 : 2;
@@ -386,7 +386,8 @@ bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ++t_launches;
-  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT>, m[0], m[1], m[2], m[3], m[4], a) == cudaSuccess;
+  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT>, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a) ==
+         cudaSuccess;
 }
 
 // Prefill form: gather the expert input into pair order, plan the token
@@ -399,15 +400,20 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   const int P = T * k;
   const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
   const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
-  CUtensorMap mg[5], md[5];   // q0, q1, s0, s1, token rows
+  CUtensorMap mg[8], md[8];   // q0, q1, s0, s1, token rows in boxes of 128, 64, 32, 16 rows
   if (!pf_weight_maps(w->gate_q, w->gate_s, rows_gu, H, &mg[0], &mg[2]) ||
       !pf_weight_maps(w->up_q, w->up_s, rows_gu, H, &mg[1], &mg[3]) ||
-      !encode_2d(&mg[4], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.xg, H, static_cast<uint64_t>(P) + T,
-                 static_cast<uint64_t>(H) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !pf_weight_maps(w->down_q, w->down_s, rows_dn, I, &md[0], &md[2]) ||
-      !encode_2d(&md[4], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.hq, I, static_cast<uint64_t>(P) + static_cast<uint64_t>(S) * T,
-                 static_cast<uint64_t>(I) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+      !pf_weight_maps(w->down_q, w->down_s, rows_dn, I, &md[0], &md[2]))
     return COLI_ERR_CUDA;
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t box = 128u >> j;
+    if (!encode_2d(&mg[4 + j], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.xg, H, static_cast<uint64_t>(P) + T,
+                   static_cast<uint64_t>(H) * 2, 64, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&md[4 + j], CU_TENSOR_MAP_DATA_TYPE_UINT16, ws.hq, I,
+                   static_cast<uint64_t>(P) + static_cast<uint64_t>(S) * T, static_cast<uint64_t>(I) * 2, 64, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return COLI_ERR_CUDA;
+  }
   md[1] = md[0];
   md[3] = md[2];
 

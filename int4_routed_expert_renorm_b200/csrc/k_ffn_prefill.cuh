@@ -249,7 +249,8 @@ template <int NMAT>
 __global__ void __launch_bounds__(kPfThreads, 1)
     ffn_prefill_kernel(const __grid_constant__ CUtensorMap mq0, const __grid_constant__ CUtensorMap mq1,
                        const __grid_constant__ CUtensorMap ms0, const __grid_constant__ CUtensorMap ms1,
-                       const __grid_constant__ CUtensorMap mb, PfArgs a) {
+                       const __grid_constant__ CUtensorMap mb128, const __grid_constant__ CUtensorMap mb64,
+                       const __grid_constant__ CUtensorMap mb32, const __grid_constant__ CUtensorMap mb16, PfArgs a) {
   using C = PfCfg<NMAT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -292,7 +293,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&mq0);
     if (NMAT == 2) prefetch_tensormap(&mq1);
-    prefetch_tensormap(&mb);
+    prefetch_tensormap(&mb128);
+    prefetch_tensormap(&mb16);
   }
   if (warp == 1) tmem_alloc(tmem_slot, kPfTmemCols);
   pdl_wait();
@@ -329,7 +331,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
         const int row0 = ti.e * R + ti.rblk * kRowBlock;
-        const int nbox = ti.npad >> 4;
         for (int kb = 0; ok && kb < nk; ++kb) {
           if (kb % cps == 0) {
             const int cs = static_cast<int>(cst % C::NSC);
@@ -353,8 +354,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int s = static_cast<int>(bit % C::NSB);
           if (!(ok = mbar_wait(&b_empty[s], ((bit / C::NSB) & 1u) ^ 1u, abort_flag, a.status))) break;
           uint8_t* dst = bst_base + s * C::BSTAGE;
-          mbar_arrive_expect_tx(&b_full[s], nbox * 2048);
-          for (int j = 0; j < nbox; ++j) tma_load_2d(dst + j * 2048, &mb, &b_full[s], kb * 64, ti.brow + j * 16);
+          mbar_arrive_expect_tx(&b_full[s], ti.npad * 128);
+          // the token tile in as few boxes as possible (128/64/32/16 rows): the TMA
+          // engine's cost per box is large next to its cost per row
+          int row = ti.brow, rem = ti.npad;
+          uint8_t* d = dst;
+          for (; rem >= 128; rem -= 128, row += 128, d += 128 * 128) tma_load_2d(d, &mb128, &b_full[s], kb * 64, row);
+          if (rem >= 64) { tma_load_2d(d, &mb64, &b_full[s], kb * 64, row); rem -= 64; row += 64; d += 64 * 128; }
+          if (rem >= 32) { tma_load_2d(d, &mb32, &b_full[s], kb * 64, row); rem -= 32; row += 32; d += 32 * 128; }
+          if (rem >= 16) tma_load_2d(d, &mb16, &b_full[s], kb * 64, row);
           ++bit;
         }
       }
