@@ -31,7 +31,8 @@ namespace coli {
 
 constexpr int kPfTeams = 2;       // dequantisation teams of 8 warps; team t takes chunks t, t+2, ...
 constexpr int kPfDqWarps = 8 * kPfTeams;
-constexpr int kPfThreads = (4 + kPfDqWarps) * 32;   // warp 0 TMA, warp 1 MMA + TMEM owner, warps 4.. dequant + epilogue
+constexpr int kPfThreads = (4 + kPfDqWarps) * 32;   // warp 0 weight TMA, warp 1 MMA + TMEM owner, warp 2 token
+                                                    // TMA, warps 4.. dequant + epilogue
 constexpr int kPfMaxN = 160;      // tokens per tile (MMA N is this rounded up to 16)
 constexpr int kPfAutoMinT = 32;   // smallest batch for which the form is chosen by default
 constexpr int kPfTmemCols = 512;
@@ -57,12 +58,14 @@ struct PfCfg {
   static constexpr int SC_SLOT = kRowBlock * 16;                    // scales of one matrix, 4 chunks
   static constexpr int CSTAGE = NMAT * (CODE_SLOT + SC_SLOT);
   static constexpr int BSTAGE = kPfMaxN * 128;                      // token tile of one chunk
-  static constexpr int NSC = NMAT == 2 ? 3 : 4;
-  static constexpr int NSB = NMAT == 2 ? 4 : 5;
-  static constexpr int NBUF = NMAT == 2 ? 3 : 6;                    // A buffers in TMEM
+  // A chunk slot = one A buffer in TMEM + one token-tile stage in shared
+  // memory, released together by one tcgen05.commit.
+  static constexpr int NSC = 4;
+  static constexpr int NBUF = NMAT == 2 ? 3 : 6;                    // chunk slots
+  static constexpr int NSB = NBUF;
   static constexpr int ACOL = NMAT * kPfMaxN;                       // first A column
   static constexpr int META_INTS = 3 * kMaxSeg + 4;
-  static constexpr int NBAR = 2 * NSC + 2 * NSB + 2 * NBUF + 3;
+  static constexpr int NBAR = 2 * NSC + NSB + 2 * NBUF + 3;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(NSC) * CSTAGE + static_cast<size_t>(NSB) * BSTAGE +
                                  META_INTS * 4 + NBAR * 8 + 16;
   static_assert(CSTAGE % 1024 == 0 && BSTAGE % 1024 == 0, "stage alignment");
@@ -261,10 +264,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* code_full = bars;
   uint64_t* code_empty = code_full + C::NSC;
   uint64_t* b_full = code_empty + C::NSC;
-  uint64_t* b_empty = b_full + C::NSB;
-  uint64_t* a_full = b_empty + C::NSB;
-  uint64_t* a_empty = a_full + C::NBUF;
-  uint64_t* acc_full = a_empty + C::NBUF;
+  uint64_t* a_full = b_full + C::NSB;
+  uint64_t* slot_empty = a_full + C::NBUF;   // chunk slot consumed by the MMAs (A buffer + token stage)
+  uint64_t* acc_full = slot_empty + C::NBUF;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -278,11 +280,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int q = 0; q < C::NSB; ++q) {
       mbar_init(&b_full[q], 1);
-      mbar_init(&b_empty[q], 1);
     }
     for (int q = 0; q < C::NBUF; ++q) {
       mbar_init(&a_full[q], 8);
-      mbar_init(&a_empty[q], 1);
+      mbar_init(&slot_empty[q], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kPfDqWarps);
@@ -293,6 +294,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&mq0);
     if (NMAT == 2) prefetch_tensormap(&mq1);
+  }
+  if (warp == 2 && lane == 0) {
     prefetch_tensormap(&mb128);
     prefetch_tensormap(&mb16);
   }
@@ -324,35 +327,53 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int tiles = total_blocks * mbk;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // -------------------------------------------------- weight producer
+    // Codes and scales run up to NSC stages (4 chunks each) ahead, paced only
+    // by the dequantisation warps -- never by the MMA's token stages.
     if (lane == 0) {
-      uint32_t cst = 0, bit = 0;
+      uint32_t cst = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
         const int row0 = ti.e * R + ti.rblk * kRowBlock;
-        for (int kb = 0; ok && kb < nk; ++kb) {
-          if (kb % cps == 0) {
-            const int cs = static_cast<int>(cst % C::NSC);
-            if (!(ok = mbar_wait(&code_empty[cs], ((cst / C::NSC) & 1u) ^ 1u, abort_flag, a.status))) break;
-            uint8_t* dst = cst_base + cs * C::CSTAGE;
-            mbar_arrive_expect_tx(&code_full[cs], NMAT * kRowBlock * cps * 36);
-            tma_load_2d(dst, &mq0, &code_full[cs], kb * 32, row0);
-            if (NMAT == 2) tma_load_2d(dst + C::CODE_SLOT, &mq1, &code_full[cs], kb * 32, row0);
-            uint8_t* sdst = dst + NMAT * C::CODE_SLOT;
-            if (one_stage) {
-              bulk_load(sdst, a.s0 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4, &code_full[cs]);
-              if (NMAT == 2)
-                bulk_load(sdst + C::SC_SLOT, a.s1 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4,
-                          &code_full[cs]);
-            } else {
-              tma_load_2d(sdst, &ms0, &code_full[cs], kb * 2, row0);
-              if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, &ms1, &code_full[cs], kb * 2, row0);
-            }
-            ++cst;
+        for (int kb = 0; ok && kb < nk; kb += cps) {
+          const int cs = static_cast<int>(cst % C::NSC);
+          if (!(ok = mbar_wait(&code_empty[cs], ((cst / C::NSC) & 1u) ^ 1u, abort_flag, a.status))) break;
+          uint8_t* dst = cst_base + cs * C::CSTAGE;
+          mbar_arrive_expect_tx(&code_full[cs], NMAT * kRowBlock * cps * 36);
+          tma_load_2d(dst, &mq0, &code_full[cs], kb * 32, row0);
+          if (NMAT == 2) tma_load_2d(dst + C::CODE_SLOT, &mq1, &code_full[cs], kb * 32, row0);
+          uint8_t* sdst = dst + NMAT * C::CODE_SLOT;
+          if (one_stage) {
+            bulk_load(sdst, a.s0 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4, &code_full[cs]);
+            if (NMAT == 2)
+              bulk_load(sdst + C::SC_SLOT, a.s1 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4,
+                        &code_full[cs]);
+          } else {
+            tma_load_2d(sdst, &ms0, &code_full[cs], kb * 2, row0);
+            if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, &ms1, &code_full[cs], kb * 2, row0);
           }
+          ++cst;
+        }
+      }
+      if (!ok) {
+        // bounded wait (ignoring the abort flag) for the copies still in flight
+        int dummy = 0;
+        for (uint32_t q = cst > C::NSC ? cst - C::NSC : 0; q < cst; ++q)
+          mbar_wait(&code_full[q % C::NSC], (q / C::NSC) & 1u, reinterpret_cast<volatile int*>(&dummy), a.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------- token-tile producer
+    if (lane == 0) {
+      uint32_t bit = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
+        for (int kb = 0; ok && kb < nk; ++kb) {
           const int s = static_cast<int>(bit % C::NSB);
-          if (!(ok = mbar_wait(&b_empty[s], ((bit / C::NSB) & 1u) ^ 1u, abort_flag, a.status))) break;
+          if (!(ok = mbar_wait(&slot_empty[s], ((bit / C::NSB) & 1u) ^ 1u, abort_flag, a.status))) break;
           uint8_t* dst = bst_base + s * C::BSTAGE;
           mbar_arrive_expect_tx(&b_full[s], ti.npad * 128);
           // the token tile in as few boxes as possible (128/64/32/16 rows): the TMA
@@ -367,10 +388,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       if (!ok) {
-        // bounded wait (ignoring the abort flag) for the copies still in flight
         int dummy = 0;
-        for (uint32_t q = cst > C::NSC ? cst - C::NSC : 0; q < cst; ++q)
-          mbar_wait(&code_full[q % C::NSC], (q / C::NSC) & 1u, reinterpret_cast<volatile int*>(&dummy), a.status);
         for (uint32_t q = bit > C::NSB ? bit - C::NSB : 0; q < bit; ++q)
           mbar_wait(&b_full[q % C::NSB], (q / C::NSB) & 1u, reinterpret_cast<volatile int*>(&dummy), a.status);
       }
@@ -401,8 +419,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int m = 0; m < NMAT; ++m)
               mma_bf16_ts(tbase + m * kPfMaxN, acol + m * 32 + kk * 8, bdesc, idesc, (kb | kk) != 0);
           }
-          tc_commit(&a_empty[b]);
-          tc_commit(&b_empty[s]);
+          tc_commit(&slot_empty[b]);   // b == s: the slot's A buffer and token stage
           ++it;
           ++bit;
         }
@@ -464,7 +481,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (lane == 0) mbar_arrive(&code_empty[cs]);
         }
         const int b = static_cast<int>(it % C::NBUF);
-        if (!(ok = warp_wait(&a_empty[b], ((it / C::NBUF) & 1u) ^ 1u, abort_flag, a.status))) break;
+        if (!(ok = warp_wait(&slot_empty[b], ((it / C::NBUF) & 1u) ^ 1u, abort_flag, a.status))) break;
         tc_fence_after();
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
