@@ -97,6 +97,8 @@ coli_status dev_info(DevInfo* out) {
                                static_cast<int>(PfCfg<1>::SMEM)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(union_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kUnionWarps * 1024 * 4) == cudaSuccess;
     const int ru_smem = (kUnionWarps * 1024 + kFusedRouteMaxT * 32) * 4;
     ok &= cudaFuncSetAttribute(route_union_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
     ok &= cudaFuncSetAttribute(route_union_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, ru_smem) == cudaSuccess;
@@ -181,6 +183,7 @@ struct Ws {
   int32_t* seg_off;  // [min(E,P)+1]
   int32_t* perm;     // [P]
   int32_t* pair_pos; // [P]
+  int32_t* ucnt;     // [ceil(P / union_chunk(P))][E] per-chunk expert counts of the many-CTA union
   int32_t* plan;     // [min(E,P)+S+3]
   int32_t* tb_done;  // [token blocks upper bound] gate/up completion per token block
   int32_t* rb_done;  // [H/128] down completion per output row block
@@ -213,6 +216,10 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
   ws.seg_off = static_cast<int32_t*>(take((Umax + 1) * 4));
   ws.perm = static_cast<int32_t*>(take(P * 4));
   ws.pair_pos = static_cast<int32_t*>(take(P * 4));
+  {
+    const size_t chunk = static_cast<size_t>(union_chunk(static_cast<int>(P)));
+    ws.ucnt = static_cast<int32_t*>(take((P + chunk - 1) / chunk * E * 4));
+  }
   ws.plan = static_cast<int32_t*>(take((Umax + S + 3) * 4));
   {
     const size_t tokb = T <= 8 ? 8 : 32;
@@ -708,10 +715,23 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   } else {
     if (!launch_route(lg, w->router_bias, T, E, k, ids, tw, di.status, s)) return COLI_ERR_CUDA;
     rec.mark(3);
-    if (!launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4, s,
-                static_cast<const int32_t*>(ids), T * k, E, lay.unique, lay.n_unique, lay.seg_off, lay.perm,
-                lay.pair_pos, di.status, T, S, tokb, lay.plan, lay.tb_done, lay.rb_done, H / kRowBlock))
+    const int P = T * k;
+    if (form == Form::kPrefill) {
+      // many-CTA union; the prefill form computes its own tile plan afterwards
+      const int chunk = union_chunk(P), NB = (P + chunk - 1) / chunk;
+      const int32_t* cids = ids;
+      if (!launch(union_count_kernel, dim3(NB), dim3(1024), static_cast<size_t>(E) * 4, s, cids, P, E, chunk, lay.ucnt,
+                  di.status) ||
+          !launch(union_scan_kernel, dim3(1), dim3(1024), 0, s, lay.ucnt, NB, E, lay.unique, lay.n_unique,
+                  lay.seg_off) ||
+          !launch(union_scatter_kernel, dim3(NB), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4, s,
+                  cids, P, E, chunk, static_cast<const int32_t*>(lay.ucnt), lay.perm, lay.pair_pos))
+        return COLI_ERR_CUDA;
+    } else if (!launch(union_kernel, dim3(1), dim3(kUnionThreads), static_cast<size_t>(kUnionWarps) * E * 4, s,
+                       static_cast<const int32_t*>(ids), P, E, lay.unique, lay.n_unique, lay.seg_off, lay.perm,
+                       lay.pair_pos, di.status, T, S, tokb, lay.plan, lay.tb_done, lay.rb_done, H / kRowBlock)) {
       return COLI_ERR_CUDA;
+    }
     rec.mark_through(4, 5);
   }
   // 3. expert FFN and combine

@@ -63,9 +63,13 @@ struct PfCfg {
   static constexpr int NSC = 4;
   static constexpr int NBUF = NMAT == 2 ? 3 : 6;                    // chunk slots
   static constexpr int NSB = NBUF;
-  static constexpr int ACOL = NMAT * kPfMaxN;                       // first A column
+  // Accumulator buffers: two for the down GEMM, so that the epilogue of one
+  // tile overlaps the MMAs of the next; gate/up needs both of its matrices'
+  // accumulators and has room for one set only.
+  static constexpr int ACC_BUFS = NMAT == 1 ? 2 : 1;
+  static constexpr int ACOL = ACC_BUFS * NMAT * kPfMaxN;            // first A column
   static constexpr int META_INTS = 3 * kMaxSeg + 4;
-  static constexpr int NBAR = 2 * NSC + NSB + 2 * NBUF + 3;
+  static constexpr int NBAR = 2 * NSC + NSB + 2 * NBUF + 2 * ACC_BUFS + 1;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(NSC) * CSTAGE + static_cast<size_t>(NSB) * BSTAGE +
                                  META_INTS * 4 + NBAR * 8 + 16;
   static_assert(CSTAGE % 1024 == 0 && BSTAGE % 1024 == 0, "stage alignment");
@@ -267,8 +271,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* a_full = b_full + C::NSB;
   uint64_t* slot_empty = a_full + C::NBUF;   // chunk slot consumed by the MMAs (A buffer + token stage)
   uint64_t* acc_full = slot_empty + C::NBUF;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* mma_done = acc_empty + 1;
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  uint64_t* mma_done = acc_empty + C::ACC_BUFS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -285,8 +289,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&a_full[q], 8);
       mbar_init(&slot_empty[q], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kPfDqWarps);
+    for (int q = 0; q < C::ACC_BUFS; ++q) {
+      mbar_init(&acc_full[q], 1);
+      mbar_init(&acc_empty[q], kPfDqWarps);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -402,7 +408,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
         const uint32_t idesc = idesc_bf16_m128(ti.npad);
-        if (!(ok = mbar_wait(acc_empty, (tt & 1u) ^ 1u, abort_flag, a.status))) break;
+        const int ab = static_cast<int>(tt % C::ACC_BUFS);
+        const uint32_t dbase = tbase + ab * NMAT * kPfMaxN;
+        if (!(ok = mbar_wait(&acc_empty[ab], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag, a.status))) break;
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
           const int b = static_cast<int>(it % C::NBUF);
@@ -417,14 +425,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const uint64_t bdesc = sw128_kmajor_desc(bs + kk * 32);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              mma_bf16_ts(tbase + m * kPfMaxN, acol + m * 32 + kk * 8, bdesc, idesc, (kb | kk) != 0);
+              mma_bf16_ts(dbase + m * kPfMaxN, acol + m * 32 + kk * 8, bdesc, idesc, (kb | kk) != 0);
           }
           tc_commit(&slot_empty[b]);   // b == s: the slot's A buffer and token stage
           ++it;
           ++bit;
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(&acc_full[ab]);
         ++tt;
       }
       // every MMA of this CTA has completed before TMEM is released
@@ -447,9 +455,51 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     uint32_t it = 0, tt = 0;
     uint32_t scl[NMAT][4];                    // this row's fp16 scales of the current code stage
     bool ok = true;
+    // epilogue of one tile: accumulators -> h (gate/up) or y (down)
+    auto epilogue = [&](const PfTile& et, uint32_t ett) -> bool {
+      const int ab = static_cast<int>(ett % C::ACC_BUFS);
+      if (!warp_wait(&acc_full[ab], (ett / C::ACC_BUFS) & 1u, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint32_t dbase = tbase + lane_bits + ab * NMAT * kPfMaxN;
+      const int grow = et.rblk * kRowBlock + r;     // output row within the expert
+      const int hpos = frag_pos(grow);
+      for (int c8 = dw >> 2; c8 < (et.npad >> 3); c8 += kPfDqWarps / 4) {
+        uint32_t d0[8], d1[8];
+        tmem_ld8(dbase + c8 * 8, d0);
+        if (NMAT == 2) tmem_ld8(dbase + kPfMaxN + c8 * 8, d1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          const int i = c8 * 8 + n;
+          if (i < et.ntok) {
+            if (NMAT == 2) {
+              const float gv = __uint_as_float(d0[n]), uv = __uint_as_float(d1[n]);
+              const float hv = gv / (1.0f + expf(-gv)) * uv;
+              a.hq[static_cast<size_t>(et.orow + i) * a.I + hpos] = float_to_bf16_bits(hv);
+            } else {
+              a.ypair[static_cast<size_t>(et.orow + i) * a.H + grow] = __uint_as_float(d0[n]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      return true;
+    };
+    // with two accumulator buffers a tile's epilogue waits until the first
+    // kDefer chunks of the next tile are dequantised, so those MMAs run under it
+    constexpr int kDefer = C::NBUF;
+    PfTile pend{};
+    uint32_t pend_tt = 0;
+    bool has_pend = false;
     for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
       const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
       for (int kb = 0; kb < nk; ++kb, ++it) {
+        if (C::ACC_BUFS > 1 && has_pend && kb == (kDefer < nk ? kDefer : nk - 1)) {
+          if (!(ok = epilogue(pend, pend_tt))) break;
+          has_pend = false;
+        }
         if (static_cast<int>(it % kPfTeams) != team) continue;
         const int ci = kb % cps;                       // chunks are stage-aligned: it % cps == kb % cps
         const uint32_t stage = it / cps;
@@ -503,35 +553,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) mbar_arrive(&a_full[b]);
       }
       if (!ok) break;
-      // epilogue: accumulators -> h (gate/up) or y (down)
-      if (!(ok = warp_wait(acc_full, tt & 1u, abort_flag, a.status))) break;
-      tc_fence_after();
-      const int grow = ti.rblk * kRowBlock + r;     // output row within the expert
-      const int hpos = frag_pos(grow);
-      for (int c8 = dw >> 2; c8 < (ti.npad >> 3); c8 += kPfDqWarps / 4) {
-        uint32_t d0[8], d1[8];
-        tmem_ld8(tbase + lane_bits + c8 * 8, d0);
-        if (NMAT == 2) tmem_ld8(tbase + lane_bits + kPfMaxN + c8 * 8, d1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          const int i = c8 * 8 + n;
-          if (i < ti.ntok) {
-            if (NMAT == 2) {
-              const float gv = __uint_as_float(d0[n]), uv = __uint_as_float(d1[n]);
-              const float hv = gv / (1.0f + expf(-gv)) * uv;
-              a.hq[static_cast<size_t>(ti.orow + i) * a.I + hpos] = float_to_bf16_bits(hv);
-            } else {
-              a.ypair[static_cast<size_t>(ti.orow + i) * a.H + grow] = __uint_as_float(d0[n]);
-            }
-          }
-        }
+      if (C::ACC_BUFS == 1) {
+        if (!(ok = epilogue(ti, tt))) break;
+      } else {
+        pend = ti;
+        pend_tt = tt;
+        has_pend = true;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
       ++tt;
     }
+    if (ok && has_pend) ok = epilogue(pend, pend_tt);
   }
   tc_fence_before();
   __syncthreads();

@@ -176,6 +176,150 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
   if (plan) block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
 }
 
+// ---------------------------------------------------------------------------
+// Union of a large batch over many CTAs (the prefill form's batches): the same
+// stable counting sort, split in three launches.
+//   1. union_count_kernel: CTA b counts the ids of its chunk of pairs per
+//      expert (shared-memory atomics: counts do not depend on order) into
+//      cnt[b][e];
+//   2. union_scan_kernel (one CTA): per expert, an exclusive scan over the
+//      chunks; over experts, the segment starts; cnt[b][e] becomes the first
+//      position of chunk b's pairs of expert e; unique ids and segments;
+//   3. union_scatter_kernel: CTA b ranks its pairs inside each expert with
+//      per-warp histograms over contiguous pair ranges (as block_union does)
+//      and writes perm / pair_pos, so equal ids keep pair order.
+// cnt: ceil(P / chunk) * E ints of workspace; chunk a multiple of 1024.
+inline int union_chunk(int P) {
+  const int c = (P + 511) / 512;
+  return c <= 1024 ? 1024 : (c + 1023) / 1024 * 1024;
+}
+
+__global__ void __launch_bounds__(1024) union_count_kernel(const int32_t* __restrict__ ids, int P, int E, int chunk,
+                                                           int32_t* __restrict__ cnt, uint32_t* __restrict__ status) {
+  extern __shared__ int hist[];
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int p0 = blockIdx.x * chunk, p1 = min(P, p0 + chunk);
+  bool bad = false;
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int e = ids[p];
+    if (e < 0 || e >= E) bad = true;
+    else atomicAdd(&hist[e], 1);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(1024) union_scan_kernel(int32_t* __restrict__ cnt, int NB, int E,
+                                                          int32_t* __restrict__ unique_ids,
+                                                          int32_t* __restrict__ n_unique,
+                                                          int32_t* __restrict__ seg_off) {
+  __shared__ int scratch[33];
+  __shared__ int carry_pairs, carry_u;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    carry_pairs = 0;
+    carry_u = 0;
+  }
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    int tot = 0;
+    if (e < E)
+      for (int b = 0; b < NB; ++b) {
+        int32_t* c = cnt + static_cast<size_t>(b) * E + e;
+        const int v = *c;
+        *c = tot;
+        tot += v;
+      }
+    int tot_pairs = 0, tot_u = 0;
+    const int off = block_exclusive_scan(tot, scratch, &tot_pairs);
+    const int uidx = block_exclusive_scan(tot > 0 ? 1 : 0, scratch, &tot_u);
+    const int cp = carry_pairs, cu = carry_u;
+    if (e < E) {
+      for (int b = 0; b < NB; ++b) cnt[static_cast<size_t>(b) * E + e] += cp + off;
+      if (tot > 0) {
+        unique_ids[cu + uidx] = e;
+        seg_off[cu + uidx] = cp + off;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      carry_pairs = cp + tot_pairs;
+      carry_u = cu + tot_u;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *n_unique = carry_u;
+    seg_off[carry_u] = carry_pairs;
+  }
+}
+
+// Dynamic shared memory: kUnionWarps * E ints.
+__global__ void __launch_bounds__(kUnionThreads) union_scatter_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                                      int chunk, const int32_t* __restrict__ base,
+                                                                      int32_t* __restrict__ perm,
+                                                                      int32_t* __restrict__ pair_pos) {
+  extern __shared__ int hist[];
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kUnionWarps * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int c0 = blockIdx.x * chunk, c1 = min(P, c0 + chunk);
+  const int per_warp = chunk / kUnionWarps;                   // a multiple of 32
+  const int p_begin = min(c1, c0 + warp * per_warp), p_end = min(c1, p_begin + per_warp);
+  int* myhist = hist + warp * E;
+  for (int b0 = p_begin; b0 < p_end; b0 += 32) {
+    const int p = b0 + lane;
+    int e = -1;
+    if (p < p_end) {
+      e = ids[p];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) myhist[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per (warp, expert) first position: the chunk's base for the expert plus
+  // the counts of the lower warps
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int off = base[static_cast<size_t>(blockIdx.x) * E + e];
+    for (int w = 0; w < kUnionWarps; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = off;
+      off += c;
+    }
+  }
+  __syncthreads();
+  for (int b0 = p_begin; b0 < p_end; b0 += 32) {
+    const int p = b0 + lane;
+    int e = -1;
+    if (p < p_end) {
+      e = ids[p];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const unsigned lower = peers & ((1u << lane) - 1u);
+    if (e >= 0) {
+      const int pos = myhist[e] + __popc(lower);
+      perm[pos] = p;
+      pair_pos[p] = pos;
+    } else if (p < p_end) {
+      pair_pos[p] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) myhist[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 // Plan from an existing union (coli_moe_expert_ffn), one CTA.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ n_unique,
                                                     const int32_t* __restrict__ seg_off, int T, int S, int tokb,
