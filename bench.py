@@ -187,6 +187,30 @@ def oracle_sample(shape: synth.LayerShape, seconds: float):
     return tok_done / elapsed, 1, desc
 
 
+# ---- replicas over ranks (the path has no exchange step) -------------------
+
+def rank_batches(rank: int, nb: int) -> list[int]:
+    """Seed indices of the nb rotating input batches of one rank: every rank
+    draws its own batches, so ranks never process the same tokens."""
+    return [rank * nb + b for b in range(nb)]
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """A rank's device-timed milliseconds -> the maximum over all ranks."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: the tokens of all ranks over the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -235,11 +259,11 @@ def main():
         b = li.bias()
         layers.append(cm.MoELayer(dims, sg.expert_tensors(shape, 0, l), rw, None if b is None else torch.from_numpy(b).cuda()))
     NB = a.batches
-    xs = [torch.from_numpy(synth.activations(shape, 0, rank * NB + b).view(np.int16)).cuda() for b in range(NB)]
+    xs = [torch.from_numpy(synth.activations(shape, 0, bi).view(np.int16)).cuda() for bi in rank_batches(rank, NB)]
     lgs = [None] * NB
     if shape.logits_in:
-        lgs = [torch.from_numpy(synth.normal_f32(0, 1000 + rank * NB + b, synth.LOGITS_IN, (T, E), 1.0)).cuda()
-               for b in range(NB)]
+        lgs = [torch.from_numpy(synth.normal_f32(0, 1000 + bi, synth.LOGITS_IN, (T, E), 1.0)).cuda()
+               for bi in rank_batches(rank, NB)]
     ws = layers[0].workspace(T)
     outs = [torch.empty((T, H), dtype=torch.int16, device="cuda") for _ in range(2)]
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -324,12 +348,8 @@ def main():
         raise RuntimeError(f"device status flags {fl:#x} in the timed region")
 
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * T * K / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), world, "cuda")
+    value = job_throughput(world, T, K, total_ms)
 
     # dominant kernel, timed live on the launching stream (stage 5 -> 6): the
     # decode form's one persistent FFN launch (gate/up, down and, for T <= 4,
@@ -418,12 +438,8 @@ def main():
         oh.copy_(od, non_blocking=True)
         ee[i].record()
     torch.cuda.synchronize()
-    e2e_ms = sum(es[i].elapsed_time(ee[i]) for i in range(K2))
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * T * K2 / (e2e_ms / 1e3), "unit": UNIT,
+    e2e_ms = max_over_ranks(sum(es[i].elapsed_time(ee[i]) for i in range(K2)), world, "cuda")
+    e2e = {"value": job_throughput(world, T, K2, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": T * H * 2 + (T * E * 4 if shape.logits_in else 0), "d2h_bytes_per_step": T * H * 2}
 
     cpu = None
