@@ -296,3 +296,21 @@ def test_glm_prefill_4096_sampled(lib, glm_layer):
     err, g = check_layer(lib, shape, glm_layer, oracle_weights(shape), synth.activations(shape),
                          sample=[0, 1777, 4095], logits_in=li.logits())
     print(f"prefill 4096: max rel err {err:.3e}")
+
+
+# ---------------------------------------------------------------- batch invariance
+
+@pytest.mark.parametrize("T", [2, 4, 8])
+def test_decode_batch_invariance(lib, glm_layer, T):
+    """A token's output in a batch of T (draft + verify tokens decoded in one
+    forward) is bit-identical to its output when decoded alone: each token's
+    dot products, group scaling, K-half reduction and combine run in the same
+    order whatever the batch, and routing is per token."""
+    shape = synth.DECODE_B1
+    x = np.concatenate([synth.activations(shape, 0, b) for b in range(T)])
+    gb = run_gpu_layer(lib, glm_layer, x, residual_bits=x, flags=lib._lib.COLI_LAYER_PRENORM)
+    assert gb["flags"] == 0
+    for t in range(T):
+        g1 = run_gpu_layer(lib, glm_layer, x[t:t + 1], residual_bits=x[t:t + 1], flags=lib._lib.COLI_LAYER_PRENORM)
+        assert np.array_equal(g1["ids"][0], gb["ids"][t])
+        assert np.array_equal(g1["out"][0], gb["out"][t]), t
