@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--form", choices=["auto", "decode", "prefill"], default="auto",
                     help="FFN form (COLI_PATH_*); auto lets the library choose")
+    ap.add_argument("--graph", choices=["on", "off"], default="on",
+                    help="replay each step from a CUDA graph captured once per input batch (the stage breakdown "
+                         "then comes from separate eager steps)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="target length of the oracle sample")
     a = ap.parse_args()
     if a.steps is None:
@@ -315,14 +318,35 @@ def main():
     torch.cuda.synchronize()
 
     K = a.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     M = min(K, 64)
+    use_graph = a.graph == "on"
+    graphs = []
+    launches_per_step = None
     stage = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(M)]
     for evs in stage:  # create the events (they exist once recorded)
         for e in evs:
             e.record()
     torch.cuda.synchronize()
+    if use_graph:
+        # stage breakdown from eager steps (events cannot sit inside the graphs)
+        for i in range(M):
+            flush_l2()
+            cm.coli_moe_set_stage_events(stage[i])
+            step(i % NB)
+        torch.cuda.synchronize()
+        cm.coli_moe_launch_count(reset=True)
+        for bi in range(NB):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(bi)
+            graphs.append(g)
+        launches_per_step = cm.coli_moe_launch_count(reset=True) // NB
+        for bi in range(NB):   # warm replays
+            graphs[bi].replay()
+        torch.cuda.synchronize()
+
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -333,13 +357,16 @@ def main():
     for i in range(K):
         flush_l2()
         ev_s[i].record()
-        if i < M:
-            cm.coli_moe_set_stage_events(stage[i])
-        step(i % NB)
+        if use_graph:
+            graphs[i % NB].replay()
+        else:
+            if i < M:
+                cm.coli_moe_set_stage_events(stage[i])
+            step(i % NB)
         ev_e[i].record()
     torch.cuda.synchronize()
     t_wall1 = time.time()
-    launches = cm.coli_moe_launch_count()
+    launches = launches_per_step * K if use_graph else cm.coli_moe_launch_count()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
@@ -423,6 +450,22 @@ def main():
     e2e_ms = []
     es = [torch.cuda.Event(enable_timing=True) for _ in range(K2)]
     ee = [torch.cuda.Event(enable_timing=True) for _ in range(K2)]
+
+    def e2e_step(bi):
+        if ld is not None:
+            lgs_save = lgs[bi]
+            lgs[bi] = ld
+        step(bi, x=xd, out=od)
+        if ld is not None:
+            lgs[bi] = lgs_save
+
+    g_e2e = None
+    if use_graph:   # one graph on the static device buffers the host copies fill
+        e2e_step(0)
+        torch.cuda.synchronize()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            e2e_step(0)
     for i in range(K2):
         bi = i % NB
         flush_l2()
@@ -430,11 +473,10 @@ def main():
         xd.copy_(xh[bi], non_blocking=True)
         if ld is not None:
             ld.copy_(lh[bi], non_blocking=True)
-            lgs_save = lgs[bi]
-            lgs[bi] = ld
-        step(bi, x=xd, out=od)
-        if ld is not None:
-            lgs[bi] = lgs_save
+        if g_e2e is not None:
+            g_e2e.replay()
+        else:
+            e2e_step(bi)
         oh.copy_(od, non_blocking=True)
         ee[i].record()
     torch.cuda.synchronize()
@@ -451,7 +493,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": a.warmup,
             "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "ffn_form": form,
+            "dtype": "bf16", "data": "synthetic", "ffn_form": form, "cuda_graph": use_graph,
             "config": {"workload": shape.name, "tokens": T, "hidden": H, "inter": I, "experts": E, "top_k": k,
                        "shared": S, "layers": shape.layers, "union_per_batch": U,
                        "union_per_layer": u_stack or None, "l2": "flushed before every step (256 MiB write, then 256 MiB read), outside the timed events",
