@@ -61,7 +61,8 @@ def parse():
     if a.steps is None:
         a.steps = {"glm52_layer_decode_b1": 2000, "glm52_layer_decode_b64_zipf": 400,
                    "glm52_layer_prefill_4096": 40, "glm52_stack16_decode_b4": 200,
-                   "glm52_layer_prefill_512_e32": 50}.get(a.workload, 20)
+                   "glm52_layer_prefill_512_e32": 50, "glm52_layer_decode_b1_gs64": 2000,
+                   "glm52_layer_prefill_4096_gs64": 40}.get(a.workload, 20)
     a.warmup = max(a.warmup, 3)
     return a
 
@@ -254,7 +255,7 @@ def main():
 
     shape = synth.WORKLOADS[a.workload]
     T, H, I, E, k, S = shape.tokens, shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared
-    dims = cm.dims_for(H, I, E, k, S)
+    dims = cm.dims_for(H, I, E, k, S, shape.group)
     layers = []
     for l in range(shape.layers):
         li = synth.LayerInputs(shape, 0, l)
@@ -390,7 +391,7 @@ def main():
     P = T * k
     u_step = [U[i % NB] for i in range(M)]  # the first layer of each step carries the stage events
     form = a.form if a.form != "auto" else ("prefill" if prefill_form(shape) else "decode")
-    per_mat = H * I // 2 + (H * I // 32) * 2          # codes + scales of one matrix
+    per_mat = H * I // 2 + (H * I // shape.group) * 2   # codes + scales of one matrix
     if form == "prefill" and not prefill_form(shape):
         # prefill form on a decode-sized batch: the gate/up GEMM streams the
         # gate and up matrices of every touched expert

@@ -21,13 +21,16 @@
  *            w_j = exp(l'_j - l'_max) / sum_{i<k} exp(l'_i - l'_max)
  *   union    unique experts ascending; pairs p = t*k + j grouped by expert,
  *            stable in p
- *   expert   W = code * scale, code int4 in [-8,7], fp16 scale per 32 along K;
+ *   expert   W = code * scale, code int4 in [-8,7], fp16 scale per G along K;
  *            h = bf16( silu(W_gate x) * (W_up x) ),  y = W_down h   (fp32 accumulate)
  *   combine  out[t] = bf16( sum_j w[t,j] * y_{id[t,j]} + sum_s y_{E+s} + residual[t] )
  *
  * Container format (row-major, K contiguous):
  *   gate_q, up_q  uint8 [E+S][I][H/2]   down_q uint8 [E+S][H][I/2]
- *   gate_s, up_s  fp16  [E+S][I][H/32]  down_s fp16  [E+S][H][I/32]
+ *   gate_s, up_s  fp16  [E+S][I][H/G]   down_s fp16  [E+S][H][I/G]
+ *   G = dims.group = 32, or 64 for the group-scaled "gs64" container the
+ *   README recommends ("2. Scarica il modello"): scale c / G of a row
+ *   multiplies its element c.
  *   Element c of a row is nibble (c & 1) of byte c/2 (low nibble first); the
  *   nibble n encodes code n - 16*(n >= 8).  Shared experts are ids E..E+S-1.
  *
@@ -44,7 +47,8 @@
  *     of range, a pipeline wait that timed out) set bits in a per-device
  *     status word that coli_moe_get_status reads and clears; kernels never
  *     trap.
- *   - Supported shapes: group == 32, H % 256 == 0, I % 256 == 0 or I == 128,
+ *   - Supported shapes: group == 32 with H % 256 == 0, I % 256 == 0 or
+ *     I == 128; group == 64 with H % 512 == 0, I % 512 == 0; and for both
  *     1 <= k <= min(E, 32), E <= 1024, 0 <= S <= 4, T >= 0, T*k <= 2^24.
  *     Anything else returns COLI_ERR_UNSUPPORTED.
  *   - Thread safety: calls may be made concurrently from several host
@@ -90,7 +94,7 @@ typedef struct {
   int32_t n_experts;  /* E: routed experts */
   int32_t top_k;      /* k */
   int32_t n_shared;   /* S: shared experts, always active with weight 1.0 */
-  int32_t group;      /* quantisation group along K; must be 32 */
+  int32_t group;      /* quantisation group along K: 32 or 64 */
 } coli_moe_dims;
 
 typedef struct {

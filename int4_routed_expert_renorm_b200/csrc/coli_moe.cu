@@ -79,22 +79,29 @@ coli_status dev_info(DevInfo* out) {
   }
   if (!g_attr_done[dev]) {
     bool ok = true;
-#define COLI_SET_SMEM(NT, SG, KCD)                                                                   \
-  ok &= cudaFuncSetAttribute(ffn_fused_kernel<NT, SG, KCD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(FusedCfg<NT, KCD>::SMEM)) == cudaSuccess;
-    COLI_SET_SMEM(1, true, 256)
-    COLI_SET_SMEM(1, false, 256)
-    COLI_SET_SMEM(4, false, 256)
-    COLI_SET_SMEM(1, true, 128)
-    COLI_SET_SMEM(1, false, 128)
-    COLI_SET_SMEM(4, false, 128)
-    COLI_SET_SMEM(1, true, 512)
-    COLI_SET_SMEM(1, false, 512)
+#define COLI_SET_SMEM(NT, SG, KCD, GR)                                                                   \
+  ok &= cudaFuncSetAttribute(ffn_fused_kernel<NT, SG, KCD, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(FusedCfg<NT, KCD, GR>::SMEM)) == cudaSuccess;
+    COLI_SET_SMEM(1, true, 256, 32)
+    COLI_SET_SMEM(1, false, 256, 32)
+    COLI_SET_SMEM(4, false, 256, 32)
+    COLI_SET_SMEM(1, true, 128, 32)
+    COLI_SET_SMEM(1, false, 128, 32)
+    COLI_SET_SMEM(4, false, 128, 32)
+    COLI_SET_SMEM(1, true, 512, 32)
+    COLI_SET_SMEM(1, false, 512, 32)
+    COLI_SET_SMEM(1, true, 512, 64)
+    COLI_SET_SMEM(1, false, 512, 64)
+    COLI_SET_SMEM(4, false, 256, 64)
 #undef COLI_SET_SMEM
-    ok &= cudaFuncSetAttribute(ffn_prefill_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PfCfg<2>::SMEM)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(ffn_prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PfCfg<1>::SMEM)) == cudaSuccess;
+#define COLI_SET_PF_SMEM(NMAT, GR)                                                                      \
+  ok &= cudaFuncSetAttribute(ffn_prefill_kernel<NMAT, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(PfCfg<NMAT>::SMEM)) == cudaSuccess;
+    COLI_SET_PF_SMEM(2, 32)
+    COLI_SET_PF_SMEM(1, 32)
+    COLI_SET_PF_SMEM(2, 64)
+    COLI_SET_PF_SMEM(1, 64)
+#undef COLI_SET_PF_SMEM
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
     ok &= cudaFuncSetAttribute(union_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -147,9 +154,11 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 coli_status check_dims(const coli_moe_dims* d) {
   if (!d) return COLI_ERR_INVALID_ARG;
-  if (d->group != 32) return COLI_ERR_UNSUPPORTED;
+  if (d->group != 32 && d->group != 64) return COLI_ERR_UNSUPPORTED;
   if (d->hidden <= 0 || d->hidden % 256 != 0) return COLI_ERR_UNSUPPORTED;
   if (d->inter <= 0 || !(d->inter % 256 == 0 || d->inter == 128)) return COLI_ERR_UNSUPPORTED;
+  // 64-wide groups: scale rows are read in 16-byte boxes of 8 scales (512 K)
+  if (d->group == 64 && (d->hidden % 512 != 0 || d->inter % 512 != 0)) return COLI_ERR_UNSUPPORTED;
   if (d->n_experts < 1 || d->n_experts > 1024) return COLI_ERR_UNSUPPORTED;
   if (d->top_k < 1 || d->top_k > 32 || d->top_k > d->n_experts) return COLI_ERR_UNSUPPORTED;
   if (d->n_shared < 0 || d->n_shared > 4) return COLI_ERR_UNSUPPORTED;
@@ -244,8 +253,9 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 }
 
 // Tensor maps of one matrix kind: codes [rows_total][K/2] bytes and scales
-// [rows_total][K/32] fp16, tiles of 128 rows x KC elements.
-bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, CUtensorMap* mq,
+// [rows_total][K/group] fp16, tiles of 128 rows x KC elements; the scale box
+// is KC/32 scales (group 32) or 8 scales (group 64, K a multiple of 512).
+bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, int group, CUtensorMap* mq,
                  CUtensorMap* ms) {
   // stages of 512 K move their codes as two 128-byte-wide boxes
   const CUtensorMapSwizzle swz = KC >= 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -253,8 +263,8 @@ bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K
                  swz))
     return false;
   if (KC < K) {
-    if (!encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / 32, rows_total, (K / 32) * 2, KC / 32, kRowBlock,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / group, rows_total, (K / group) * 2,
+                   group == 32 ? KC / 32 : 8, kRowBlock, CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   } else {
     std::memset(ms, 0, sizeof(*ms));  // scales move by 1-D bulk copies when a stage spans K
@@ -264,12 +274,12 @@ bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K
 
 // The persistent FFN kernel is launched cooperatively (all CTAs resident, so
 // the counter waits of down tiles on gate/up tiles always make progress).
-template <int NT, bool SG, int KCD>
+template <int NT, bool SG, int KCD, int GR>
 bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kFfnThreads);
-  cfg.dynamicSmemBytes = FusedCfg<NT, KCD>::SMEM;
+  cfg.dynamicSmemBytes = FusedCfg<NT, KCD, GR>::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -279,12 +289,12 @@ bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStre
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   ++t_launches;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD, GR>, m[0], m[1], m[2], m[3], m[4], m[5], a);
   if (e != cudaSuccess) {
     // without overlap with the previous kernel
     cudaGetLastError();
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+    e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD, GR>, m[0], m[1], m[2], m[3], m[4], m[5], a);
   }
   return e == cudaSuccess;
 }
@@ -293,9 +303,9 @@ bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStre
 // tiles while T <= 8, else 32-token tiles.
 template <int KCD>
 bool launch_ffn_for(int T, const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
-  if (T == 1) return launch_ffn_fused<1, true, KCD>(m, a, grid, st);
-  if (T <= 8) return launch_ffn_fused<1, false, KCD>(m, a, grid, st);
-  return launch_ffn_fused<4, false, KCD>(m, a, grid, st);
+  if (T == 1) return launch_ffn_fused<1, true, KCD, 32>(m, a, grid, st);
+  if (T <= 8) return launch_ffn_fused<1, false, KCD, 32>(m, a, grid, st);
+  return launch_ffn_fused<4, false, KCD, 32>(m, a, grid, st);
 }
 
 inline int tok_block(int T) { return T <= 8 ? 8 : 32; }
@@ -366,12 +376,15 @@ Form choose_form(uint32_t flags, int T, int E, int k) {
 // rows x cps*32 bytes (128B / 64B swizzle), scales [rows][K/32] fp16 in boxes
 // of 128 rows x cps*2 (unless one stage spans K), token rows [rows][K] bf16 in
 // boxes of 128/64/32/16 rows x 64 elements (128B swizzle).
-bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, CUtensorMap* mq,
+bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int group, CUtensorMap* mq,
                     CUtensorMap* ms) {
   const int cps = (K % 256 == 0) ? 4 : 2;
   const CUtensorMapSwizzle swz = cps == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, cps * 32, kRowBlock, swz))
     return false;
+  if (group == 64)   // boxes of 8 scales (two code stages); K is a multiple of 512
+    return encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / 64, rows_total, (K / 64) * 2, 8, kRowBlock,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (K == cps * 64) {
     std::memset(ms, 0, sizeof(*ms));
     return true;
@@ -380,7 +393,7 @@ bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, in
                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int NMAT>
+template <int NMAT, int GR>
 bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -393,7 +406,7 @@ bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ++t_launches;
-  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT>, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a) ==
+  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT, GR>, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a) ==
          cudaSuccess;
 }
 
@@ -408,9 +421,10 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
   const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
   CUtensorMap mg[8], md[8];   // q0, q1, s0, s1, token rows in boxes of 128, 64, 32, 16 rows
-  if (!pf_weight_maps(w->gate_q, w->gate_s, rows_gu, H, &mg[0], &mg[2]) ||
-      !pf_weight_maps(w->up_q, w->up_s, rows_gu, H, &mg[1], &mg[3]) ||
-      !pf_weight_maps(w->down_q, w->down_s, rows_dn, I, &md[0], &md[2]))
+  const int G = d->group;
+  if (!pf_weight_maps(w->gate_q, w->gate_s, rows_gu, H, G, &mg[0], &mg[2]) ||
+      !pf_weight_maps(w->up_q, w->up_s, rows_gu, H, G, &mg[1], &mg[3]) ||
+      !pf_weight_maps(w->down_q, w->down_s, rows_dn, I, G, &md[0], &md[2]))
     return COLI_ERR_CUDA;
   for (int j = 0; j < 4; ++j) {
     const uint32_t box = 128u >> j;
@@ -457,11 +471,15 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   };
   a.s0 = w->gate_s;
   a.s1 = w->up_s;
-  if (!launch_prefill<2>(mg, a, grid_for(I / kRowBlock), st)) return COLI_ERR_CUDA;
+  if (!(G == 32 ? launch_prefill<2, 32>(mg, a, grid_for(I / kRowBlock), st)
+                : launch_prefill<2, 64>(mg, a, grid_for(I / kRowBlock), st)))
+    return COLI_ERR_CUDA;
   rec.mark(6);
   a.s0 = w->down_s;
   a.s1 = w->down_s;
-  if (!launch_prefill<1>(md, a, grid_for(H / kRowBlock), st)) return COLI_ERR_CUDA;
+  if (!(G == 32 ? launch_prefill<1, 32>(md, a, grid_for(H / kRowBlock), st)
+                : launch_prefill<1, 64>(md, a, grid_for(H / kRowBlock), st)))
+    return COLI_ERR_CUDA;
   rec.mark(7);
   {
     const long work = static_cast<long>(T) * (H / 4);
@@ -494,10 +512,11 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   CUtensorMap maps[6];   // gate q, up q, gate s, up s, down q, down s
   // down stages: 512 K (two 128-byte code boxes) for the one-n-tile forms,
   // whose activation slice per stage stays small
+  const int G = d->group;
   const int kc_dn = (I % 512 == 0 && T <= 8) ? 512 : (I % 256 == 0) ? 256 : 128;
-  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, &maps[0], &maps[2]) ||
-      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, &maps[1], &maps[3]) ||
-      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, &maps[4], &maps[5]))
+  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, G, &maps[0], &maps[2]) ||
+      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, G, &maps[1], &maps[3]) ||
+      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, G, &maps[4], &maps[5]))
     return COLI_ERR_CUDA;
 
   FfnArgs a{};
@@ -530,8 +549,13 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
     const long tiles = blocks_ub * (I / kRowBlock + H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
     bool ok;
-    if (kc_dn == 512)
-      ok = T == 1 ? launch_ffn_fused<1, true, 512>(maps, a, grid, st) : launch_ffn_fused<1, false, 512>(maps, a, grid, st);
+    if (G == 64)   // I % 512 == 0: 512-K down stages while T <= 8
+      ok = T == 1   ? launch_ffn_fused<1, true, 512, 64>(maps, a, grid, st)
+           : T <= 8 ? launch_ffn_fused<1, false, 512, 64>(maps, a, grid, st)
+                    : launch_ffn_fused<4, false, 256, 64>(maps, a, grid, st);
+    else if (kc_dn == 512)
+      ok = T == 1 ? launch_ffn_fused<1, true, 512, 32>(maps, a, grid, st)
+                  : launch_ffn_fused<1, false, 512, 32>(maps, a, grid, st);
     else
       ok = kc_dn == 256 ? launch_ffn_for<256>(T, maps, a, grid, st) : launch_ffn_for<128>(T, maps, a, grid, st);
     if (!ok) return COLI_ERR_CUDA;

@@ -68,7 +68,11 @@ struct FfnArgs {
 
 // Shared-memory layout constants.  KC elements of K per stage; NT n-tiles of 8
 // tokens per tile; NMAT matrices per stage (2 = gate+up, 1 = down).
-template <int KC, int NT, int NMAT>
+// GROUP: K elements per fp16 scale (32, or 64 for the gs64 container).  With
+// GROUP 64 a stage's scale rows are always one 16-byte box of 8 scales (512 K),
+// loaded whole by the stage (a 256-K stage uses half of it; the next stage
+// reloads the same box, from L2).
+template <int KC, int NT, int NMAT, int GROUP = 32>
 struct StageCfg {
   static constexpr int TOKB = 8 * NT;
   static constexpr int GPW = KC / 64;                 // groups per warp per stage (two K-halves)
@@ -76,7 +80,7 @@ struct StageCfg {
   static constexpr int SUBS = KC >= 512 ? KC / 256 : 1;   // 128-byte-wide code sub-tiles per stage
   static constexpr int RSTR = ROWB / SUBS;            // row stride inside a code sub-tile
   static constexpr int SUB_BYTES = kRowBlock * RSTR;
-  static constexpr int SROWB = KC / 16;               // scale bytes per row
+  static constexpr int SROWB = GROUP == 32 ? KC / 16 : 16;   // scale bytes per row
   static constexpr int CODE_BYTES = kRowBlock * ROWB;
   static constexpr int SC_BYTES = kRowBlock * SROWB;
   static constexpr int W_BYTES = NMAT * (CODE_BYTES + SC_BYTES);
@@ -85,12 +89,13 @@ struct StageCfg {
   static constexpr bool SWZ = (KC >= 256);
   static_assert(CODE_BYTES % 1024 == 0 && SC_BYTES % 1024 == 0, "stage regions must stay 1 KiB aligned");
   static_assert(NMAT == 1 || KC <= 256, "wide stages are for the down projection only");
+  static_assert(GROUP == 32 || (GROUP == 64 && KC >= 256), "64-wide groups need stages of 256 K or more");
 };
 
-template <int NT, int KCD>
+template <int NT, int KCD, int GROUP = 32>
 struct FusedCfg {
-  using GU = StageCfg<256, NT, 2>;
-  using DN = StageCfg<KCD, NT, 1>;
+  using GU = StageCfg<256, NT, 2, GROUP>;
+  using DN = StageCfg<KCD, NT, 1, GROUP>;
   static constexpr int STAGE = ((GU::STAGE_USED > DN::STAGE_USED ? GU::STAGE_USED : DN::STAGE_USED) + 1023) / 1024 * 1024;
   static constexpr int RED_BYTES = kRowWarps * 32 * NT * 4 * 2 * 4;   // K-half partials (2 matrices)
   static constexpr int META_BYTES = (3 * kMaxSeg + 4) * 4;            // cached plan / unique / seg_off
@@ -227,13 +232,13 @@ __device__ __forceinline__ bool wait_h_ready(const FfnArgs& a, int tbg, int targ
 // Producer: fills the stages of one tile.  For a down tile the weight copies
 // go out immediately; the h rows wait (bounded) for the tile's token block to
 // be complete in gate/up.  Returns false on a timeout.
-template <int KC, int NT, int NMAT, int NS, int STAGE>
+template <int KC, int NT, int NMAT, int NS, int STAGE, int GROUP>
 __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& ti, const CUtensorMap* mq0,
                                              const CUtensorMap* mq1, const CUtensorMap* ms0, const CUtensorMap* ms1,
                                              const uint16_t* s0_1d, const uint16_t* s1_1d, int K, int R, int nrb_gu,
                                              uint8_t* smem, uint64_t* full, uint64_t* empty, int& s, uint32_t& ph,
                                              long& issued, volatile int* abort_flag, int lane) {
-  using C = StageCfg<KC, NT, NMAT>;
+  using C = StageCfg<KC, NT, NMAT, GROUP>;
   const int row0 = ti.e * R + ti.rb * kRowBlock;
   const int nkc = K / KC;
   const uint16_t* bsrc = a.xq;
@@ -284,11 +289,13 @@ __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& t
       if (NMAT == 2) tma_load_2d(st + C::CODE_BYTES, mq1, &full[s], kc * C::ROWB, row0);
       uint8_t* sc = st + NMAT * C::CODE_BYTES;
       if (KC == K) {
-        bulk_load(sc, s0_1d + static_cast<size_t>(row0) * (K / 32), C::SC_BYTES, &full[s]);
-        if (NMAT == 2) bulk_load(sc + C::SC_BYTES, s1_1d + static_cast<size_t>(row0) * (K / 32), C::SC_BYTES, &full[s]);
+        bulk_load(sc, s0_1d + static_cast<size_t>(row0) * (K / GROUP), C::SC_BYTES, &full[s]);
+        if (NMAT == 2)
+          bulk_load(sc + C::SC_BYTES, s1_1d + static_cast<size_t>(row0) * (K / GROUP), C::SC_BYTES, &full[s]);
       } else {
-        tma_load_2d(sc, ms0, &full[s], kc * (KC / 32), row0);
-        if (NMAT == 2) tma_load_2d(sc + C::SC_BYTES, ms1, &full[s], kc * (KC / 32), row0);
+        const int sx = GROUP == 32 ? kc * (KC / 32) : ((kc * (KC / 64)) & ~7);
+        tma_load_2d(sc, ms0, &full[s], sx, row0);
+        if (NMAT == 2) tma_load_2d(sc + C::SC_BYTES, ms1, &full[s], sx, row0);
       }
     }
     __syncwarp();
@@ -374,12 +381,12 @@ __device__ __forceinline__ void warp_combine_rows(const FfnArgs& a, int rb, int 
 }
 
 // Consumers: one tile.  Returns false on a timeout.
-template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE>
+template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP>
 __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, const TileInfo& ti, int K, int R,
                                              uint8_t* smem, float* red, uint64_t* full, uint64_t* empty,
                                              uint64_t* red_full, uint64_t* red_empty, int& s, uint32_t& ph,
                                              uint32_t& rph, volatile int* abort_flag, int warp, int lane) {
-  using C = StageCfg<KC, NT, NMAT>;
+  using C = StageCfg<KC, NT, NMAT, GROUP>;
   const int rw = warp & (kRowWarps - 1);   // 16-row slice
   const int half = warp / kRowWarps;       // which half of each stage's groups
   const int g = lane >> 2, c = lane & 3;
@@ -389,7 +396,9 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   // rl0 & 7 == (rl0 + 8) & 7 == g; bits 4..6 of cbase hold g, so chunk j is
   // cbase ^ (j << 4).
   const uint32_t cbase = rl0 * C::RSTR + (C::SWZ ? (g << 4) : 0) + 4 * c;
-  const uint32_t sbase = rl0 * C::SROWB + half * C::GPW * 2;
+  // this half's first scale: GPW 32-wide sub-groups are GPW scales (GROUP 32)
+  // or GPW / 2 scales (GROUP 64)
+  const uint32_t sbase = rl0 * C::SROWB + half * (GROUP == 32 ? C::GPW * 2 : C::GPW);
   const uint32_t xbase = C::W_BYTES + g * C::XROW + (half * C::GPW * 32 + 8 * c) * 2;
   const int nnt = (ti.ntok + 7) >> 3;
   const int nkc = K / KC;
@@ -408,7 +417,23 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
     const uint8_t* sc = st + NMAT * C::CODE_BYTES + sbase;
     // this warp's fp16 scales for its GPW groups (rows rl0 and rl0 + 8, both matrices)
     __half2 sh0[4], sh1[4], th0[4], th1[4];
-    if (C::GPW == 8) {
+    if (GROUP == 64) {
+      // the stage's scales start at element (kc * KC / 64) & 7 of the 8-scale box row
+      const uint8_t* sq = sc + ((kc * (KC / 64)) & 7) * 2;
+      if (C::GPW == 8) {   // 4 scales per half
+        const uint2 v0 = *reinterpret_cast<const uint2*>(sq);
+        const uint2 v1 = *reinterpret_cast<const uint2*>(sq + 8 * C::SROWB);
+        sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
+        sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y);
+      } else {             // GPW 4: 2 scales per half
+        sh0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq));
+        sh1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + 8 * C::SROWB));
+        if (NMAT == 2) {
+          th0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + C::SC_BYTES));
+          th1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + C::SC_BYTES + 8 * C::SROWB));
+        }
+      }
+    } else if (C::GPW == 8) {
       const uint4 v0 = *reinterpret_cast<const uint4*>(sc);
       const uint4 v1 = *reinterpret_cast<const uint4*>(sc + 8 * C::SROWB);
       sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y); sh0[2] = u32_as_half2(v0.z); sh0[3] = u32_as_half2(v0.w);
@@ -443,16 +468,17 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
       const uint8_t* ca = st + (C::SUBS == 1 ? 0 : (j >> 3) * C::SUB_BYTES) + (cbase ^ static_cast<uint32_t>(jc << 4));
       const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
       const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::RSTR);
-      const float s0 = half2_pick(sh0[jj >> 1], jj & 1);
-      const float s1 = half2_pick(sh1[jj >> 1], jj & 1);
+      const int si = GROUP == 32 ? jj : (jj >> 1);            // this sub-group's scale among the half's
+      const float s0 = half2_pick(sh0[si >> 1], si & 1);
+      const float s1 = half2_pick(sh1[si >> 1], si & 1);
       uint32_t pg[8], pu[8];
       dq_word_pair(pg, w0, w1);
       float t0 = 0.f, t1 = 0.f;
       if (NMAT == 2) {
         const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
         const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::RSTR);
-        t0 = half2_pick(th0[jj >> 1], jj & 1);
-        t1 = half2_pick(th1[jj >> 1], jj & 1);
+        t0 = half2_pick(th0[si >> 1], si & 1);
+        t1 = half2_pick(th1[si >> 1], si & 1);
         dq_word_pair(pu, v0, v1);
       }
 #pragma unroll
@@ -540,13 +566,13 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
 // The persistent FFN kernel (gate/up tiles, then down tiles).  Launched
 // cooperatively so that every CTA is resident: a down tile only waits for
 // gate/up tiles, which every CTA processes before any of its down tiles.
-template <int NT, bool SINGLE, int KCD>
+template <int NT, bool SINGLE, int KCD, int GROUP>
 __global__ void __launch_bounds__(kFfnThreads, 1)
     ffn_fused_kernel(const __grid_constant__ CUtensorMap gq, const __grid_constant__ CUtensorMap uq,
                      const __grid_constant__ CUtensorMap gs, const __grid_constant__ CUtensorMap us,
                      const __grid_constant__ CUtensorMap dq, const __grid_constant__ CUtensorMap ds,
                      const FfnArgs a) {
-  using F = FusedCfg<NT, KCD>;
+  using F = FusedCfg<NT, KCD, GROUP>;
   constexpr int NS = F::NS, STAGE = F::STAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -613,10 +639,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     for (int tile = blockIdx.x; ok && tile < m.tiles_all; tile += gridDim.x) {
       const TileInfo ti = decode_tile<TOKB>(a, m, tile);
       if (!ti.down)
-        ok = produce_tile<256, NT, 2, NS, STAGE>(a, ti, &gq, &uq, &gs, &us, a.gate_s, a.up_s, a.H, a.I, m.nrb_gu,
+        ok = produce_tile<256, NT, 2, NS, STAGE, GROUP>(a, ti, &gq, &uq, &gs, &us, a.gate_s, a.up_s, a.H, a.I, m.nrb_gu,
                                                  smem, full, empty, s, ph, issued, abort_flag, lane);
       else
-        ok = produce_tile<KCD, NT, 1, NS, STAGE>(a, ti, &dq, &dq, &ds, &ds, a.down_s, a.down_s, a.I, a.H, m.nrb_gu,
+        ok = produce_tile<KCD, NT, 1, NS, STAGE, GROUP>(a, ti, &dq, &dq, &ds, &ds, a.down_s, a.down_s, a.I, a.H, m.nrb_gu,
                                                  smem, full, empty, s, ph, issued, abort_flag, lane);
     }
     if (!ok && lane == 0) {
@@ -640,10 +666,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     const TileInfo ti = decode_tile<TOKB>(a, m, tile);
     bool ok;
     if (!ti.down)
-      ok = consume_tile<256, NT, 2, SINGLE, NS, STAGE>(a, m, ti, a.H, a.I, smem, red, full, empty, red_full,
+      ok = consume_tile<256, NT, 2, SINGLE, NS, STAGE, GROUP>(a, m, ti, a.H, a.I, smem, red, full, empty, red_full,
                                                         red_empty, s, ph, rph, abort_flag, warp, lane);
     else
-      ok = consume_tile<KCD, NT, 1, SINGLE, NS, STAGE>(a, m, ti, a.I, a.H, smem, red, full, empty, red_full,
+      ok = consume_tile<KCD, NT, 1, SINGLE, NS, STAGE, GROUP>(a, m, ti, a.I, a.H, smem, red, full, empty, red_full,
                                                         red_empty, s, ph, rph, abort_flag, warp, lane);
     if (!ok) return;
   }

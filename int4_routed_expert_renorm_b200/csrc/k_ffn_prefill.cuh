@@ -252,7 +252,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int NMAT>
+// GROUP: K elements per fp16 scale.  GROUP 32: a 64-wide chunk has two scales,
+// one per 32-wide K half.  GROUP 64: one scale per chunk; a stage's 4 scales
+// are half of a 16-byte box of 8 (the scale map's box), so two consecutive
+// stages load the same box and each reads its own half (K a multiple of 512).
+template <int NMAT, int GROUP>
 __global__ void __launch_bounds__(kPfThreads, 1)
     ffn_prefill_kernel(const __grid_constant__ CUtensorMap mq0, const __grid_constant__ CUtensorMap mq1,
                        const __grid_constant__ CUtensorMap ms0, const __grid_constant__ CUtensorMap ms1,
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int mbk = R / kRowBlock;
   const int nk = K / 64;
   const int cps = (K % 256 == 0) ? 4 : 2;            // 64-wide chunks per code stage
-  const bool one_stage = (K == cps * 64);            // scales then move by one 1-D copy
+  const bool one_stage = GROUP == 32 && (K == cps * 64);   // scales then move by one 1-D copy
   const int tiles = total_blocks * mbk;
 
   if (warp == 0) {
@@ -356,8 +360,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               bulk_load(sdst + C::SC_SLOT, a.s1 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4,
                         &code_full[cs]);
           } else {
-            tma_load_2d(sdst, &ms0, &code_full[cs], kb * 2, row0);
-            if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, &ms1, &code_full[cs], kb * 2, row0);
+            const int sx = GROUP == 32 ? kb * 2 : (kb & ~7);
+            tma_load_2d(sdst, &ms0, &code_full[cs], sx, row0);
+            if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, &ms1, &code_full[cs], sx, row0);
           }
           ++cst;
         }
@@ -510,7 +515,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             const uint8_t* sp = stg + NMAT * C::CODE_SLOT + m * C::SC_SLOT + r * cps * 4;
-            if (cps == 4) {
+            if (GROUP == 64) {                         // 4 scales at element (kb - ci) & 7 of the 8-scale row
+              const uint2 v = *reinterpret_cast<const uint2*>(sp + ((kb - ci) & 7) * 2);
+              scl[m][0] = v.x; scl[m][1] = v.y; scl[m][2] = 0u; scl[m][3] = 0u;
+            } else if (cps == 4) {
               const uint4 v = *reinterpret_cast<const uint4*>(sp);
               scl[m][0] = v.x; scl[m][1] = v.y; scl[m][2] = v.z; scl[m][3] = v.w;
             } else {
@@ -535,8 +543,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-          const uint32_t sw = ci == 0 ? scl[m][0] : ci == 1 ? scl[m][1] : ci == 2 ? scl[m][2] : scl[m][3];
-          const uint32_t sh = sw >> (g * 16);
+          uint32_t sh;
+          if (GROUP == 64) {                           // chunk ci's one scale, for both K halves
+            sh = (ci < 2 ? scl[m][0] : scl[m][1]) >> ((ci & 1) * 16);
+          } else {
+            const uint32_t sw = ci == 0 ? scl[m][0] : ci == 1 ? scl[m][1] : ci == 2 ? scl[m][2] : scl[m][3];
+            sh = sw >> (g * 16);
+          }
           const uint16_t sb = float_to_bf16_bits(half_bits_to_float(static_cast<uint16_t>(sh & 0xFFFFu)));
           const uint32_t s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
           const uint32_t wd[4] = {cw[m].x, cw[m].y, cw[m].z, cw[m].w};

@@ -24,6 +24,13 @@ class MoELayer:
                  bias: torch.Tensor | None = None):
         self.dims = dims
         self.t = dict(tensors)
+        H, I, G = dims.hidden, dims.inter, dims.group
+        n = dims.n_experts + dims.n_shared
+        want = {"gate_q": (n, I, H // 2), "up_q": (n, I, H // 2), "down_q": (n, H, I // 2),
+                "gate_s": (n, I, H // G), "up_s": (n, I, H // G), "down_s": (n, H, I // G)}
+        for name, shp in want.items():
+            if self.t[name].numel() != shp[0] * shp[1] * shp[2]:
+                raise ValueError(f"{name}: {self.t[name].numel()} elements, the dims need {shp}")
         self.router_w = router_w
         self.bias = bias
         p = lambda x: None if x is None else ctypes.c_void_p(x.data_ptr())  # noqa: E731

@@ -171,8 +171,13 @@ DECODE_B1_E16 = LayerShape("glm52_layer_decode_b1_e16", 6144, 2048, 16, 8, 1, 1)
 # Prefill tiles of the same shape as PREFILL_4096 (~128 tokens on every expert;
 # 32 routed + 1 shared expert resident, 0.7 GB): for profiler captures.
 PREFILL_512_E32 = LayerShape("glm52_layer_prefill_512_e32", 6144, 2048, 32, 8, 1, 512, logits_in=True)
+# The same layer in the group-scaled gs64 container (one fp16 scale per 64
+# codes along K; 20,054,016 bytes per expert instead of 21,233,664).
+DECODE_B1_GS64 = LayerShape("glm52_layer_decode_b1_gs64", 6144, 2048, 256, 8, 1, 1, group=64)
+PREFILL_4096_GS64 = LayerShape("glm52_layer_prefill_4096_gs64", 6144, 2048, 256, 8, 1, 4096, group=64,
+                               logits_in=True)
 WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16,
-                                 PREFILL_512_E32)}
+                                 PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64)}
 
 
 class LayerInputs:
@@ -199,7 +204,7 @@ class LayerInputs:
         return code_bytes(self.keys[kind], e * n, n).reshape(rows, k // 2)
 
     def expert_scales(self, kind: int, e: int) -> np.ndarray:
-        """uint16 fp16 bits [rows, K/32] of expert ``e``."""
+        """uint16 fp16 bits [rows, K/group] of expert ``e``."""
         n = self.per_expert(kind)
         h, i, g = self.shape.hidden, self.shape.inter, self.shape.group
         rows, k = (h, i) if kind == DOWN_S else (i, h)

@@ -58,7 +58,7 @@ def expert_tensors(shape: LayerShape, seed: int = 0, layer: int = 0, device="cud
         fill_codes(q, stream_key(seed, layer, kind))
         out[name + "_q"] = q
     for name, kind, (r, K) in (("gate", GATE_S, (I, H)), ("up", UP_S, (I, H)), ("down", DOWN_S, (H, I))):
-        s = torch.empty((n, r, K // 32), dtype=torch.int16, device=device)
+        s = torch.empty((n, r, K // shape.group), dtype=torch.int16, device=device)
         fill_scales(s, stream_key(seed, layer, kind))
         out[name + "_s"] = s
     return out

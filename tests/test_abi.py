@@ -59,7 +59,13 @@ def test_workspace_bytes(colimoe):
     assert 0 < n1 < n64
     # ypair rows (T*k + S*T) x H fp32 dominate: at least that much
     assert n64 >= (64 * 8 + 64) * 6144 * 4
-    assert m.coli_moe_workspace_bytes(_dims(m, group=64), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, group=64), 4) == m.coli_moe_workspace_bytes(d, 4)
+    assert m.coli_moe_workspace_bytes(_dims(m, group=16), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, group=128), 4) == 0
+    # group 64 reads scales in boxes of 8 (512 codes): H and I multiples of 512
+    assert m.coli_moe_workspace_bytes(_dims(m, group=64, hidden=6400), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, group=64, inter=768), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, group=32, hidden=6400, inter=768), 4) > 0
     assert m.coli_moe_workspace_bytes(_dims(m, hidden=6000), 4) == 0
     assert m.coli_moe_workspace_bytes(_dims(m, top_k=300), 4) == 0
 
@@ -98,7 +104,8 @@ def test_layer_argument_checks(colimoe):
     L = lambda d_, w_, x_, T, ws_, nbytes, flags=0: lib.coli_moe_layer(  # noqa: E731
         ctypes.byref(d_), ctypes.byref(w_), x_, T, None, None, flags, out, None, None, None, ws_, nbytes, None)
     assert L(d, w, x, 4, ws, need - 1) == m._lib.COLI_ERR_WORKSPACE
-    assert L(_dims(m, group=64), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, group=16), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, group=64, inter=1280), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, inter=384), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, n_shared=9), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(d, _weights(m, misalign=True), x, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG

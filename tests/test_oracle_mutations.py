@@ -52,6 +52,15 @@ def _interleaved_scales(q_bytes, s_bits, group=32):
     return (q.reshape(rows, group, k // group) * s[:, None, :]).reshape(rows, k)
 
 
+def _scale_per_32_codes(q_bytes, s_bits, group=32):
+    """Every scale applied to 32 codes whatever the group, the row's tail
+    keeping the last scale."""
+    q = M.unpack_int4(q_bytes).astype(np.float64)
+    s = M.fp16_bits_to_f64(s_bits)
+    idx = np.minimum(np.arange(q.shape[1]) // 32, s.shape[1] - 1)
+    return q * s[:, idx]
+
+
 def _route_high_index_ties(l32, k):
     l = np.asarray(l32, dtype=np.float32).astype(np.float64)
     T, E = l.shape
@@ -124,6 +133,7 @@ MUTATIONS = {
     "nibble order swapped": ("unpack_int4", _swap_nibbles),
     "offset-8 codes instead of two's complement": ("unpack_int4", _offset_codes),
     "scale group index transposed": ("dequant", _interleaved_scales),
+    "group size ignored (32 codes per scale)": ("dequant", _scale_per_32_codes),
     "ties to the highest index": ("route", _route_high_index_ties),
     "weights not renormalised": ("route", _route_not_renormalised),
     "union not stable": ("batch_union", _union_unstable),

@@ -57,18 +57,43 @@ def test_dequant_hand_worked():
 
 
 def test_dequant_group_index_and_rows():
-    """Scale (r, c // 32) multiplies element (r, c): each scale set to a power
-    of two tagging its (row, group) is recovered from a code-1 matrix."""
-    rows, K = 3, 128
+    _check_group_index(32)
+
+
+def test_dequant_gs64_group_index_and_rows():
+    """Group 64 is the gs64 container (Colibri README, "2. Scarica il modello")."""
+    _check_group_index(64)
+
+
+def _check_group_index(group):
+    """Scale (r, c // group) multiplies element (r, c): each scale set to a
+    power of two tagging its (row, group) is recovered from a code-1 matrix."""
+    rows, K = 3, 256
+    ng = K // group
     q = np.full((rows, K // 2), 0x11, np.uint8)            # every code = +1
-    s = np.zeros((rows, K // 32), np.float16)
+    s = np.zeros((rows, ng), np.float16)
     for r in range(rows):
-        for g in range(K // 32):
-            s[r, g] = 2.0 ** -(r * 4 + g)
-    W = oracle.dequant(q, s.view(np.uint16), 32)
+        for g in range(ng):
+            s[r, g] = 2.0 ** -(r * ng + g)
+    W = oracle.dequant(q, s.view(np.uint16), group)
     for r in range(rows):
         for c in range(K):
-            assert W[r, c] == 2.0 ** -(r * 4 + c // 32)
+            assert W[r, c] == 2.0 ** -(r * ng + c // group)
+
+
+def test_dequant_gs64_is_gs32_with_paired_scales():
+    """A group-64 container equals the group-32 container whose two scales of
+    every 64-wide span are both that span's scale (seeded codes and scales)."""
+    rng = np.random.default_rng(64)
+    rows, K = 5, 512
+    q = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    s64 = rng.uniform(0.005, 0.02, (rows, K // 64)).astype(np.float16)
+    s32 = np.repeat(s64, 2, axis=1)
+    W64 = oracle.dequant(q, s64.view(np.uint16), 64)
+    W32 = oracle.dequant(q, s32.view(np.uint16), 32)
+    assert np.array_equal(W64, W32)
+    codes = oracle.unpack_int4(q).astype(np.float64)
+    assert np.array_equal(W64, codes * np.repeat(s64.astype(np.float64), 64, axis=1))
 
 
 def test_round_bf16_matches_torch_on_fp32_inputs():
