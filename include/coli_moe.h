@@ -183,7 +183,7 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
  *   - Arguments and results are those of coli_moe_layer, without ws/ws_bytes.
  *   - Batches whose coli_moe_workspace_bytes(dims, T) exceeds
  *     COLI_NOALLOC_SCRATCH_BYTES are rejected with COLI_ERR_WORKSPACE before
- *     anything is launched (up to 21 tokens for H=6144, I=2048, E=256, k=8, S=1).
+ *     anything is launched (up to 87 tokens for H=6144, I=2048, E=256, k=8, S=1).
  *   - The first call on a device looks up the array's device address (one
  *     cudaGetSymbolAddress with that device current); make that first call
  *     before capturing a stream.  No call allocates or frees device memory.
@@ -192,7 +192,7 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
  *     Calls that can overlap on the GPU (different streams without ordering
  *     between them) race on the array and give undefined results: order them.
  */
-#define COLI_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define COLI_NOALLOC_SCRATCH_BYTES (32u << 20)
 coli_status coli_moe_layer_noalloc(const coli_moe_dims *dims, const coli_moe_weights *w,
                                    const uint16_t *x, int T, const float *logits_in,
                                    const uint16_t *residual, uint32_t flags, uint16_t *out,

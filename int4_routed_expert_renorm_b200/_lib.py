@@ -23,7 +23,7 @@ COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
            "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc")
-COLI_NOALLOC_SCRATCH_BYTES = 8 << 20
+COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class ColiError(RuntimeError):

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "k_ffn_decode.cuh"
 #include "k_ffn_prefill.cuh"
+#include "k_ffn_splitk.cuh"
 #include "k_router.cuh"
 #include "k_union.cuh"
 
@@ -102,6 +103,14 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_PF_SMEM(2, 64)
     COLI_SET_PF_SMEM(1, 64)
 #undef COLI_SET_PF_SMEM
+#define COLI_SET_SK_SMEM(SG, GR)                                                                        \
+  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<SG, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(SkCfg<GR>::SMEM)) == cudaSuccess;
+    COLI_SET_SK_SMEM(true, 32)
+    COLI_SET_SK_SMEM(false, 32)
+    COLI_SET_SK_SMEM(true, 64)
+    COLI_SET_SK_SMEM(false, 64)
+#undef COLI_SET_SK_SMEM
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
     ok &= cudaFuncSetAttribute(union_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -201,6 +210,10 @@ struct Ws {
   size_t bytes;
 };
 
+// Split-K form: batches of <= kSkMaxT tokens whose down scale rows are whole
+// 16-byte units (I a multiple of 256; of 512 with 64-wide groups, as always).
+inline bool use_splitk(const coli_moe_dims* d, int T) { return T <= kSkMaxT && d->inter % 256 == 0; }
+
 Ws layout(const coli_moe_dims* d, int T, void* base) {
   Ws ws{};
   const size_t H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
@@ -237,7 +250,11 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
     ws.rb_done = static_cast<int32_t*>(take(H / 128 * 4));
   }
   ws.hq = static_cast<uint16_t*>(take(rows * I * 2));
-  ws.ypair = static_cast<float*>(take(rows * H * 4));
+  {
+    // the split-K form keeps y as I/128 partials per (pair, row) in the same region
+    const size_t yb = rows * H * 4, pb = use_splitk(d, T) ? rows * (I / 128) * H * 4 : 0;
+    ws.ypair = static_cast<float*>(take(yb > pb ? yb : pb));
+  }
   ws.bytes = o;
   return ws;
 }
@@ -272,14 +289,16 @@ bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K
   return true;
 }
 
-// The persistent FFN kernel is launched cooperatively (all CTAs resident, so
-// the counter waits of down tiles on gate/up tiles always make progress).
-template <int NT, bool SG, int KCD, int GR>
-bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
+// The persistent FFN kernels are launched cooperatively (all CTAs resident,
+// so the counter waits between CTAs always make progress).
+using FfnKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, FfnArgs);
+
+bool launch_cooperative(FfnKernel kernel, size_t smem, const CUtensorMap* m, const FfnArgs& a, int grid,
+                        cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kFfnThreads);
-  cfg.dynamicSmemBytes = FusedCfg<NT, KCD, GR>::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -289,14 +308,19 @@ bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStre
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   ++t_launches;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD, GR>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, m[0], m[1], m[2], m[3], m[4], m[5], a);
   if (e != cudaSuccess) {
     // without overlap with the previous kernel
     cudaGetLastError();
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel<NT, SG, KCD, GR>, m[0], m[1], m[2], m[3], m[4], m[5], a);
+    e = cudaLaunchKernelEx(&cfg, kernel, m[0], m[1], m[2], m[3], m[4], m[5], a);
   }
   return e == cudaSuccess;
+}
+
+template <int NT, bool SG, int KCD, int GR>
+bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
+  return launch_cooperative(ffn_fused_kernel<NT, SG, KCD, GR>, FusedCfg<NT, KCD, GR>::SMEM, m, a, grid, st);
 }
 
 // Decode-form variant for this batch: one token per tile when T == 1, 8-token
@@ -545,6 +569,24 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   a.E = E;
   a.S = S;
   a.P = P;
+  if (use_splitk(d, T)) {
+    // down maps of the split-K form: codes in boxes of 128 rows x 64 bytes
+    // (one 128-wide K slice, 64B swizzle), scales in boxes of 8 x 128 rows
+    if (!encode_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->down_q, I / 2, rows_dn, I / 2, 64, kRowBlock,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_2d(&maps[5], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->down_s, I / G, rows_dn, (I / G) * 2, 8, kRowBlock,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return COLI_ERR_CUDA;
+    a.ypart = ws.ypair;
+    const long tiles = blocks_ub * (I / kRowBlock);
+    const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
+    FfnKernel k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32> : ffn_splitk_kernel<true, 64>)
+                         : (G == 32 ? ffn_splitk_kernel<false, 32> : ffn_splitk_kernel<false, 64>);
+    if (!launch_cooperative(k, G == 32 ? SkCfg<32>::SMEM : SkCfg<64>::SMEM, maps, a, grid, st)) return COLI_ERR_CUDA;
+    rec.mark_through(6, 7);
+    rec.mark(8);
+    return COLI_OK;
+  }
   {
     const long tiles = blocks_ub * (I / kRowBlock + H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);

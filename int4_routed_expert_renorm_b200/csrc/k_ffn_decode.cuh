@@ -48,6 +48,7 @@ struct FfnArgs {
   const uint16_t* xq;        // fragment-ordered expert input [T][H]
   uint16_t* hq;              // h, fragment-ordered [P+S*T][I]
   float* ypair;              // y [P+S*T][H]
+  float* ypart;              // split-K form: y partials [P+S*T][I/128][H]
   const uint16_t* gate_s;    // scales for 1-D copies when a stage spans all of K
   const uint16_t* up_s;
   const uint16_t* down_s;
@@ -380,12 +381,21 @@ __device__ __forceinline__ void warp_combine_rows(const FfnArgs& a, int rb, int 
   }
 }
 
-// Consumers: one tile.  Returns false on a timeout.
-template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP>
+// Padded row of one token's 128-element h slice in shared memory (split-K form).
+constexpr int kSkHRow = 128 * 2 + 64;
+
+// Consumers: one tile.  Returns false on a timeout.  HSMEM (gate/up of the
+// split-K form): h of the tile's 128 rows goes to the shared-memory slice
+// buffer `hbuf` ([token][kSkHRow bytes], fragment order) once every consumer
+// warp has released the previous unit's slice (h_free), and is announced on
+// h_ready; nothing is written to global memory.
+template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP, bool HSMEM = false>
 __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, const TileInfo& ti, int K, int R,
                                              uint8_t* smem, float* red, uint64_t* full, uint64_t* empty,
                                              uint64_t* red_full, uint64_t* red_empty, int& s, uint32_t& ph,
-                                             uint32_t& rph, volatile int* abort_flag, int warp, int lane) {
+                                             uint32_t& rph, volatile int* abort_flag, int warp, int lane,
+                                             uint16_t* hbuf = nullptr, uint64_t* h_free = nullptr,
+                                             uint64_t* h_ready = nullptr, uint32_t lu = 0) {
   using C = StageCfg<KC, NT, NMAT, GROUP>;
   const int rw = warp & (kRowWarps - 1);   // 16-row slice
   const int half = warp / kRowWarps;       // which half of each stage's groups
@@ -526,6 +536,22 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   mbar_arrive(&red_empty[rw]);
   rph ^= 1u;
   // epilogue: d0 (row g, col 2c), d1 (row g, col 2c+1), d2 (row g+8, col 2c), d3 (row g+8, col 2c+1)
+  if (HSMEM) {
+    static_assert(!HSMEM || (NMAT == 2 && NT == 1), "h slices in shared memory are for 8-token gate/up tiles");
+    if (lu > 0 && !mbar_wait(h_free, (lu - 1) & 1u, abort_flag, a.status)) return false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = 2 * c + (q & 1);
+      if (i < ti.ntok && !(SINGLE && (q & 1))) {
+        const float gv = acc0[0][q], uv = acc1[0][q];
+        const float hv = gv / (1.0f + expf(-gv)) * uv;
+        hbuf[i * (kSkHRow / 2) + frag_pos(rl0 + ((q & 2) ? 8 : 0))] = float_to_bf16_bits(hv);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(h_ready);
+    return true;
+  }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if (nt < nnt) {

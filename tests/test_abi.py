@@ -133,3 +133,17 @@ def test_binding_fails_loudly_without_library(tmp_path):
     from int4_routed_expert_renorm_b200 import _lib
     with pytest.raises(ImportError):
         _lib.load(str(tmp_path / "libcolimoe.so"))
+
+
+def test_binding_constants_match_the_header(colimoe):
+    """Every #define of the header that the binding mirrors has the same value."""
+    src = open(os.path.join(ROOT, "include", "coli_moe.h")).read()
+    found = 0
+    for m in re.finditer(r"#define\s+(COLI_[A-Z_]+)\s+\(?(0x[0-9a-fA-F]+|\d+)u?(?:\s*<<\s*(\d+))?\)?", src):
+        name, val, sh = m.group(1), int(m.group(2), 0), m.group(3)
+        if sh:
+            val <<= int(sh)
+        if hasattr(colimoe._lib, name):
+            assert getattr(colimoe._lib, name) == val, name
+            found += 1
+    assert found >= 7
