@@ -68,20 +68,20 @@ def parse():
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture
-# of the same kernel build: (workload, FFN form) -> bytes.  The batch-1 capture
-# ran on the 16-expert variant of the layer, which moves the same 9 experts per
-# step (profiles/ffn_fused_kernel_glm52_layer_decode_b1_e16.md).
-# The prefill capture ran on the 32-expert, 512-token variant (same tile
+# of the same kernel build: (workload, FFN form) -> bytes.  The prefill capture ran on the 32-expert, 512-token variant (same tile
 # shapes): there DRAM traffic was 1.063x the algorithmic bytes of the gate/up
 # launch (profiles/ffn_prefill_kernel_glm52_layer_prefill_512_e32.md); the
 # 4096-token figure is that ratio times its own algorithmic bytes (257 experts'
 # gate+up codes and scales, 36,864 gathered rows, h written).
 _PF_RATIO = (532.544256e6 + 16.89984e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
-TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.752704e6 + 4.751616e6,
-           ("glm52_layer_decode_b1_e16", "decode"): 191.752704e6 + 4.751616e6,
-           ("glm52_layer_prefill_512_e32", "prefill"): 532.544256e6 + 16.89984e6,
+TRAFFIC = {("glm52_layer_prefill_512_e32", "prefill"): 532.544256e6 + 16.89984e6,
            ("glm52_layer_prefill_4096", "prefill"):
                _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)}
+
+
+def splitk_form(shape) -> bool:
+    """The library's decode form for batches of <= 8 tokens (I a multiple of 256)."""
+    return shape.tokens <= 8 and shape.inter % 256 == 0
 
 
 def prefill_form(shape) -> bool:
@@ -412,6 +412,17 @@ def main():
                 "kernel": "ffn_prefill_kernel<2> (gate/up grouped GEMM, tcgen05 kind::f16, A in TMEM)",
                 "algorithmic": f"{flops} FLOP per launch = 4*H*I per (pair or shared row)",
                 "peak_kind": f"{src} burst bf16"}
+    elif splitk_form(shape):
+        act = T * H * 2 * (3 if shape.prenorm else 2)      # x read, out write (+ residual read)
+        per_launch = [(u + S) * shape.expert_bytes() + act for u in u_step]
+        achieved = statistics.mean(b / (ms / 1e3) / 1e9 for b, ms in zip(per_launch, gu_ms))
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": None,
+                "kernel": "ffn_splitk_kernel (decode form for T <= 8: gate/up, split-K down and combine in one "
+                          "launch)",
+                "algorithmic": "int4 codes + fp16 scales of every unique and shared expert (3 matrices) "
+                               "+ x read + out write" + (" + residual read" if shape.prenorm else ""),
+                "peak_kind": f"{src} HBM copy"}
     else:
         rows = P + S * T
         fused_combine = T <= 4

@@ -57,6 +57,7 @@ struct SkCfg {
   static_assert(2 * NS + 2 * kRowWarps + 4 <= NBAR, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(kSkDnCode % 1024 == 0, "64B-swizzled boxes need 512-byte alignment");
+  static_assert(H_BYTES >= kSkMaxT * 32 * 8, "the combine's pair_pos / topk_w copies fit in the h buffer");
 };
 
 // Producer: the down stages of one unit (K slice rb of expert e, every output
@@ -191,11 +192,14 @@ __device__ __forceinline__ bool wait_counter(const int32_t* cnt, int target, vol
   }
 }
 
-// out rows of this CTA after every partial is in: see the file comment.  The
-// idle stage ring holds the per-pair sums.  `cbar` (count: consumer warps)
-// separates the two passes; returns false on a timeout.
-__device__ __forceinline__ bool splitk_combine(const FfnArgs& a, uint8_t* ring, int ring_bytes, uint64_t* cbar,
-                                               uint32_t& cph, volatile int* abort_flag, int warp, int lane) {
+// The CTA's share of the output after every partial is in: see the file
+// comment.  pos_s / w_s are shared-memory copies of pair_pos and topk_w
+// (T*k each, made before the grid-wide wait); the idle stage ring holds the
+// per-pair sums.  `cbar` (count: consumer warps) separates the two passes;
+// returns false on a timeout.
+__device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* pos_s, const float* w_s,
+                                               uint8_t* ring, int ring_bytes, uint64_t* cbar, uint32_t& cph,
+                                               volatile int* abort_flag, int warp, int lane) {
   const int tid = warp * 32 + lane;
   const int nthr = kFfnConsumerWarps * 32;
   const int q4 = a.H / 4;
@@ -208,35 +212,52 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, uint8_t* ring, 
   float4* ysum = reinterpret_cast<float4*>(ring);
   for (int cu = u0; cu < u1; cu += ch) {
     const int cn = (u1 - cu) < ch ? (u1 - cu) : ch;
+    // this thread's output unit of the second pass: its residual load goes
+    // out now and lands while the first pass runs
+    uint2 rv = make_uint2(0u, 0u);
+    if (a.residual && tid < cn) {
+      const int u = cu + tid;
+      const int t = u / q4, r = (u - t * q4) * 4;
+      rv = __ldg(reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r));
+    }
     // y of one (token, 4 rows, pair) by a quad of lanes: lane p sums the
     // slices p, p+4, ... in order, then the quad adds (p0 + p1) + (p2 + p3)
-    // (every lane ends with the same bits: each add is commutative)
-    for (int t0 = warp * 8; t0 < cn * nj; t0 += kFfnConsumerWarps * 8) {
-      const int task = t0 + (lane >> 2), p = lane & 3;
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (task < cn * nj) {
-        const int ui = task / nj, jj = task - ui * nj;
-        const int u = cu + ui;
-        const int t = u / q4, r = (u - t * q4) * 4;
-        const int row = jj < a.k ? __ldg(a.pair_pos + t * a.k + jj) : a.P + (jj - a.k) * a.T + t;
-        const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
+    // (every lane ends with the same bits: each add is commutative); two
+    // tasks per quad and round keep 8 loads in flight per lane
+    for (int t0 = warp * 16; t0 < cn * nj; t0 += kFfnConsumerWarps * 16) {
+      float4 y[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int task = t0 + 8 * h + (lane >> 2), p = lane & 3;
+        y[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (task < cn * nj) {
+          const int ui = task / nj, jj = task - ui * nj;
+          const int u = cu + ui;
+          const int t = u / q4, r = (u - t * q4) * 4;
+          const int row = jj < a.k ? pos_s[t * a.k + jj] : a.P + (jj - a.k) * a.T + t;
+          const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
 #pragma unroll 4
-        for (int sl = p; sl < nsl; sl += 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * a.H));
-          y.x += v.x;
-          y.y += v.y;
-          y.z += v.z;
-          y.w += v.w;
+          for (int sl = p; sl < nsl; sl += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * a.H));
+            y[h].x += v.x;
+            y[h].y += v.y;
+            y[h].z += v.z;
+            y[h].w += v.w;
+          }
         }
       }
 #pragma unroll
-      for (int m = 1; m <= 2; m <<= 1) {
-        y.x += __shfl_xor_sync(0xffffffffu, y.x, m);
-        y.y += __shfl_xor_sync(0xffffffffu, y.y, m);
-        y.z += __shfl_xor_sync(0xffffffffu, y.z, m);
-        y.w += __shfl_xor_sync(0xffffffffu, y.w, m);
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int m = 1; m <= 2; m <<= 1) {
+          y[h].x += __shfl_xor_sync(0xffffffffu, y[h].x, m);
+          y[h].y += __shfl_xor_sync(0xffffffffu, y[h].y, m);
+          y[h].z += __shfl_xor_sync(0xffffffffu, y[h].z, m);
+          y[h].w += __shfl_xor_sync(0xffffffffu, y[h].w, m);
+        }
+        const int task = t0 + 8 * h + (lane >> 2);
+        if ((lane & 3) == 0 && task < cn * nj) ysum[task] = y[h];
       }
-      if (p == 0 && task < cn * nj) ysum[task] = y;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(cbar);
@@ -247,7 +268,7 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, uint8_t* ring, 
       const int t = u / q4, r = (u - t * q4) * 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int j = 0; j < a.k; ++j) {
-        const float w = __ldg(a.topk_w + t * a.k + j);
+        const float w = w_s[t * a.k + j];
         const float4 y = ysum[ui * nj + j];
         acc.x = fmaf(w, y.x, acc.x);
         acc.y = fmaf(w, y.y, acc.y);
@@ -262,7 +283,8 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, uint8_t* ring, 
         acc.w += y.w;
       }
       if (a.residual) {
-        const uint2 rv = *reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r);
+        if (ui != tid)
+          rv = __ldg(reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r));
         acc.x += __uint_as_float(rv.x << 16);
         acc.y += __uint_as_float(rv.x & 0xffff0000u);
         acc.z += __uint_as_float(rv.y << 16);
@@ -403,13 +425,25 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   if (lane == 0) mbar_arrive(cbar);
   if (!mbar_wait(cbar, cph, abort_flag, a.status)) return;
   cph ^= 1u;
+  // the h slice buffer is free now: it takes the batch's pair_pos and
+  // topk_w for the combine while the grid-wide wait runs
+  int32_t* pos_s = reinterpret_cast<int32_t*>(hbuf);
+  float* w_s = reinterpret_cast<float*>(pos_s + kSkMaxT * 32);
+  for (int i = warp * 32 + lane; i < a.T * a.k; i += kFfnConsumerWarps * 32) {
+    pos_s[i] = __ldg(a.pair_pos + i);
+    w_s[i] = __ldg(a.topk_w + i);
+  }
   if (warp == 0 && lane == 0) {
     __threadfence();
     atomicAdd(a.rb_done, 1);
     if (wait_counter(a.rb_done, static_cast<int>(gridDim.x), abort_flag, a.status)) mbar_arrive(gbar);
   }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(cbar);
+  if (!mbar_wait(cbar, cph, abort_flag, a.status)) return;
+  cph ^= 1u;
   if (!mbar_wait(gbar, 0, abort_flag, a.status)) return;
-  splitk_combine(a, smem, NS * STAGE, cbar, cph, abort_flag, warp, lane);
+  splitk_combine(a, pos_s, w_s, smem, NS * STAGE, cbar, cph, abort_flag, warp, lane);
 }
 
 }  // namespace coli
