@@ -21,7 +21,8 @@
  *            w_j = exp(l'_j - l'_max) / sum_{i<k} exp(l'_i - l'_max)
  *   union    unique experts ascending; pairs p = t*k + j grouped by expert,
  *            stable in p
- *   expert   W = code * scale, code int4 in [-8,7], fp16 scale per G along K;
+ *   expert   W = code * scale, code int4 in [-8,7] (or int8 in [-128,127]),
+ *            fp16 scale per G along K;
  *            h = bf16( silu(W_gate x) * (W_up x) ),  y = W_down h   (fp32 accumulate)
  *   combine  out[t] = bf16( sum_j w[t,j] * y_{id[t,j]} + sum_s y_{E+s} + residual[t] )
  *
@@ -33,6 +34,11 @@
  *   multiplies its element c.
  *   Element c of a row is nibble (c & 1) of byte c/2 (low nibble first); the
  *   nibble n encodes code n - 16*(n >= 8).  Shared experts are ids E..E+S-1.
+ *   int8 container (dims.code_bits == 8; the README requires the MTP head to
+ *   be int8, "Decodifica speculativa, onestamente"): the same layout with one
+ *   two's-complement byte per code, gate_q/up_q [E+S][I][H], down_q
+ *   [E+S][H][I].  It runs in the decode form for T <= 8 (the MTP head's draft
+ *   batches); other batches and the prefill form return COLI_ERR_UNSUPPORTED.
  *
  * Conventions for every call:
  *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
@@ -48,7 +54,8 @@
  *     status word that coli_moe_get_status reads and clears; kernels never
  *     trap.
  *   - Supported shapes: group == 32 with H % 256 == 0, I % 256 == 0 or
- *     I == 128; group == 64 with H % 512 == 0, I % 512 == 0; and for both
+ *     I == 128; group == 64 with H % 512 == 0, I % 512 == 0; int8 codes
+ *     need I % 256 == 0 (group 32) or I % 512 == 0 (group 64); and for all
  *     1 <= k <= min(E, 32), E <= 1024, 0 <= S <= 4, T >= 0, T*k <= 2^24.
  *     Anything else returns COLI_ERR_UNSUPPORTED.
  *   - Thread safety: calls may be made concurrently from several host
@@ -95,6 +102,7 @@ typedef struct {
   int32_t top_k;      /* k */
   int32_t n_shared;   /* S: shared experts, always active with weight 1.0 */
   int32_t group;      /* quantisation group along K: 32 or 64 */
+  int32_t code_bits;  /* code container: 4 (or 0) = int4, two codes per byte; 8 = int8, one code per byte */
 } coli_moe_dims;
 
 typedef struct {

@@ -34,7 +34,8 @@ class ColiError(RuntimeError):
 
 class coli_moe_dims(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
-                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("group", ctypes.c_int32)]
+                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("code_bits", ctypes.c_int32)]
 
 
 class coli_moe_weights(ctypes.Structure):

@@ -11,8 +11,9 @@ import torch
 from ._lib import coli_moe_dims, coli_moe_layer, coli_moe_weights, coli_moe_workspace_bytes
 
 
-def dims_for(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int, group: int = 32) -> coli_moe_dims:
-    return coli_moe_dims(hidden, inter, n_experts, top_k, n_shared, group)
+def dims_for(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int, group: int = 32,
+             code_bits: int = 4) -> coli_moe_dims:
+    return coli_moe_dims(hidden, inter, n_experts, top_k, n_shared, group, code_bits)
 
 
 class MoELayer:
@@ -26,7 +27,8 @@ class MoELayer:
         self.t = dict(tensors)
         H, I, G = dims.hidden, dims.inter, dims.group
         n = dims.n_experts + dims.n_shared
-        want = {"gate_q": (n, I, H // 2), "up_q": (n, I, H // 2), "down_q": (n, H, I // 2),
+        cb = 8 if dims.code_bits == 8 else 4
+        want = {"gate_q": (n, I, H * cb // 8), "up_q": (n, I, H * cb // 8), "down_q": (n, H, I * cb // 8),
                 "gate_s": (n, I, H // G), "up_s": (n, I, H // G), "down_s": (n, H, I // G)}
         for name, shp in want.items():
             if self.t[name].numel() != shp[0] * shp[1] * shp[2]:

@@ -88,12 +88,23 @@ def unpack_int4(q_bytes: np.ndarray) -> np.ndarray:
     return (nib - 16 * (nib >= 8)).astype(np.int8)
 
 
-def dequant(q_bytes: np.ndarray, s_bits: np.ndarray, group: int = 32) -> np.ndarray:
+def unpack_int8(q_bytes: np.ndarray) -> np.ndarray:
+    """int8 container: codes uint8 [rows, K] -> signed codes int8 [rows, K].
+
+    READING (the README requires the MTP head to be int8, "Decodifica
+    speculativa, onestamente" and "2. Scarica il modello", but gives no
+    layout): the int4 container with one byte per code, element c of a row
+    in byte c, read as two's complement, so codes span [-128, 127]."""
+    return np.asarray(q_bytes, dtype=np.uint8).view(np.int8).copy()
+
+
+def dequant(q_bytes: np.ndarray, s_bits: np.ndarray, group: int = 32, bits: int = 4) -> np.ndarray:
     """Weights W[r, c] = code[r, c] * scale[r, c // group]   (float64, exact).
 
     Scales are fp16 [rows, K/group], one per group of ``group`` consecutive
-    elements along K (the row)."""
-    q = unpack_int4(q_bytes).astype(np.float64)
+    elements along K (the row).  ``bits`` selects the int4 (4) or int8 (8)
+    code container."""
+    q = (unpack_int4 if bits == 4 else unpack_int8)(q_bytes).astype(np.float64)
     s = fp16_bits_to_f64(s_bits)
     rows, k = q.shape
     assert s.shape == (rows, k // group)
@@ -202,15 +213,15 @@ class ExpertWeights:
     codes and fp16 scale bits for kind 'gate', 'up' or 'down'.  A small cache
     keeps the most recently dequantised matrices (``cache`` entries)."""
 
-    def __init__(self, get_codes, get_scales, group: int = 32, cache: int = 0):
-        self._c, self._s, self.group = get_codes, get_scales, group
+    def __init__(self, get_codes, get_scales, group: int = 32, cache: int = 0, bits: int = 4):
+        self._c, self._s, self.group, self.bits = get_codes, get_scales, group, bits
         self._cache, self._cap = {}, cache
 
     def matrix(self, kind: str, e: int) -> np.ndarray:
         key = (kind, e)
         if key in self._cache:
             return self._cache[key]
-        m = dequant(self._c(kind, e), self._s(kind, e), self.group)
+        m = dequant(self._c(kind, e), self._s(kind, e), self.group, self.bits)
         if self._cap:
             if len(self._cache) >= self._cap:
                 self._cache.pop(next(iter(self._cache)))
@@ -225,13 +236,13 @@ class ExpertWeights:
         sk = {"gate": synth.GATE_S, "up": synth.UP_S, "down": synth.DOWN_S}
         return ExpertWeights(lambda k, e: inputs.expert_codes(qk[k], e),
                              lambda k, e: inputs.expert_scales(sk[k], e),
-                             inputs.shape.group, cache)
+                             inputs.shape.group, cache, inputs.shape.bits)
 
     @staticmethod
-    def from_arrays(arrays: dict, group: int = 32) -> "ExpertWeights":
+    def from_arrays(arrays: dict, group: int = 32, bits: int = 4) -> "ExpertWeights":
         """arrays: {'gate': (codes, scales), 'up': (...), 'down': (...)} with a
         leading expert axis."""
-        return ExpertWeights(lambda k, e: arrays[k][0][e], lambda k, e: arrays[k][1][e], group)
+        return ExpertWeights(lambda k, e: arrays[k][0][e], lambda k, e: arrays[k][1][e], group, bits=bits)
 
 
 def expert_ffn_tokens(W: ExpertWeights, e: int, x64: np.ndarray) -> np.ndarray:

@@ -76,7 +76,7 @@ def words(key: int, start: int, count: int) -> np.ndarray:
 
 
 def code_bytes(key: int, start: int, count: int) -> np.ndarray:
-    """Bytes ``start .. start+count-1`` of a packed int4 code tensor (uint8)."""
+    """Bytes ``start .. start+count-1`` of a code tensor (uint8; int4 or int8 codes)."""
     w0 = start // 8
     w1 = (start + count + 7) // 8
     w = words(key, w0, w1 - w0)
@@ -148,15 +148,16 @@ class LayerShape:
     zipf_bias: bool = False
     logits_in: bool = False   # logits drawn i.i.d. N(0,1) instead of x @ W_r^T
     prenorm: bool = False     # stack: pre-RMSNorm and residual between layers
+    bits: int = 4             # code container: int4 (two codes per byte) or int8 (one per byte)
 
     @property
     def n_total(self) -> int:
         return self.n_experts + self.n_shared
 
     def expert_bytes(self) -> int:
-        """int4 codes + fp16 scales of one expert (gate, up and down)."""
+        """Codes + fp16 scales of one expert (gate, up and down)."""
         h, i, g = self.hidden, self.inter, self.group
-        return 3 * (h * i // 2) + 3 * (h * i // g) * 2
+        return 3 * (h * i * self.bits // 8) + 3 * (h * i // g) * 2
 
 
 # The five workloads (sizes of the GLM-5.2-shaped layer; tiny case for fast parity).
@@ -176,8 +177,12 @@ PREFILL_512_E32 = LayerShape("glm52_layer_prefill_512_e32", 6144, 2048, 32, 8, 1
 DECODE_B1_GS64 = LayerShape("glm52_layer_decode_b1_gs64", 6144, 2048, 256, 8, 1, 1, group=64)
 PREFILL_4096_GS64 = LayerShape("glm52_layer_prefill_4096_gs64", 6144, 2048, 256, 8, 1, 4096, group=64,
                                logits_in=True)
+# The same layer with int8 codes (the container the README requires for the MTP
+# head, whose drafts are decoded in batches of 1..4): 37,748,736 + 2,359,296
+# bytes per expert.
+DECODE_B1_INT8 = LayerShape("glm52_layer_int8_decode_b1", 6144, 2048, 256, 8, 1, 1, bits=8)
 WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16,
-                                 PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64)}
+                                 PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64, DECODE_B1_INT8)}
 
 
 class LayerInputs:
@@ -193,15 +198,16 @@ class LayerInputs:
     # flat element counts per expert for each tensor kind
     def per_expert(self, kind: int) -> int:
         h, i, g = self.shape.hidden, self.shape.inter, self.shape.group
-        return {GATE_Q: i * h // 2, UP_Q: i * h // 2, DOWN_Q: h * i // 2,
+        cb = h * i * self.shape.bits // 8
+        return {GATE_Q: cb, UP_Q: cb, DOWN_Q: cb,
                 GATE_S: i * h // g, UP_S: i * h // g, DOWN_S: h * i // g}[kind]
 
     def expert_codes(self, kind: int, e: int) -> np.ndarray:
-        """uint8 [rows, K/2] codes of expert ``e`` (gate/up: rows=I, K=H; down: rows=H, K=I)."""
+        """uint8 [rows, K*bits/8] codes of expert ``e`` (gate/up: rows=I, K=H; down: rows=H, K=I)."""
         n = self.per_expert(kind)
         h, i = self.shape.hidden, self.shape.inter
         rows, k = (h, i) if kind == DOWN_Q else (i, h)
-        return code_bytes(self.keys[kind], e * n, n).reshape(rows, k // 2)
+        return code_bytes(self.keys[kind], e * n, n).reshape(rows, k * self.shape.bits // 8)
 
     def expert_scales(self, kind: int, e: int) -> np.ndarray:
         """uint16 fp16 bits [rows, K/group] of expert ``e``."""

@@ -54,7 +54,7 @@ def expert_tensors(shape: LayerShape, seed: int = 0, layer: int = 0, device="cud
     H, I, n = shape.hidden, shape.inter, shape.n_total
     out = {}
     for name, kind, (r, K) in (("gate", GATE_Q, (I, H)), ("up", UP_Q, (I, H)), ("down", DOWN_Q, (H, I))):
-        q = torch.empty((n, r, K // 2), dtype=torch.uint8, device=device)
+        q = torch.empty((n, r, K * shape.bits // 8), dtype=torch.uint8, device=device)
         fill_codes(q, stream_key(seed, layer, kind))
         out[name + "_q"] = q
     for name, kind, (r, K) in (("gate", GATE_S, (I, H)), ("up", UP_S, (I, H)), ("down", DOWN_S, (H, I))):

@@ -37,7 +37,7 @@ def device_layer(shape: synth.LayerShape, seed: int = 0, layer: int = 0):
     rw = torch.from_numpy(li.router_w()).cuda()
     b = li.bias()
     bias = None if b is None else torch.from_numpy(b).cuda()
-    dims = dims_for(shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared, shape.group)
+    dims = dims_for(shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared, shape.group, shape.bits)
     return MoELayer(dims, t, rw, bias)
 
 

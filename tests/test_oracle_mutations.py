@@ -61,6 +61,10 @@ def _scale_per_32_codes(q_bytes, s_bits, group=32):
     return q * s[:, idx]
 
 
+def _int8_unsigned(q_bytes):
+    return np.asarray(q_bytes, dtype=np.uint8).astype(np.int16)
+
+
 def _route_high_index_ties(l32, k):
     l = np.asarray(l32, dtype=np.float32).astype(np.float64)
     T, E = l.shape
@@ -134,6 +138,7 @@ MUTATIONS = {
     "offset-8 codes instead of two's complement": ("unpack_int4", _offset_codes),
     "scale group index transposed": ("dequant", _interleaved_scales),
     "group size ignored (32 codes per scale)": ("dequant", _scale_per_32_codes),
+    "int8 codes read unsigned": ("unpack_int8", _int8_unsigned),
     "ties to the highest index": ("route", _route_high_index_ties),
     "weights not renormalised": ("route", _route_not_renormalised),
     "union not stable": ("batch_union", _union_unstable),

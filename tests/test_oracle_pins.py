@@ -56,6 +56,28 @@ def test_dequant_hand_worked():
         assert W[0, 30] == float(f[2]) and W[0, 31] == float(f[3])
 
 
+def test_unpack_int8_every_byte():
+    """Every byte value decodes to its two's-complement code (Python's own
+    signed conversion, not numpy's)."""
+    b = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    want = [int.from_bytes(bytes([v]), "little", signed=True) for v in range(256)]
+    assert oracle.unpack_int8(b)[0].tolist() == want
+
+
+def test_dequant_int8_hand_worked():
+    for ln in _golden("dequant_int8_hand.txt"):
+        f = [p.strip() for p in ln.split("|")]
+        byte, sb, want = int(f[0], 16), int(f[1], 16), float(f[2])
+        W = oracle.dequant(np.array([[byte] * 32], np.uint8), np.array([[sb]], np.uint16), 32, bits=8)
+        assert W.shape == (1, 32)
+        assert W[0].tolist() == [want] * 32
+
+
+def test_dequant_int8_group_index_and_rows():
+    _check_group_index(32, bits=8)
+    _check_group_index(64, bits=8)
+
+
 def test_dequant_group_index_and_rows():
     _check_group_index(32)
 
@@ -65,17 +87,17 @@ def test_dequant_gs64_group_index_and_rows():
     _check_group_index(64)
 
 
-def _check_group_index(group):
+def _check_group_index(group, bits=4):
     """Scale (r, c // group) multiplies element (r, c): each scale set to a
     power of two tagging its (row, group) is recovered from a code-1 matrix."""
     rows, K = 3, 256
     ng = K // group
-    q = np.full((rows, K // 2), 0x11, np.uint8)            # every code = +1
+    q = np.full((rows, K // 2), 0x11, np.uint8) if bits == 4 else np.full((rows, K), 0x01, np.uint8)  # codes = +1
     s = np.zeros((rows, ng), np.float16)
     for r in range(rows):
         for g in range(ng):
             s[r, g] = 2.0 ** -(r * ng + g)
-    W = oracle.dequant(q, s.view(np.uint16), group)
+    W = oracle.dequant(q, s.view(np.uint16), group, bits)
     for r in range(rows):
         for c in range(K):
             assert W[r, c] == 2.0 ** -(r * ng + c // group)
@@ -267,11 +289,11 @@ def test_silu_matches_library():
     assert oracle.silu(np.array([0.0]))[0] == 0.0
 
 
-def _rand_layer(rng, H, I, E, S, zero_routed=False):
+def _rand_layer(rng, H, I, E, S, zero_routed=False, bits=4):
     n = E + S
     arr = {}
     for kind, (r, K) in {"gate": (I, H), "up": (I, H), "down": (H, I)}.items():
-        c = rng.integers(0, 256, size=(n, r, K // 2), dtype=np.uint8)
+        c = rng.integers(0, 256, size=(n, r, K * bits // 8), dtype=np.uint8)
         if zero_routed:
             c[:E] = 0
         s = rng.uniform(0.005, 0.02, size=(n, r, K // 32)).astype(np.float16).view(np.uint16)
@@ -279,15 +301,20 @@ def _rand_layer(rng, H, I, E, S, zero_routed=False):
     return arr
 
 
-def _py_dequant(codes, scales):
+def _py_dequant(codes, scales, bits=4):
     """Pure-Python dequant from the container definition (independent loops)."""
     rows, kb = codes.shape
-    out = [[0.0] * (2 * kb) for _ in range(rows)]
+    K = kb * 8 // bits
+    out = [[0.0] * K for _ in range(rows)]
     for r in range(rows):
-        for c in range(2 * kb):
-            byte = int(codes[r, c // 2])
-            nib = (byte >> 4) if (c % 2) else (byte & 15)
-            code = nib - 16 if nib > 7 else nib
+        for c in range(K):
+            if bits == 4:
+                byte = int(codes[r, c // 2])
+                nib = (byte >> 4) if (c % 2) else (byte & 15)
+                code = nib - 16 if nib > 7 else nib
+            else:
+                byte = int(codes[r, c])
+                code = byte - 256 if byte > 127 else byte
             out[r][c] = code * float(np.uint16(scales[r, c // 32]).view(np.float16))
     return out
 
@@ -305,14 +332,22 @@ def _py_dense_swiglu(x, Wg, Wu, Wd):
 
 def test_dense_identity_one_expert():
     """E=1, k=1, S=0: the layer equals a dense SwiGLU FFN (Python loops)."""
+    _dense_identity(bits=4)
+
+
+def test_dense_identity_one_expert_int8():
+    _dense_identity(bits=8)
+
+
+def _dense_identity(bits):
     rng = np.random.default_rng(6)
     H, I, T = 64, 32, 3
-    arr = _rand_layer(rng, H, I, 1, 0)
-    W = oracle.ExpertWeights.from_arrays(arr)
+    arr = _rand_layer(rng, H, I, 1, 0, bits=bits)
+    W = oracle.ExpertWeights.from_arrays(arr, bits=bits)
     x_bits = synth.normal_bf16(9, 0, 1, (T, H))
     ids = np.zeros((T, 1), np.int32)
     out, acc = oracle.moe_ffn_combine(W, x_bits, ids, np.ones((T, 1)), 1, 0, return_f64=True)
-    Wg, Wu, Wd = (_py_dequant(*(a[0] for a in arr[k])) for k in ("gate", "up", "down"))
+    Wg, Wu, Wd = (_py_dequant(*(a[0] for a in arr[k]), bits=bits) for k in ("gate", "up", "down"))
     for t in range(T):
         x = oracle.bf16_bits_to_f64(x_bits[t]).tolist()
         ref = _py_dense_swiglu(x, Wg, Wu, Wd)
