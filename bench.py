@@ -62,7 +62,8 @@ def parse():
         a.steps = {"glm52_layer_decode_b1": 2000, "glm52_layer_decode_b64_zipf": 400,
                    "glm52_layer_prefill_4096": 40, "glm52_stack16_decode_b4": 200,
                    "glm52_layer_prefill_512_e32": 50, "glm52_layer_decode_b1_gs64": 2000,
-                   "glm52_layer_prefill_4096_gs64": 40}.get(a.workload, 20)
+                   "glm52_layer_prefill_4096_gs64": 40,
+                   "glm52_layer_int8_decode_b1": 1000}.get(a.workload, 20)
     a.warmup = max(a.warmup, 3)
     return a
 
@@ -179,7 +180,8 @@ def oracle_sample(shape: synth.LayerShape, seconds: float):
             need = sorted(set(ids.ravel().tolist()) | set(range(shape.n_experts, shape.n_total)))
             kinds = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
             pre = {(k, e): (li.expert_codes(q, e), li.expert_scales(s, e)) for k, (q, s) in kinds.items() for e in need}
-            W = oracle.ExpertWeights(lambda k, e: pre[(k, e)][0], lambda k, e: pre[(k, e)][1])
+            W = oracle.ExpertWeights(lambda k, e: pre[(k, e)][0], lambda k, e: pre[(k, e)][1], shape.group,
+                                     bits=shape.bits)
             xin = x
             t0 = time.perf_counter()
             if shape.prenorm:
@@ -259,7 +261,7 @@ def main():
 
     shape = synth.WORKLOADS[a.workload]
     T, H, I, E, k, S = shape.tokens, shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared
-    dims = cm.dims_for(H, I, E, k, S, shape.group)
+    dims = cm.dims_for(H, I, E, k, S, shape.group, shape.bits)
     layers = []
     for l in range(shape.layers):
         li = synth.LayerInputs(shape, 0, l)

@@ -103,13 +103,17 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_PF_SMEM(2, 64)
     COLI_SET_PF_SMEM(1, 64)
 #undef COLI_SET_PF_SMEM
-#define COLI_SET_SK_SMEM(SG, GR)                                                                        \
-  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<SG, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(SkCfg<GR>::SMEM)) == cudaSuccess;
-    COLI_SET_SK_SMEM(true, 32)
-    COLI_SET_SK_SMEM(false, 32)
-    COLI_SET_SK_SMEM(true, 64)
-    COLI_SET_SK_SMEM(false, 64)
+#define COLI_SET_SK_SMEM(SG, GR, B)                                                                        \
+  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<SG, GR, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(SkCfg<GR, B>::SMEM)) == cudaSuccess;
+    COLI_SET_SK_SMEM(true, 32, 4)
+    COLI_SET_SK_SMEM(false, 32, 4)
+    COLI_SET_SK_SMEM(true, 64, 4)
+    COLI_SET_SK_SMEM(false, 64, 4)
+    COLI_SET_SK_SMEM(true, 32, 8)
+    COLI_SET_SK_SMEM(false, 32, 8)
+    COLI_SET_SK_SMEM(true, 64, 8)
+    COLI_SET_SK_SMEM(false, 64, 8)
 #undef COLI_SET_SK_SMEM
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
@@ -164,6 +168,9 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 coli_status check_dims(const coli_moe_dims* d) {
   if (!d) return COLI_ERR_INVALID_ARG;
   if (d->group != 32 && d->group != 64) return COLI_ERR_UNSUPPORTED;
+  if (d->code_bits != 0 && d->code_bits != 4 && d->code_bits != 8) return COLI_ERR_UNSUPPORTED;
+  // int8 codes run in the split-K decode form only: whole 16-byte down scale rows
+  if (d->code_bits == 8 && d->inter % 256 != 0) return COLI_ERR_UNSUPPORTED;
   if (d->hidden <= 0 || d->hidden % 256 != 0) return COLI_ERR_UNSUPPORTED;
   if (d->inter <= 0 || !(d->inter % 256 == 0 || d->inter == 128)) return COLI_ERR_UNSUPPORTED;
   // 64-wide groups: scale rows are read in 16-byte boxes of 8 scales (512 K)
@@ -213,6 +220,8 @@ struct Ws {
 // Split-K form: batches of <= kSkMaxT tokens whose down scale rows are whole
 // 16-byte units (I a multiple of 256; of 512 with 64-wide groups, as always).
 inline bool use_splitk(const coli_moe_dims* d, int T) { return T <= kSkMaxT && d->inter % 256 == 0; }
+
+inline int code_bits(const coli_moe_dims* d) { return d->code_bits == 8 ? 8 : 4; }
 
 Ws layout(const coli_moe_dims* d, int T, void* base) {
   Ws ws{};
@@ -269,19 +278,21 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor maps of one matrix kind: codes [rows_total][K/2] bytes and scales
-// [rows_total][K/group] fp16, tiles of 128 rows x KC elements; the scale box
-// is KC/32 scales (group 32) or 8 scales (group 64, K a multiple of 512).
-bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, int group, CUtensorMap* mq,
-                 CUtensorMap* ms) {
-  // stages of 512 K move their codes as two 128-byte-wide boxes
-  const CUtensorMapSwizzle swz = KC >= 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, rows_total, K / 2, KC >= 256 ? 128 : KC / 2, kRowBlock,
-                 swz))
+// Tensor maps of one matrix kind: codes [rows_total][K*bits/8] bytes and
+// scales [rows_total][K/group] fp16, tiles of 128 rows x KC elements; the
+// scale box is KC/32 scales (int4, group 32) or 8 scales (otherwise; K a
+// multiple of 512 with group 64).
+bool matrix_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, int K, int KC, int group, int bits,
+                 CUtensorMap* mq, CUtensorMap* ms) {
+  // stage rows of 256 bytes move as two 128-byte-wide boxes
+  const int rowb = KC * bits / 8;
+  const CUtensorMapSwizzle swz = rowb >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!encode_2d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, static_cast<uint64_t>(K) * bits / 8, rows_total,
+                 static_cast<uint64_t>(K) * bits / 8, rowb >= 128 ? 128 : rowb, kRowBlock, swz))
     return false;
   if (KC < K) {
     if (!encode_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, K / group, rows_total, (K / group) * 2,
-                   group == 32 ? KC / 32 : 8, kRowBlock, CU_TENSOR_MAP_SWIZZLE_NONE))
+                   (group == 32 && bits == 4) ? KC / 32 : 8, kRowBlock, CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   } else {
     std::memset(ms, 0, sizeof(*ms));  // scales move by 1-D bulk copies when a stage spans K
@@ -384,11 +395,13 @@ bool launch_route_union(const float* lg, const float* bias, int T, int E, int k,
 
 // FFN form for this call: the tcgen05 grouped GEMM when forced, or by default
 // once the batch averages >= 32 tokens per expert of the union's upper bound.
-enum class Form { kDecode, kPrefill, kInvalid };
+enum class Form { kDecode, kPrefill, kInvalid, kUnsupported };
 
-Form choose_form(uint32_t flags, int T, int E, int k) {
+Form choose_form(uint32_t flags, int T, const coli_moe_dims* d) {
+  const int E = d->n_experts, k = d->top_k;
   const bool fd = (flags & COLI_PATH_DECODE) != 0, fp = (flags & COLI_PATH_PREFILL) != 0;
   if (fd && fp) return Form::kInvalid;
+  if (code_bits(d) == 8) return (fp || !use_splitk(d, T)) ? Form::kUnsupported : Form::kDecode;
   if (fd) return Form::kDecode;
   if (fp) return Form::kPrefill;
   const long P = static_cast<long>(T) * k;
@@ -536,11 +549,12 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   CUtensorMap maps[6];   // gate q, up q, gate s, up s, down q, down s
   // down stages: 512 K (two 128-byte code boxes) for the one-n-tile forms,
   // whose activation slice per stage stays small
-  const int G = d->group;
+  const int G = d->group, B = code_bits(d);
   const int kc_dn = (I % 512 == 0 && T <= 8) ? 512 : (I % 256 == 0) ? 256 : 128;
-  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, 256, G, &maps[0], &maps[2]) ||
-      !matrix_maps(w->up_q, w->up_s, rows_gu, H, 256, G, &maps[1], &maps[3]) ||
-      !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, G, &maps[4], &maps[5]))
+  const int kc_gu = B == 4 ? 256 : 128;
+  if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, kc_gu, G, B, &maps[0], &maps[2]) ||
+      !matrix_maps(w->up_q, w->up_s, rows_gu, H, kc_gu, G, B, &maps[1], &maps[3]) ||
+      (B == 4 && !matrix_maps(w->down_q, w->down_s, rows_dn, I, kc_dn, G, B, &maps[4], &maps[5])))
     return COLI_ERR_CUDA;
 
   FfnArgs a{};
@@ -570,19 +584,30 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   a.S = S;
   a.P = P;
   if (use_splitk(d, T)) {
-    // down maps of the split-K form: codes in boxes of 128 rows x 64 bytes
-    // (one 128-wide K slice, 64B swizzle), scales in boxes of 8 x 128 rows
-    if (!encode_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->down_q, I / 2, rows_dn, I / 2, 64, kRowBlock,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+    // down maps of the split-K form: codes in boxes of 128 rows x one
+    // 128-wide K slice (64 bytes, 64B swizzle; int8: 128 bytes, 128B
+    // swizzle), scales in boxes of 8 x 128 rows
+    const uint64_t drow = static_cast<uint64_t>(I) * B / 8;
+    if (!encode_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->down_q, drow, rows_dn, drow, 16 * B, kRowBlock,
+                   B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&maps[5], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->down_s, I / G, rows_dn, (I / G) * 2, 8, kRowBlock,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
       return COLI_ERR_CUDA;
     a.ypart = ws.ypair;
     const long tiles = blocks_ub * (I / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
-    FfnKernel k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32> : ffn_splitk_kernel<true, 64>)
-                         : (G == 32 ? ffn_splitk_kernel<false, 32> : ffn_splitk_kernel<false, 64>);
-    if (!launch_cooperative(k, G == 32 ? SkCfg<32>::SMEM : SkCfg<64>::SMEM, maps, a, grid, st)) return COLI_ERR_CUDA;
+    FfnKernel k;
+    size_t smem;
+    if (B == 4) {
+      k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32, 4> : ffn_splitk_kernel<true, 64, 4>)
+                 : (G == 32 ? ffn_splitk_kernel<false, 32, 4> : ffn_splitk_kernel<false, 64, 4>);
+      smem = G == 32 ? SkCfg<32, 4>::SMEM : SkCfg<64, 4>::SMEM;
+    } else {
+      k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32, 8> : ffn_splitk_kernel<true, 64, 8>)
+                 : (G == 32 ? ffn_splitk_kernel<false, 32, 8> : ffn_splitk_kernel<false, 64, 8>);
+      smem = G == 32 ? SkCfg<32, 8>::SMEM : SkCfg<64, 8>::SMEM;
+    }
+    if (!launch_cooperative(k, smem, maps, a, grid, st)) return COLI_ERR_CUDA;
     rec.mark_through(6, 7);
     rec.mark(8);
     return COLI_OK;
@@ -695,8 +720,9 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
     return COLI_ERR_INVALID_ARG;
   if (x == out) return COLI_ERR_INVALID_ARG;
-  const Form form = choose_form(flags, T, dims->n_experts, dims->top_k);
+  const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
+  if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
   DevInfo di;
@@ -731,8 +757,9 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
     return COLI_ERR_INVALID_ARG;
   if (x == out) return COLI_ERR_INVALID_ARG;
-  const Form form = choose_form(flags, T, dims->n_experts, dims->top_k);
+  const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
+  if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
   DevInfo di;

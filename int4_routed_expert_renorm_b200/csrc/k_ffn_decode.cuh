@@ -69,28 +69,32 @@ struct FfnArgs {
 
 // Shared-memory layout constants.  KC elements of K per stage; NT n-tiles of 8
 // tokens per tile; NMAT matrices per stage (2 = gate+up, 1 = down).
-// GROUP: K elements per fp16 scale (32, or 64 for the gs64 container).  With
-// GROUP 64 a stage's scale rows are always one 16-byte box of 8 scales (512 K),
-// loaded whole by the stage (a 256-K stage uses half of it; the next stage
-// reloads the same box, from L2).
-template <int KC, int NT, int NMAT, int GROUP = 32>
+// GROUP: K elements per fp16 scale (32, or 64 for the gs64 container).  BITS:
+// 4 (int4 codes, two per byte) or 8 (int8 codes).  A stage with fewer than 8
+// scales per row loads them as one 16-byte box of 8 (the smallest aligned TMA
+// box): consecutive stages load the same box (the later ones from L2) and each
+// reads its own part (BOX8).
+template <int KC, int NT, int NMAT, int GROUP = 32, int BITS = 4>
 struct StageCfg {
   static constexpr int TOKB = 8 * NT;
   static constexpr int GPW = KC / 64;                 // groups per warp per stage (two K-halves)
-  static constexpr int ROWB = KC / 2;                 // code bytes per row
-  static constexpr int SUBS = KC >= 512 ? KC / 256 : 1;   // 128-byte-wide code sub-tiles per stage
+  static constexpr int ROWB = KC * BITS / 8;          // code bytes per row
+  static constexpr int SUBS = ROWB >= 256 ? ROWB / 128 : 1;   // 128-byte-wide code sub-tiles per stage
   static constexpr int RSTR = ROWB / SUBS;            // row stride inside a code sub-tile
   static constexpr int SUB_BYTES = kRowBlock * RSTR;
-  static constexpr int SROWB = GROUP == 32 ? KC / 16 : 16;   // scale bytes per row
+  static constexpr int SPS = KC / GROUP;              // scales per row per stage
+  static constexpr int SROWB = (GROUP == 32 && BITS == 4) ? KC / 16 : 16;   // scale bytes per row
+  static constexpr bool BOX8 = SROWB == 16 && SPS < 8;
   static constexpr int CODE_BYTES = kRowBlock * ROWB;
   static constexpr int SC_BYTES = kRowBlock * SROWB;
   static constexpr int W_BYTES = NMAT * (CODE_BYTES + SC_BYTES);
   static constexpr int XROW = KC * 2 + 64;            // padded activation row (bank-conflict free)
   static constexpr int STAGE_USED = W_BYTES + TOKB * XROW;
-  static constexpr bool SWZ = (KC >= 256);
+  static constexpr bool SWZ = (ROWB >= 128);
   static_assert(CODE_BYTES % 1024 == 0 && SC_BYTES % 1024 == 0, "stage regions must stay 1 KiB aligned");
   static_assert(NMAT == 1 || KC <= 256, "wide stages are for the down projection only");
-  static_assert(GROUP == 32 || (GROUP == 64 && KC >= 256), "64-wide groups need stages of 256 K or more");
+  static_assert(GROUP == 32 || (GROUP == 64 && KC >= 128), "64-wide groups need stages of 128 K or more");
+  static_assert(BITS == 4 || (BITS == 8 && KC == 128 && NT == 1), "int8 stages: 128 K, one n-tile");
 };
 
 template <int NT, int KCD, int GROUP = 32>
@@ -124,6 +128,39 @@ __device__ __forceinline__ void dq_word_pair(uint32_t (&p)[8], uint32_t w0, uint
   p[4] = dq_pair(w1, 0); p[5] = dq_pair(w1, 4); p[6] = dq_pair(w1, 8); p[7] = dq_pair(w1, 12);
 }
 
+// int8 codes: q = 16 * hi + lo with hi the signed high nibble and lo the
+// unsigned low nibble.  One word of 4 codes gives two bf16x2 pairs of each:
+// (w >> sh) & 0x000F000F puts one nibble in each 16-bit half; under the
+// exponent of 2048 (0x4500) the nibble n ^ 8 is worth 16 * (n ^ 8), and
+// subtracting 2048 + 128 leaves 16 * hi exactly; under 128 (0x4300) the plain
+// nibble is worth n, and subtracting 128 leaves lo.
+__device__ __forceinline__ uint32_t dq_hi16(uint32_t w, int sh) {
+  uint32_t r, q;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(w >> sh), "r"(0x000F000Fu), "r"(0x45084508u));
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(r), "r"(0x45084508u));
+  return q;
+}
+
+__device__ __forceinline__ uint32_t dq_lo(uint32_t w, int sh) {
+  uint32_t r, q;
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(r) : "r"(w >> sh), "r"(0x000F000Fu), "r"(0x43004300u));
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(r), "r"(0x43004300u));
+  return q;
+}
+
+// 8 int8 codes c0..c7 of one row (two words) -> the pairs (c0,c4), (c1,c5),
+// (c2,c6), (c3,c7) of 16 * hi and of lo, the same pairing (and activation
+// fragment order) as the int4 codes of dq_word_pair.
+__device__ __forceinline__ void dq8_row(uint32_t (&hi)[4], uint32_t (&lo)[4], uint2 v) {
+  uint32_t w1, w2;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(w1) : "r"(v.x), "r"(v.y));   // c0 c1 c4 c5
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(w2) : "r"(v.x), "r"(v.y));   // c2 c3 c6 c7
+  hi[0] = dq_hi16(w1, 4);  lo[0] = dq_lo(w1, 0);
+  hi[1] = dq_hi16(w1, 12); lo[1] = dq_lo(w1, 8);
+  hi[2] = dq_hi16(w2, 4);  lo[2] = dq_lo(w2, 0);
+  hi[3] = dq_hi16(w2, 12); lo[3] = dq_lo(w2, 8);
+}
+
 __device__ __forceinline__ void mma_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -148,10 +185,46 @@ __device__ __forceinline__ void group_acc(float (&acc)[4], const uint32_t (&p)[8
   }
 }
 
+// One 32-wide group of int8 codes: rows g (h0, l0) and g + 8 (h1, l1); the
+// 16*hi and lo parts of every code meet the same activation fragment.
+template <bool SINGLE>
+__device__ __forceinline__ void group_acc8(float (&acc)[4], const uint32_t (&h0)[4], const uint32_t (&h1)[4],
+                                           const uint32_t (&l0)[4], const uint32_t (&l1)[4], const uint4& b,
+                                           float s0, float s1) {
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_16816(d, h0[0], h1[0], h0[1], h1[1], b.x, b.y);
+  mma_16816(d, h0[2], h1[2], h0[3], h1[3], b.z, b.w);
+  mma_16816(d, l0[0], l1[0], l0[1], l1[1], b.x, b.y);
+  mma_16816(d, l0[2], l1[2], l0[3], l1[3], b.z, b.w);
+  acc[0] = fmaf(s0, d[0], acc[0]);
+  acc[2] = fmaf(s1, d[2], acc[2]);
+  if (!SINGLE) {
+    acc[1] = fmaf(s0, d[1], acc[1]);
+    acc[3] = fmaf(s1, d[3], acc[3]);
+  }
+}
+
 __device__ __forceinline__ __half2 u32_as_half2(uint32_t v) {
   __half2 h;
   memcpy(&h, &v, 4);
   return h;
+}
+
+// N fp16 scales at p (N = 1, 2, 4, 8; p aligned to 2N bytes) as half2 pairs.
+template <int N>
+__device__ __forceinline__ void load_scales(const uint8_t* p, __half2 (&h)[4]) {
+  if (N == 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    h[0] = u32_as_half2(v.x); h[1] = u32_as_half2(v.y); h[2] = u32_as_half2(v.z); h[3] = u32_as_half2(v.w);
+  } else if (N == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    h[0] = u32_as_half2(v.x); h[1] = u32_as_half2(v.y);
+  } else if (N == 2) {
+    h[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(p));
+  } else {
+    const uint32_t x = *reinterpret_cast<const uint16_t*>(p);
+    h[0] = u32_as_half2(x | (x << 16));
+  }
 }
 
 __device__ __forceinline__ float half2_pick(const __half2& h, int hi) {
@@ -233,13 +306,13 @@ __device__ __forceinline__ bool wait_h_ready(const FfnArgs& a, int tbg, int targ
 // Producer: fills the stages of one tile.  For a down tile the weight copies
 // go out immediately; the h rows wait (bounded) for the tile's token block to
 // be complete in gate/up.  Returns false on a timeout.
-template <int KC, int NT, int NMAT, int NS, int STAGE, int GROUP>
+template <int KC, int NT, int NMAT, int NS, int STAGE, int GROUP, int BITS = 4>
 __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& ti, const CUtensorMap* mq0,
                                              const CUtensorMap* mq1, const CUtensorMap* ms0, const CUtensorMap* ms1,
                                              const uint16_t* s0_1d, const uint16_t* s1_1d, int K, int R, int nrb_gu,
                                              uint8_t* smem, uint64_t* full, uint64_t* empty, int& s, uint32_t& ph,
                                              long& issued, volatile int* abort_flag, int lane) {
-  using C = StageCfg<KC, NT, NMAT, GROUP>;
+  using C = StageCfg<KC, NT, NMAT, GROUP, BITS>;
   const int row0 = ti.e * R + ti.rb * kRowBlock;
   const int nkc = K / KC;
   const uint16_t* bsrc = a.xq;
@@ -294,7 +367,7 @@ __device__ __forceinline__ bool produce_tile(const FfnArgs& a, const TileInfo& t
         if (NMAT == 2)
           bulk_load(sc + C::SC_BYTES, s1_1d + static_cast<size_t>(row0) * (K / GROUP), C::SC_BYTES, &full[s]);
       } else {
-        const int sx = GROUP == 32 ? kc * (KC / 32) : ((kc * (KC / 64)) & ~7);
+        const int sx = C::BOX8 ? ((kc * C::SPS) & ~7) : kc * C::SPS;
         tma_load_2d(sc, ms0, &full[s], sx, row0);
         if (NMAT == 2) tma_load_2d(sc + C::SC_BYTES, ms1, &full[s], sx, row0);
       }
@@ -389,14 +462,14 @@ constexpr int kSkHRow = 128 * 2 + 64;
 // buffer `hbuf` ([token][kSkHRow bytes], fragment order) once every consumer
 // warp has released the previous unit's slice (h_free), and is announced on
 // h_ready; nothing is written to global memory.
-template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP, bool HSMEM = false>
+template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP, bool HSMEM = false, int BITS = 4>
 __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, const TileInfo& ti, int K, int R,
                                              uint8_t* smem, float* red, uint64_t* full, uint64_t* empty,
                                              uint64_t* red_full, uint64_t* red_empty, int& s, uint32_t& ph,
                                              uint32_t& rph, volatile int* abort_flag, int warp, int lane,
                                              uint16_t* hbuf = nullptr, uint64_t* h_free = nullptr,
                                              uint64_t* h_ready = nullptr, uint32_t lu = 0) {
-  using C = StageCfg<KC, NT, NMAT, GROUP>;
+  using C = StageCfg<KC, NT, NMAT, GROUP, BITS>;
   const int rw = warp & (kRowWarps - 1);   // 16-row slice
   const int half = warp / kRowWarps;       // which half of each stage's groups
   const int g = lane >> 2, c = lane & 3;
@@ -405,10 +478,15 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   // 128B swizzle the 16-byte chunk j of row r sits at chunk j ^ (r & 7), and
   // rl0 & 7 == (rl0 + 8) & 7 == g; bits 4..6 of cbase hold g, so chunk j is
   // cbase ^ (j << 4).
-  const uint32_t cbase = rl0 * C::RSTR + (C::SWZ ? (g << 4) : 0) + 4 * c;
-  // this half's first scale: GPW 32-wide sub-groups are GPW scales (GROUP 32)
-  // or GPW / 2 scales (GROUP 64)
-  const uint32_t sbase = rl0 * C::SROWB + half * (GROUP == 32 ? C::GPW * 2 : C::GPW);
+  // int8: thread c's 8 bytes of a group (codes 8c .. 8c+7, the int4 codes'
+  // ownership) are 16-byte chunk 2j + (c >> 1), bytes 8 (c & 1) ..; with the
+  // swizzle that chunk is (2j) ^ (g ^ (c >> 1)).
+  const uint32_t cbase = BITS == 4 ? rl0 * C::RSTR + (C::SWZ ? (g << 4) : 0) + 4 * c
+                                   : rl0 * C::RSTR + ((g ^ (c >> 1)) << 4) + 8 * (c & 1);
+  // this half's scales: SPH fp16 values (its GPW 32-wide sub-groups share
+  // them when GROUP is 64)
+  constexpr int SPH = C::GPW * 32 / GROUP;
+  const uint32_t sbase = rl0 * C::SROWB + half * SPH * 2;
   const uint32_t xbase = C::W_BYTES + g * C::XROW + (half * C::GPW * 32 + 8 * c) * 2;
   const int nnt = (ti.ntok + 7) >> 3;
   const int nkc = K / KC;
@@ -427,77 +505,59 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
     const uint8_t* sc = st + NMAT * C::CODE_BYTES + sbase;
     // this warp's fp16 scales for its GPW groups (rows rl0 and rl0 + 8, both matrices)
     __half2 sh0[4], sh1[4], th0[4], th1[4];
-    if (GROUP == 64) {
-      // the stage's scales start at element (kc * KC / 64) & 7 of the 8-scale box row
-      const uint8_t* sq = sc + ((kc * (KC / 64)) & 7) * 2;
-      if (C::GPW == 8) {   // 4 scales per half
-        const uint2 v0 = *reinterpret_cast<const uint2*>(sq);
-        const uint2 v1 = *reinterpret_cast<const uint2*>(sq + 8 * C::SROWB);
-        sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
-        sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y);
-      } else {             // GPW 4: 2 scales per half
-        sh0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq));
-        sh1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + 8 * C::SROWB));
-        if (NMAT == 2) {
-          th0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + C::SC_BYTES));
-          th1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sq + C::SC_BYTES + 8 * C::SROWB));
-        }
-      }
-    } else if (C::GPW == 8) {
-      const uint4 v0 = *reinterpret_cast<const uint4*>(sc);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(sc + 8 * C::SROWB);
-      sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y); sh0[2] = u32_as_half2(v0.z); sh0[3] = u32_as_half2(v0.w);
-      sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y); sh1[2] = u32_as_half2(v1.z); sh1[3] = u32_as_half2(v1.w);
-    } else if (C::GPW == 4) {
-      const uint2 v0 = *reinterpret_cast<const uint2*>(sc);
-      const uint2 v1 = *reinterpret_cast<const uint2*>(sc + 8 * C::SROWB);
-      sh0[0] = u32_as_half2(v0.x); sh0[1] = u32_as_half2(v0.y);
-      sh1[0] = u32_as_half2(v1.x); sh1[1] = u32_as_half2(v1.y);
+    {
+      const uint8_t* sq = sc + (C::BOX8 ? ((kc * C::SPS) & 7) * 2 : 0);
+      load_scales<SPH>(sq, sh0);
+      load_scales<SPH>(sq + 8 * C::SROWB, sh1);
       if (NMAT == 2) {
-        const uint2 u0 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES);
-        const uint2 u1 = *reinterpret_cast<const uint2*>(sc + C::SC_BYTES + 8 * C::SROWB);
-        th0[0] = u32_as_half2(u0.x); th0[1] = u32_as_half2(u0.y);
-        th1[0] = u32_as_half2(u1.x); th1[1] = u32_as_half2(u1.y);
-      }
-    } else {
-      sh0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc));
-      sh1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + 8 * C::SROWB));
-      sh0[1] = sh0[0];
-      sh1[1] = sh1[0];
-      if (NMAT == 2) {
-        th0[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES));
-        th1[0] = u32_as_half2(*reinterpret_cast<const uint32_t*>(sc + C::SC_BYTES + 8 * C::SROWB));
-        th0[1] = th0[0];
-        th1[1] = th1[0];
+        load_scales<SPH>(sq + C::SC_BYTES, th0);
+        load_scales<SPH>(sq + C::SC_BYTES + 8 * C::SROWB, th1);
       }
     }
 #pragma unroll
     for (int jj = 0; jj < C::GPW; ++jj) {
       const int j = half * C::GPW + jj;                       // group within the stage
-      const int jc = C::SUBS == 1 ? j : (j & 7);              // 16-byte chunk within the sub-tile row
-      const uint8_t* ca = st + (C::SUBS == 1 ? 0 : (j >> 3) * C::SUB_BYTES) + (cbase ^ static_cast<uint32_t>(jc << 4));
-      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
-      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::RSTR);
       const int si = GROUP == 32 ? jj : (jj >> 1);            // this sub-group's scale among the half's
       const float s0 = half2_pick(sh0[si >> 1], si & 1);
       const float s1 = half2_pick(sh1[si >> 1], si & 1);
-      uint32_t pg[8], pu[8];
-      dq_word_pair(pg, w0, w1);
       float t0 = 0.f, t1 = 0.f;
       if (NMAT == 2) {
-        const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
-        const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::RSTR);
         t0 = half2_pick(th0[si >> 1], si & 1);
         t1 = half2_pick(th1[si >> 1], si & 1);
-        dq_word_pair(pu, v0, v1);
       }
+      if (BITS == 4) {
+        const int jc = C::SUBS == 1 ? j : (j & 7);            // 16-byte chunk within the sub-tile row
+        const uint8_t* ca = st + (C::SUBS == 1 ? 0 : (j >> 3) * C::SUB_BYTES) + (cbase ^ static_cast<uint32_t>(jc << 4));
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * C::RSTR);
+        uint32_t pg[8], pu[8];
+        dq_word_pair(pg, w0, w1);
+        if (NMAT == 2) {
+          const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES);
+          const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ca + C::CODE_BYTES + 8 * C::RSTR);
+          dq_word_pair(pu, v0, v1);
+        }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        if (NT == 1 || nt < nnt) {
-          uint4 b = make_uint4(0u, 0u, 0u, 0u);
-          if (nt * 8 + g < ti.ntok) b = *reinterpret_cast<const uint4*>(st + xbase + nt * 8 * C::XROW + jj * 64);
-          group_acc<SINGLE>(acc0[nt], pg, b, s0, s1);
-          if (NMAT == 2) group_acc<SINGLE>(acc1[nt], pu, b, t0, t1);
+        for (int nt = 0; nt < NT; ++nt) {
+          if (NT == 1 || nt < nnt) {
+            uint4 b = make_uint4(0u, 0u, 0u, 0u);
+            if (nt * 8 + g < ti.ntok) b = *reinterpret_cast<const uint4*>(st + xbase + nt * 8 * C::XROW + jj * 64);
+            group_acc<SINGLE>(acc0[nt], pg, b, s0, s1);
+            if (NMAT == 2) group_acc<SINGLE>(acc1[nt], pu, b, t0, t1);
+          }
+        }
+      } else {
+        const uint8_t* ca = st + (cbase ^ static_cast<uint32_t>((2 * j) << 4));
+        uint32_t h0[4], h1[4], l0[4], l1[4];
+        dq8_row(h0, l0, *reinterpret_cast<const uint2*>(ca));
+        dq8_row(h1, l1, *reinterpret_cast<const uint2*>(ca + 8 * C::RSTR));
+        uint4 b = make_uint4(0u, 0u, 0u, 0u);
+        if (g < ti.ntok) b = *reinterpret_cast<const uint4*>(st + xbase + jj * 64);
+        group_acc8<SINGLE>(acc0[0], h0, h1, l0, l1, b, s0, s1);
+        if (NMAT == 2) {
+          dq8_row(h0, l0, *reinterpret_cast<const uint2*>(ca + C::CODE_BYTES));
+          dq8_row(h1, l1, *reinterpret_cast<const uint2*>(ca + C::CODE_BYTES + 8 * C::RSTR));
+          group_acc8<SINGLE>(acc1[0], h0, h1, l0, l1, b, t0, t1);
         }
       }
     }
@@ -536,8 +596,8 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   mbar_arrive(&red_empty[rw]);
   rph ^= 1u;
   // epilogue: d0 (row g, col 2c), d1 (row g, col 2c+1), d2 (row g+8, col 2c), d3 (row g+8, col 2c+1)
-  if (HSMEM) {
-    static_assert(!HSMEM || (NMAT == 2 && NT == 1), "h slices in shared memory are for 8-token gate/up tiles");
+  if constexpr (HSMEM) {
+    static_assert(NMAT == 2 && NT == 1, "h slices in shared memory are for 8-token gate/up tiles");
     if (lu > 0 && !mbar_wait(h_free, (lu - 1) & 1u, abort_flag, a.status)) return false;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -551,42 +611,43 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
     __syncwarp();
     if (lane == 0) mbar_arrive(h_ready);
     return true;
-  }
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    if (nt < nnt) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i = ti.i0 + nt * 8 + 2 * c + (q & 1);
-        if (i < ti.cnt && !(SINGLE && (q & 1))) {
-          const size_t orow = static_cast<size_t>(ti.base + i);
-          const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
-          if (NMAT == 2) {
-            const float gv = acc0[nt][q], uv = acc1[nt][q];
-            const float hv = gv / (1.0f + expf(-gv)) * uv;
-            a.hq[orow * R + frag_pos(r)] = float_to_bf16_bits(hv);
-          } else {
-            a.ypair[orow * R + r] = acc0[nt][q];
+  } else {
+  #pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (nt < nnt) {
+  #pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = ti.i0 + nt * 8 + 2 * c + (q & 1);
+          if (i < ti.cnt && !(SINGLE && (q & 1))) {
+            const size_t orow = static_cast<size_t>(ti.base + i);
+            const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
+            if (NMAT == 2) {
+              const float gv = acc0[nt][q], uv = acc1[nt][q];
+              const float hv = gv / (1.0f + expf(-gv)) * uv;
+              a.hq[orow * R + frag_pos(r)] = float_to_bf16_bits(hv);
+            } else {
+              a.ypair[orow * R + r] = acc0[nt][q];
+            }
           }
         }
       }
     }
-  }
-  // publish: every lane's stores, then one increment per warp
-  __threadfence();
-  __syncwarp();
-  if (NMAT == 2) {
-    if (lane == 0) atomicAdd(a.tb_done + ti.tbg, 1);
-  } else if (a.T <= kFusedCombineMaxT) {
-    int old = 0;
-    if (lane == 0) old = atomicAdd(a.rb_done + ti.rb, 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old + 1 == m.total_blocks * kRowWarps) {   // last warp of this row block
-      __threadfence();
-      warp_combine_rows(a, ti.rb, lane);
+    // publish: every lane's stores, then one increment per warp
+    __threadfence();
+    __syncwarp();
+    if (NMAT == 2) {
+      if (lane == 0) atomicAdd(a.tb_done + ti.tbg, 1);
+    } else if (a.T <= kFusedCombineMaxT) {
+      int old = 0;
+      if (lane == 0) old = atomicAdd(a.rb_done + ti.rb, 1);
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old + 1 == m.total_blocks * kRowWarps) {   // last warp of this row block
+        __threadfence();
+        warp_combine_rows(a, ti.rb, lane);
+      }
     }
+    return true;
   }
-  return true;
 }
 
 // The persistent FFN kernel (gate/up tiles, then down tiles).  Launched

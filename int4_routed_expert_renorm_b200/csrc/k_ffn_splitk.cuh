@@ -16,7 +16,8 @@
 //   * down: stages of 512 output rows x 128 K (four 128-row tensor-map boxes
 //     of 64 code bytes per row, 64B swizzle, and the rows' 8-scale boxes);
 //     warp w owns stage rows [32 w, 32 w + 32) as two 16-row MMA slices and
-//     all 4 groups of the slice, so no K reduction between warps is needed;
+//     all 4 groups of the slice, so no K reduction between warps is needed
+//     (int8 codes: 256-row stages of two 128-byte-wide boxes, 16 rows a warp);
 //     the fp32 result is a partial y per (pair, K slice, row), ypart;
 //   * after its last unit every consumer warp fences its partials and checks in
 //     on a CTA barrier; one thread per CTA then increments a grid counter;
@@ -35,15 +36,26 @@
 namespace coli {
 
 constexpr int kSkMaxT = 8;                       // largest batch this form takes
-constexpr int kSkBoxes = 4;                      // 128-row boxes per down stage
-constexpr int kSkDnCode = kRowBlock * 64;        // codes of one box: 128 rows x 128 K
 constexpr int kSkDnScale = kRowBlock * 16;       // the rows' 16-byte (8-scale) boxes
-constexpr int kSkStageRows = kSkBoxes * kRowBlock;
 
-template <int GROUP>
+// BITS 4: gate/up stages of 256 K; down stages of four 128-row boxes of 64
+// code bytes per row (64B swizzle).  BITS 8: gate/up stages of 128 K (128 code
+// bytes per row); down stages of two 128-row boxes of 128 bytes (128B swizzle).
+template <int BITS>
+struct SkDn {
+  static constexpr int KCG = BITS == 4 ? 256 : 128;      // gate/up stage K
+  static constexpr int BOXES = BITS == 4 ? 4 : 2;         // 128-row boxes per down stage
+  static constexpr int ROWB = 128 * BITS / 8;             // code bytes per row of a 128-wide K slice
+  static constexpr int CODE = kRowBlock * ROWB;           // codes of one box
+  static constexpr int ROWS = BOXES * kRowBlock;          // output rows per down stage
+  static constexpr int WROWS = ROWS / kFfnConsumerWarps;  // rows per consumer warp (32 or 16)
+};
+
+template <int GROUP, int BITS = 4>
 struct SkCfg {
-  using GU = StageCfg<256, 1, 2, GROUP>;
-  static constexpr int DN_USED = kSkBoxes * (kSkDnCode + kSkDnScale);
+  using D = SkDn<BITS>;
+  using GU = StageCfg<D::KCG, 1, 2, GROUP, BITS>;
+  static constexpr int DN_USED = D::BOXES * (D::CODE + kSkDnScale);
   static constexpr int STAGE = ((GU::STAGE_USED > DN_USED ? GU::STAGE_USED : DN_USED) + 1023) / 1024 * 1024;
   static constexpr int RED_BYTES = kRowWarps * 32 * 4 * 2 * 4;   // K-half partials of both matrices
   static constexpr int META_BYTES = (3 * kMaxSeg + 4) * 4;
@@ -56,18 +68,19 @@ struct SkCfg {
   static_assert(NS >= 3, "pipeline depth");
   static_assert(2 * NS + 2 * kRowWarps + 4 <= NBAR, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(kSkDnCode % 1024 == 0, "64B-swizzled boxes need 512-byte alignment");
+  static_assert(D::CODE % 1024 == 0, "swizzled boxes need 1 KiB alignment");
   static_assert(H_BYTES >= kSkMaxT * 32 * 8, "the combine's pair_pos / topk_w copies fit in the h buffer");
 };
 
 // Producer: the down stages of one unit (K slice rb of expert e, every output
 // row).  Returns false on a timeout.
-template <int NS, int STAGE, int GROUP>
+template <int NS, int STAGE, int GROUP, int BITS>
 __device__ __forceinline__ bool produce_down_slice(const FfnArgs& a, const TileInfo& ti, const CUtensorMap* dq,
                                                    const CUtensorMap* ds, uint8_t* smem, uint64_t* full,
                                                    uint64_t* empty, int& s, uint32_t& ph, long& issued,
                                                    volatile int* abort_flag, int lane) {
-  const int nst = (a.H + kSkStageRows - 1) / kSkStageRows;
+  using D = SkDn<BITS>;
+  const int nst = (a.H + D::ROWS - 1) / D::ROWS;
   const int sx = ((ti.rb * kRowBlock) / GROUP) & ~7;   // the slice's first scale, rounded down to its box
   const int rbase = ti.e * a.H;
   for (int st = 0; st < nst; ++st) {
@@ -76,14 +89,14 @@ __device__ __forceinline__ bool produce_down_slice(const FfnArgs& a, const TileI
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) return false;
     if (lane == 0) {
-      const int r0 = st * kSkStageRows;
+      const int r0 = st * D::ROWS;
       const int rem = (a.H - r0) / kRowBlock;
-      const int nb = rem < kSkBoxes ? rem : kSkBoxes;
+      const int nb = rem < D::BOXES ? rem : D::BOXES;
       uint8_t* stg = smem + s * STAGE;
-      mbar_arrive_expect_tx(&full[s], nb * (kSkDnCode + kSkDnScale));
+      mbar_arrive_expect_tx(&full[s], nb * (D::CODE + kSkDnScale));
       for (int b = 0; b < nb; ++b) {
-        tma_load_2d(stg + b * kSkDnCode, dq, &full[s], ti.rb * 64, rbase + r0 + b * kRowBlock);
-        tma_load_2d(stg + kSkBoxes * kSkDnCode + b * kSkDnScale, ds, &full[s], sx, rbase + r0 + b * kRowBlock);
+        tma_load_2d(stg + b * D::CODE, dq, &full[s], ti.rb * D::ROWB, rbase + r0 + b * kRowBlock);
+        tma_load_2d(stg + D::BOXES * D::CODE + b * kSkDnScale, ds, &full[s], sx, rbase + r0 + b * kRowBlock);
       }
     }
     __syncwarp();
@@ -98,7 +111,7 @@ __device__ __forceinline__ bool produce_down_slice(const FfnArgs& a, const TileI
 
 // Consumers: the down stages of one unit, B operand = the unit's h slice in
 // shared memory.  Writes ypart[pair][rb][row].  Returns false on a timeout.
-template <bool SINGLE, int NS, int STAGE, int GROUP>
+template <bool SINGLE, int NS, int STAGE, int GROUP, int BITS>
 __device__ __forceinline__ bool consume_down_slice(const FfnArgs& a, const TileInfo& ti, const uint8_t* smem,
                                                    const uint16_t* hbuf, uint64_t* full, uint64_t* empty,
                                                    uint64_t* h_ready, uint64_t* h_free, int& s, uint32_t& ph,
@@ -112,21 +125,25 @@ __device__ __forceinline__ bool consume_down_slice(const FfnArgs& a, const TileI
     b[j] = g < ti.ntok ? *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(hbuf) + g * kSkHRow +
                                                           (j * 32 + 8 * c) * 2)
                        : make_uint4(0u, 0u, 0u, 0u);
+  using D = SkDn<BITS>;
   const int soff = ((ti.rb * kRowBlock) / GROUP) & 7;   // the slice's first scale within its box
-  const int nst = (a.H + kSkStageRows - 1) / kSkStageRows;
+  const int nst = (a.H + D::ROWS - 1) / D::ROWS;
   for (int st = 0; st < nst; ++st) {
     if (!mbar_wait(&full[s], ph, abort_flag, a.status)) return false;
     const uint8_t* stg = smem + s * STAGE;
-    const int r0 = st * kSkStageRows;
-    if (32 * warp < a.H - r0) {
+    const int r0 = st * D::ROWS;
+    if (D::WROWS * warp < a.H - r0) {
 #pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const int rl = 32 * warp + 16 * sl + g;          // stage-local rows rl and rl + 8
+      for (int sl = 0; sl < D::WROWS / 16; ++sl) {
+        const int rl = D::WROWS * warp + 16 * sl + g;    // stage-local rows rl and rl + 8
         const int bx = rl >> 7, rr = rl & 127;
-        // 64B swizzle: 16-byte chunk j of box row rr sits at chunk j ^ ((rr >> 1) & 3)
-        const uint8_t* cb = stg + bx * kSkDnCode + rr * 64 + 4 * c;
+        // int4, 64B swizzle: 16-byte chunk j of box row rr sits at chunk j ^ ((rr >> 1) & 3);
+        // int8, 128B swizzle: thread c's 8 bytes of group j are chunk (2j + (c >> 1)) ^ (rr & 7)
+        const uint8_t* cb = stg + bx * D::CODE + rr * 64 + 4 * c;   // int4
+        // int8: offset of thread c's word pair of group 0 within the (1 KiB-aligned) box
+        const uint32_t cb8 = rr * 128 + (((rr & 7) ^ (c >> 1)) << 4) + 8 * (c & 1);
         const uint32_t sw = (rr >> 1) & 3;
-        const uint8_t* sp = stg + kSkBoxes * kSkDnCode + bx * kSkDnScale + rr * 16 + soff * 2;
+        const uint8_t* sp = stg + D::BOXES * D::CODE + bx * kSkDnScale + rr * 16 + soff * 2;
         float s0[4], s1[4];
         if (GROUP == 32) {
           const uint2 v0 = *reinterpret_cast<const uint2*>(sp);
@@ -146,12 +163,20 @@ __device__ __forceinline__ bool consume_down_slice(const FfnArgs& a, const TileI
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint8_t* ca = cb + ((static_cast<uint32_t>(j) ^ sw) << 4);
-          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
-          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * 64);
-          uint32_t p[8];
-          dq_word_pair(p, w0, w1);
-          group_acc<SINGLE>(acc, p, b[j], s0[j], s1[j]);
+          if (BITS == 4) {
+            const uint8_t* ca = cb + ((static_cast<uint32_t>(j) ^ sw) << 4);
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ca);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ca + 8 * 64);
+            uint32_t p[8];
+            dq_word_pair(p, w0, w1);
+            group_acc<SINGLE>(acc, p, b[j], s0[j], s1[j]);
+          } else {
+            const uint8_t* ca = stg + bx * D::CODE + (cb8 ^ static_cast<uint32_t>((2 * j) << 4));
+            uint32_t h0[4], h1[4], l0[4], l1[4];
+            dq8_row(h0, l0, *reinterpret_cast<const uint2*>(ca));
+            dq8_row(h1, l1, *reinterpret_cast<const uint2*>(ca + 8 * 128));
+            group_acc8<SINGLE>(acc, h0, h1, l0, l1, b[j], s0[j], s1[j]);
+          }
         }
         // acc: (row rl, token 2c), (rl, 2c+1), (rl+8, 2c), (rl+8, 2c+1)
 #pragma unroll
@@ -306,14 +331,14 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* 
 
 // The split-K FFN kernel.  Cooperative launch (the final grid-wide wait needs
 // every CTA resident); a.rb_done[0] is the zeroed arrival counter.
-template <bool SINGLE, int GROUP>
+template <bool SINGLE, int GROUP, int BITS>
 __global__ void __launch_bounds__(kFfnThreads, 1)
     ffn_splitk_kernel(const __grid_constant__ CUtensorMap gq, const __grid_constant__ CUtensorMap uq,
                       const __grid_constant__ CUtensorMap gs, const __grid_constant__ CUtensorMap us,
                       const __grid_constant__ CUtensorMap dq, const __grid_constant__ CUtensorMap ds,
                       const FfnArgs a) {
-  using F = SkCfg<GROUP>;
-  constexpr int NS = F::NS, STAGE = F::STAGE;
+  using F = SkCfg<GROUP, BITS>;
+  constexpr int NS = F::NS, STAGE = F::STAGE, KCG = F::D::KCG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red = reinterpret_cast<float*>(smem + NS * STAGE);
@@ -385,10 +410,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < m.tiles_gu; t += gridDim.x) {
       const TileInfo ti = decode_tile<8>(a, m, t);
-      ok = produce_tile<256, 1, 2, NS, STAGE, GROUP>(a, ti, &gq, &uq, &gs, &us, a.gate_s, a.up_s, a.H, a.I,
-                                                     m.nrb_gu, smem, full, empty, s, ph, issued, abort_flag, lane);
-      if (ok) ok = produce_down_slice<NS, STAGE, GROUP>(a, ti, &dq, &ds, smem, full, empty, s, ph, issued,
-                                                        abort_flag, lane);
+      ok = produce_tile<KCG, 1, 2, NS, STAGE, GROUP, BITS>(a, ti, &gq, &uq, &gs, &us, a.gate_s, a.up_s, a.H, a.I,
+                                                           m.nrb_gu, smem, full, empty, s, ph, issued, abort_flag,
+                                                           lane);
+      if (ok) ok = produce_down_slice<NS, STAGE, GROUP, BITS>(a, ti, &dq, &ds, smem, full, empty, s, ph, issued,
+                                                              abort_flag, lane);
     }
     if (!ok && lane == 0) {
       // bounded wait (ignoring the abort flag) for the copies still in flight
@@ -408,12 +434,12 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   uint32_t ph = 0, rph = 0, lu = 0;
   for (int t = blockIdx.x; t < m.tiles_gu; t += gridDim.x, ++lu) {
     const TileInfo ti = decode_tile<8>(a, m, t);
-    if (!consume_tile<256, 1, 2, SINGLE, NS, STAGE, GROUP, true>(a, m, ti, a.H, a.I, smem, red, full, empty,
-                                                                 red_full, red_empty, s, ph, rph, abort_flag, warp,
-                                                                 lane, hbuf, h_free, h_ready, lu))
+    if (!consume_tile<KCG, 1, 2, SINGLE, NS, STAGE, GROUP, true, BITS>(a, m, ti, a.H, a.I, smem, red, full, empty,
+                                                                       red_full, red_empty, s, ph, rph, abort_flag,
+                                                                       warp, lane, hbuf, h_free, h_ready, lu))
       return;
-    if (!consume_down_slice<SINGLE, NS, STAGE, GROUP>(a, ti, smem, hbuf, full, empty, h_ready, h_free, s, ph, lu,
-                                                      abort_flag, warp, lane))
+    if (!consume_down_slice<SINGLE, NS, STAGE, GROUP, BITS>(a, ti, smem, hbuf, full, empty, h_ready, h_free, s, ph,
+                                                            lu, abort_flag, warp, lane))
       return;
   }
   // publish: every warp fences its partials and checks in on the CTA barrier;

@@ -46,7 +46,7 @@ def test_version_and_status_strings(colimoe):
 
 
 def _dims(m, **kw):
-    d = dict(hidden=6144, inter=2048, n_experts=256, top_k=8, n_shared=1, group=32)
+    d = dict(hidden=6144, inter=2048, n_experts=256, top_k=8, n_shared=1, group=32, code_bits=4)
     d.update(kw)
     return m.coli_moe_dims(**d)
 
@@ -66,6 +66,10 @@ def test_workspace_bytes(colimoe):
     assert m.coli_moe_workspace_bytes(_dims(m, group=64, hidden=6400), 4) == 0
     assert m.coli_moe_workspace_bytes(_dims(m, group=64, inter=768), 4) == 0
     assert m.coli_moe_workspace_bytes(_dims(m, group=32, hidden=6400, inter=768), 4) > 0
+    # int8 codes (code_bits 8): the split-K decode form needs whole 16-byte down scale rows
+    assert m.coli_moe_workspace_bytes(_dims(m, code_bits=8), 4) == m.coli_moe_workspace_bytes(d, 4)
+    assert m.coli_moe_workspace_bytes(_dims(m, code_bits=8, inter=128), 4) == 0
+    assert m.coli_moe_workspace_bytes(_dims(m, code_bits=5), 4) == 0
     assert m.coli_moe_workspace_bytes(_dims(m, hidden=6000), 4) == 0
     assert m.coli_moe_workspace_bytes(_dims(m, top_k=300), 4) == 0
 
@@ -106,6 +110,8 @@ def test_layer_argument_checks(colimoe):
     assert L(d, w, x, 4, ws, need - 1) == m._lib.COLI_ERR_WORKSPACE
     assert L(_dims(m, group=16), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, group=64, inter=1280), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, code_bits=8), w, x, 9, ws, m.coli_moe_workspace_bytes(d, 9)) == m._lib.COLI_ERR_UNSUPPORTED
+    assert L(_dims(m, code_bits=8), w, x, 4, ws, need, 0x20) == m._lib.COLI_ERR_UNSUPPORTED   # forced prefill
     assert L(_dims(m, inter=384), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, n_shared=9), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(d, _weights(m, misalign=True), x, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG
