@@ -83,16 +83,13 @@ coli_status dev_info(DevInfo* out) {
 #define COLI_SET_SMEM(NT, SG, KCD, GR)                                                                   \
   ok &= cudaFuncSetAttribute(ffn_fused_kernel<NT, SG, KCD, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(FusedCfg<NT, KCD, GR>::SMEM)) == cudaSuccess;
-    COLI_SET_SMEM(1, true, 256, 32)
-    COLI_SET_SMEM(1, false, 256, 32)
-    COLI_SET_SMEM(4, false, 256, 32)
     COLI_SET_SMEM(1, true, 128, 32)
     COLI_SET_SMEM(1, false, 128, 32)
+    COLI_SET_SMEM(2, false, 128, 32)
     COLI_SET_SMEM(4, false, 128, 32)
-    COLI_SET_SMEM(1, true, 512, 32)
-    COLI_SET_SMEM(1, false, 512, 32)
-    COLI_SET_SMEM(1, true, 512, 64)
-    COLI_SET_SMEM(1, false, 512, 64)
+    COLI_SET_SMEM(2, false, 256, 32)
+    COLI_SET_SMEM(4, false, 256, 32)
+    COLI_SET_SMEM(2, false, 256, 64)
     COLI_SET_SMEM(4, false, 256, 64)
 #undef COLI_SET_SMEM
 #define COLI_SET_PF_SMEM(NMAT, GR)                                                                      \
@@ -223,6 +220,13 @@ inline bool use_splitk(const coli_moe_dims* d, int T) { return T <= kSkMaxT && d
 
 inline int code_bits(const coli_moe_dims* d) { return d->code_bits == 8 ? 8 : 4; }
 
+// Tokens per token block of the two-phase decode form: 8 for T <= 8 (I = 128
+// only; other shapes take the split-K form), 16 up to 64 tokens, 32 above.
+// 16-token blocks leave room for a fourth pipeline stage, which outweighs the
+// extra weight reads of experts with more than 16 tokens (decode b64 Zipf:
+// 1.11x instead of 1.03x the union's bytes, 19 % less time).
+inline int tok_block(int T) { return T <= 8 ? 8 : T <= 64 ? 16 : 32; }
+
 Ws layout(const coli_moe_dims* d, int T, void* base) {
   Ws ws{};
   const size_t H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
@@ -253,7 +257,7 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
   }
   ws.plan = static_cast<int32_t*>(take((Umax + S + 3) * 4));
   {
-    const size_t tokb = T <= 8 ? 8 : 32;
+    const size_t tokb = static_cast<size_t>(tok_block(T));
     const size_t blocks_ub = Umax + P / tokb + S * ((static_cast<size_t>(T) + tokb - 1) / tokb);
     ws.tb_done = static_cast<int32_t*>(take(blocks_ub * 4));
     ws.rb_done = static_cast<int32_t*>(take(H / 128 * 4));
@@ -334,16 +338,18 @@ bool launch_ffn_fused(const CUtensorMap* m, const FfnArgs& a, int grid, cudaStre
   return launch_cooperative(ffn_fused_kernel<NT, SG, KCD, GR>, FusedCfg<NT, KCD, GR>::SMEM, m, a, grid, st);
 }
 
-// Decode-form variant for this batch: one token per tile when T == 1, 8-token
-// tiles while T <= 8, else 32-token tiles.
-template <int KCD>
+// Two-phase decode-form variant for this batch: tiles of tok_block(T) tokens
+// (T <= 8 only with I = 128, KCD = 128).
+template <int KCD, int GR>
 bool launch_ffn_for(int T, const CUtensorMap* m, const FfnArgs& a, int grid, cudaStream_t st) {
-  if (T == 1) return launch_ffn_fused<1, true, KCD, 32>(m, a, grid, st);
-  if (T <= 8) return launch_ffn_fused<1, false, KCD, 32>(m, a, grid, st);
-  return launch_ffn_fused<4, false, KCD, 32>(m, a, grid, st);
+  if (tok_block(T) == 8) {
+    if (KCD != 128 || GR != 32) return false;   // other shapes take the split-K form at T <= 8
+    return T == 1 ? launch_ffn_fused<1, true, 128, 32>(m, a, grid, st)
+                  : launch_ffn_fused<1, false, 128, 32>(m, a, grid, st);
+  }
+  if (tok_block(T) == 16) return launch_ffn_fused<2, false, KCD, GR>(m, a, grid, st);
+  return launch_ffn_fused<4, false, KCD, GR>(m, a, grid, st);
 }
-
-inline int tok_block(int T) { return T <= 8 ? 8 : 32; }
 
 bool launch_route(const float* lg, const float* bias, int T, int E, int k, int32_t* ids, float* w, uint32_t* status,
                   cudaStream_t st) {
@@ -550,7 +556,7 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   // down stages: 512 K (two 128-byte code boxes) for the one-n-tile forms,
   // whose activation slice per stage stays small
   const int G = d->group, B = code_bits(d);
-  const int kc_dn = (I % 512 == 0 && T <= 8) ? 512 : (I % 256 == 0) ? 256 : 128;
+  const int kc_dn = (I % 256 == 0) ? 256 : 128;   // two-phase form: T > 8, or I = 128
   const int kc_gu = B == 4 ? 256 : 128;
   if (!matrix_maps(w->gate_q, w->gate_s, rows_gu, H, kc_gu, G, B, &maps[0], &maps[2]) ||
       !matrix_maps(w->up_q, w->up_s, rows_gu, H, kc_gu, G, B, &maps[1], &maps[3]) ||
@@ -616,15 +622,10 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
     const long tiles = blocks_ub * (I / kRowBlock + H / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
     bool ok;
-    if (G == 64)   // I % 512 == 0: 512-K down stages while T <= 8
-      ok = T == 1   ? launch_ffn_fused<1, true, 512, 64>(maps, a, grid, st)
-           : T <= 8 ? launch_ffn_fused<1, false, 512, 64>(maps, a, grid, st)
-                    : launch_ffn_fused<4, false, 256, 64>(maps, a, grid, st);
-    else if (kc_dn == 512)
-      ok = T == 1 ? launch_ffn_fused<1, true, 512, 32>(maps, a, grid, st)
-                  : launch_ffn_fused<1, false, 512, 32>(maps, a, grid, st);
+    if (G == 64)   // I % 512 == 0, T > 8
+      ok = launch_ffn_for<256, 64>(T, maps, a, grid, st);
     else
-      ok = kc_dn == 256 ? launch_ffn_for<256>(T, maps, a, grid, st) : launch_ffn_for<128>(T, maps, a, grid, st);
+      ok = kc_dn == 256 ? launch_ffn_for<256, 32>(T, maps, a, grid, st) : launch_ffn_for<128, 32>(T, maps, a, grid, st);
     if (!ok) return COLI_ERR_CUDA;
   }
   rec.mark_through(6, 7);
