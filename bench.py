@@ -444,6 +444,10 @@ def main():
                 "peak_kind": f"{src} HBM copy"}
 
     roof["traffic"] = TRAFFIC.get((shape.name, form))
+    # the same figure against the nominal spec (8 TB/s HBM3e; 2.25 PFLOP/s dense bf16), for context
+    spec = 8000.0 if roof["unit"] == "GB/s" else 2250.0
+    roof["frac_of_spec"] = roof["achieved"] / spec
+    roof["spec"] = spec
 
     # int4 bytes touched per step (all three matrices of every unique + shared expert)
     exp_bytes = shape.expert_bytes()
