@@ -314,3 +314,19 @@ def test_decode_batch_invariance(lib, glm_layer, T):
         g1 = run_gpu_layer(lib, glm_layer, x[t:t + 1], residual_bits=x[t:t + 1], flags=lib._lib.COLI_LAYER_PRENORM)
         assert np.array_equal(g1["ids"][0], gb["ids"][t])
         assert np.array_equal(g1["out"][0], gb["out"][t]), t
+
+
+def test_two_phase_form_is_batch_invariant(lib):
+    """Batches of 9..64 tokens run 16-token tiles, larger ones 32-token tiles:
+    the tokens a 65-token batch shares with a 64-token and a 9-token batch get
+    the same bits (per-token MMA columns and fixed reduction orders)."""
+    shape = _small_shape(tokens=65, hidden=512, inter=256, n_experts=8, top_k=2, n_shared=1)
+    layer = device_layer(shape, seed=13)
+    x = synth.normal_bf16(13, 5, synth.X_IN, (65, shape.hidden))
+    g65 = run_gpu_layer(lib, layer, x, residual_bits=x)
+    g64 = run_gpu_layer(lib, layer, x[:64], residual_bits=x[:64])
+    g9 = run_gpu_layer(lib, layer, x[:9], residual_bits=x[:9])
+    assert g65["flags"] == g64["flags"] == g9["flags"] == 0
+    assert np.array_equal(g65["ids"][:64], g64["ids"])
+    assert np.array_equal(g65["out"][:64], g64["out"])
+    assert np.array_equal(g65["out"][:9], g9["out"])
