@@ -323,9 +323,11 @@ def test_two_phase_form_is_batch_invariant(lib):
     shape = _small_shape(tokens=65, hidden=512, inter=256, n_experts=8, top_k=2, n_shared=1)
     layer = device_layer(shape, seed=13)
     x = synth.normal_bf16(13, 5, synth.X_IN, (65, shape.hidden))
-    g65 = run_gpu_layer(lib, layer, x, residual_bits=x)
-    g64 = run_gpu_layer(lib, layer, x[:64], residual_bits=x[:64])
-    g9 = run_gpu_layer(lib, layer, x[:9], residual_bits=x[:9])
+    # logits given, so that routing does not depend on which logits kernel the batch size picks
+    lg = np.random.default_rng(13).standard_normal((65, shape.n_experts)).astype(np.float32)
+    g65 = run_gpu_layer(lib, layer, x, logits_in=lg, residual_bits=x)
+    g64 = run_gpu_layer(lib, layer, x[:64], logits_in=lg[:64], residual_bits=x[:64])
+    g9 = run_gpu_layer(lib, layer, x[:9], logits_in=lg[:9], residual_bits=x[:9])
     assert g65["flags"] == g64["flags"] == g9["flags"] == 0
     assert np.array_equal(g65["ids"][:64], g64["ids"])
     assert np.array_equal(g65["out"][:64], g64["out"])
