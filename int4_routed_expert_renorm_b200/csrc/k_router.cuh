@@ -129,40 +129,50 @@ __global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict_
 // prenorm every block normalises its tokens itself (n = bf16(x * r) with
 // r = 1/sqrt(mean(x^2) + 1e-6) summed in the same order as prep_kernel), so
 // the logits see exactly the normalised input the experts see.
-__device__ __forceinline__ float token_rms_scale(const uint16_t* __restrict__ xr, int H, float* red) {
-  float ss = 0.f;
-  for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
-      ss = fmaf(a, a, ss);
-      ss = fmaf(b, b, ss);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
-  return 1.0f / sqrtf(tot / static_cast<float>(H) + kRmsEps);
-}
-
 __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                                                     int T, int E, int H, int prenorm, float* __restrict__ logits,
                                                     uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float red[8];
+  __shared__ float red[8][8];
   __shared__ float rs[64];
   const int e = blockIdx.x;
   if (prenorm) {
-    for (int t = 0; t < T; ++t) {
-      const float r = token_rms_scale(x + static_cast<size_t>(t) * H, H, red);
-      if (threadIdx.x == 0) rs[t] = r;
+    // every token's sum of squares in one pass (T <= 8 with pre-norm), with
+    // prep_kernel's per-thread order, lane reduction and warp order: each
+    // token gets the same bits whatever the batch
+    float ss[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) ss[t] = 0.f;
+    for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (t < T) v[t] = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + i);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (t < T) {
+          const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
+            ss[t] = fmaf(a, a, ss[t]);
+            ss[t] = fmaf(b, b, ss[t]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss[t] += __shfl_xor_sync(0xffffffffu, ss[t], o);
+      if ((threadIdx.x & 31) == 0) red[t][threadIdx.x >> 5] = ss[t];
+    }
+    __syncthreads();
+    if (threadIdx.x < T) {
+      float tot = 0.f;
+      for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[threadIdx.x][w];
+      rs[threadIdx.x] = 1.0f / sqrtf(tot / static_cast<float>(H) + kRmsEps);
     }
     __syncthreads();
   }
