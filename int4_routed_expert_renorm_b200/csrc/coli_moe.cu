@@ -112,6 +112,8 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_SK_SMEM(true, 64, 8)
     COLI_SET_SK_SMEM(false, 64, 8)
 #undef COLI_SET_SK_SMEM
+    ok &= cudaFuncSetAttribute(logits_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+          cudaSuccess;
     ok &= cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kUnionWarps * 1024 * 4) == cudaSuccess;
     ok &= cudaFuncSetAttribute(union_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -219,6 +221,13 @@ struct Ws {
 inline bool use_splitk(const coli_moe_dims* d, int T) { return T <= kSkMaxT && d->inter % 256 == 0; }
 
 inline int code_bits(const coli_moe_dims* d) { return d->code_bits == 8 ? 8 : 4; }
+
+// Tokens per block of logits_tile_kernel: up to 8, their bf16 rows in at most
+// 200 KB of shared memory.
+inline int logits_tokens_per_block(int H) {
+  const int t = static_cast<int>((200 * 1024) / (static_cast<long>(H) * 2));
+  return t < 1 ? 1 : t > 8 ? 8 : t;
+}
 
 // Tokens per token block of the two-phase decode form: 8 for T <= 8 (I = 128
 // only; other shapes take the split-K form), 16 up to 64 tokens, 32 above.
@@ -775,7 +784,7 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   // 1. expert input (fragment order, optional pre-norm) and router logits
   float* lo = logits_out ? logits_out : lay.logits;
   const float* lg = logits_in;
-  const bool fused_front = T <= (prenorm ? 8 : 64);
+  const bool fused_front = T <= 8;
   if (fused_front) {
     const float* wr = logits_in ? nullptr : w->router_w;
     const int grid = logits_in ? T : E;
@@ -788,7 +797,9 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
     rec.mark(1);
     if (!logits_in) {
       const uint16_t* xr = prenorm ? lay.xn : x;
-      if (!launch(logits_kernel, dim3(E, (T + 7) / 8), dim3(256), 0, s, xr, w->router_w, T, E, H, lo))
+      const int tt = logits_tokens_per_block(H);
+      if (!launch(logits_tile_kernel, dim3((E + 7) / 8, (T + tt - 1) / tt), dim3(256),
+                  static_cast<size_t>(tt) * H * 2, s, xr, w->router_w, T, E, H, tt, lo))
         return COLI_ERR_CUDA;
       lg = lo;
     }

@@ -72,58 +72,75 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
   }
 }
 
-// Router logits l[t,e] = sum_h x[t,h] * W_r[e,h] in fp32.
-// Block = 8 warps for one expert e and up to 8 tokens; warp w covers the
-// H/8 slice [w*H/8, (w+1)*H/8) with float4 loads of W_r; partial sums are
-// reduced in a fixed order (lane tree, then warps 0..7), so every token's
-// logit is computed the same way whatever the batch.  H % 256 == 0.
-__global__ void __launch_bounds__(256) logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
-                                                     int T, int E, int H, float* __restrict__ logits) {
+// Router logits l[t,e] = sum_h x[t,h] * W_r[e,h] in fp32, for batches of more
+// than 8 tokens.  Block = 8 warps, 8 experts (one per warp) and up to `tt`
+// tokens whose bf16 rows the block first copies into shared memory (read once
+// per block instead of once per expert).  Lane l of a warp multiplies the
+// elements 4l + 128i .. +3 (i = 0, 1, ...) of its expert's W_r row (float4
+// loads, four in flight) with every token's, in that order, then the lanes
+// are added in a fixed tree: each (token, expert) is summed the same way
+// whatever the batch.  H % 128 == 0; dynamic shared memory tt * H * 2 bytes.
+__global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __restrict__ x,
+                                                          const float* __restrict__ wr, int T, int E, int H, int tt,
+                                                          float* __restrict__ logits) {
+  extern __shared__ uint4 xs_raw[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(xs_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.y * tt;
+  const int nt = min(tt, T - t0);
+  const int e = blockIdx.x * 8 + warp;
+  // the expert's first W_r loads do not depend on the previous kernel
+  const float* wrow = wr + static_cast<size_t>(e < E ? e : 0) * H;
+  float4 wq[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int h = lane * 4 + u * 128;
+    wq[u] = (e < E && h < H) ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   pdl_wait();
   pdl_trigger();
-  const int e = blockIdx.x;
-  const int t0 = blockIdx.y * 8;
-  const int nt = min(8, T - t0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hw = H >> 3;
-  const int h0 = warp * hw, h1 = h0 + hw;
+  const int n16 = nt * H / 8;
+  for (int i = threadIdx.x; i < n16; i += blockDim.x)
+    xs_raw[i] = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0) * H + static_cast<size_t>(i) * 8);
+  __syncthreads();
+  if (e >= E) return;
   float acc[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-  const float* wrow = wr + static_cast<size_t>(e) * H;
-  for (int h = h0 + lane * 4; h < h1; h += 128) {
-    const float4 w = __ldg(reinterpret_cast<const float4*>(wrow + h));
+  for (int h0 = 0; h0 < H; h0 += 512) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (q < nt) {
-        const uint2 xv = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t0 + q) * H + h);
-        float a = acc[q];
-        a = fmaf(__uint_as_float(xv.x << 16), w.x, a);
-        a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w.y, a);
-        a = fmaf(__uint_as_float(xv.y << 16), w.z, a);
-        a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w.w, a);
-        acc[q] = a;
+    for (int u = 0; u < 4; ++u) {
+      const int h = h0 + lane * 4 + u * 128;
+      const float4 w = wq[u];
+      // next round's load of this slot goes out before the arithmetic
+      const int hn = h + 512;
+      wq[u] = hn < H ? __ldg(reinterpret_cast<const float4*>(wrow + hn)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (h < H) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < nt) {
+            const uint2 xv = *reinterpret_cast<const uint2*>(xs + static_cast<size_t>(q) * H + h);
+            float a = acc[q];
+            a = fmaf(__uint_as_float(xv.x << 16), w.x, a);
+            a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w.y, a);
+            a = fmaf(__uint_as_float(xv.y << 16), w.z, a);
+            a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w.w, a);
+            acc[q] = a;
+          }
+        }
       }
     }
   }
-  __shared__ float part[8][8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     float v = acc[q];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) part[warp][q] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < nt) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
-    logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = s;
+    if (lane == 0 && q < nt) logits[static_cast<size_t>(t0 + q) * E + e] = v;
   }
 }
 
-// Small-batch front end (T <= 64): router logits as in logits_kernel, plus
+// Small-batch front end (T <= 8): router logits, plus
 // the fragment-ordered copy of the expert input written by the blocks whose
 // index matches a token (block b writes tokens b, b + gridDim.x, ...).  With
 // prenorm every block normalises its tokens itself (n = bf16(x * r) with
