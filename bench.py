@@ -72,7 +72,7 @@ def parse():
 # of the same kernel build: (workload, FFN form) -> bytes.  The batch-1 capture
 # ran on the 16-expert variant of the layer, which moves the same 9 experts per
 # step (profiles/ffn_splitk_kernel_glm52_layer_decode_b1_e16.md).  The prefill capture ran on the 32-expert, 512-token variant (same tile
-# shapes): there DRAM traffic was 1.062x the algorithmic bytes of the gate/up
+# shapes): there DRAM traffic was 1.063x the algorithmic bytes of the gate/up
 # launch (profiles/ffn_prefill_kernel_glm52_layer_prefill_512_e32.md); the
 # 4096-token figure is that ratio times its own algorithmic bytes (257 experts'
 # gate+up codes and scales, 36,864 gathered rows, h written).
