@@ -93,7 +93,12 @@ typedef enum {
 #define COLI_PATH_PREFILL        0x20u /* force the prefill FFN form (tcgen05 grouped GEMM) */
 /* With neither flag the prefill form is taken when T >= 32 and T*k >= 32*min(E, T*k)
  * (at least 32 tokens per expert on average), else the decode form.  Both flags
- * together return COLI_ERR_INVALID_ARG. */
+ * together return COLI_ERR_INVALID_ARG.  The decode form runs as one kernel
+ * either way: for T <= 8 (and I a multiple of 256) each gate/up tile's CTA
+ * also computes that tile's K slice of the down projection (fixed-order
+ * partial sums; a token's output is the same bits in any batch of up to 8);
+ * otherwise gate/up tiles and then down tiles, in blocks of 16 (T <= 64) or
+ * 32 tokens.  int8 codes (dims.code_bits == 8) take the first only. */
 
 typedef struct {
   int32_t hidden;     /* H */
