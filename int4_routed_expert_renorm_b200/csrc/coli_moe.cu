@@ -562,8 +562,8 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   const long blocks_ub = static_cast<long>(Umax) + P / tokb + static_cast<long>(S) * ((T + tokb - 1) / tokb);
 
   CUtensorMap maps[6];   // gate q, up q, gate s, up s, down q, down s
-  // down stages: 512 K (two 128-byte code boxes) for the one-n-tile forms,
-  // whose activation slice per stage stays small
+  // gate/up stages of 256 K (int8: 128 K); down stages of the two-phase form
+  // 256 K (128 K when I = 128); the split-K form builds its own down maps
   const int G = d->group, B = code_bits(d);
   const int kc_dn = (I % 256 == 0) ? 256 : 128;   // two-phase form: T > 8, or I = 128
   const int kc_gu = B == 4 ? 256 : 128;

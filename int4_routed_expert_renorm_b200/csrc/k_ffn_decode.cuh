@@ -1,4 +1,7 @@
-// Decode form of the int4 expert FFN and the routing-weighted combine.
+// Decode form of the int4 expert FFN and the routing-weighted combine: the
+// two-phase kernel, used for batches of more than 8 tokens (and for I = 128);
+// smaller batches take the split-K kernel of k_ffn_splitk.cuh, which reuses
+// this file's stage configuration, producer and gate/up consumer.
 //
 // The routed experts are int4 (Colibri README, "L'idea": ~19 MB per expert in
 // the int4 container; an expert's three matrices are the gate, up and down
