@@ -316,11 +316,13 @@ def test_decode_batch_invariance(lib, glm_layer, T):
         assert np.array_equal(g1["out"][0], gb["out"][t]), t
 
 
-def test_two_phase_form_is_batch_invariant(lib):
+@pytest.mark.parametrize("inter", [256, 512])
+def test_two_phase_form_is_batch_invariant(lib, inter):
     """Batches of 9..64 tokens run 16-token tiles, larger ones 32-token tiles:
     the tokens a 65-token batch shares with a 64-token and a 9-token batch get
-    the same bits (per-token MMA columns and fixed reduction orders)."""
-    shape = _small_shape(tokens=65, hidden=512, inter=256, n_experts=8, top_k=2, n_shared=1)
+    the same bits (per-token MMA columns and fixed reduction orders), with one
+    and with two 256-wide down K chunks."""
+    shape = _small_shape(tokens=65, hidden=512, inter=inter, n_experts=8, top_k=2, n_shared=1)
     layer = device_layer(shape, seed=13)
     x = synth.normal_bf16(13, 5, synth.X_IN, (65, shape.hidden))
     # logits given, so that routing does not depend on which logits kernel the batch size picks
