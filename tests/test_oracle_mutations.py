@@ -131,6 +131,32 @@ def _round_via_fp32(v):
     return np.asarray(v, np.float64).astype(np.float32).astype(np.float64).round(6)
 
 
+def _round_ties_away(v):
+    v = np.asarray(v, np.float64)
+    out = v.copy()
+    fin = np.isfinite(v) & (v != 0)
+    _, e = np.frexp(v[fin])
+    ulp = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    q = v[fin] / ulp
+    out[fin] = np.sign(q) * np.floor(np.abs(q) + 0.5) * ulp
+    return out
+
+
+def _router_w_transposed(x_bits, router_w):
+    w = np.asarray(router_w, np.float64)
+    l64 = M.bf16_bits_to_f64(x_bits) @ w.reshape(w.shape[1], w.shape[0])
+    return l64, l64.astype(np.float32)
+
+
+def _bias_ignored(l32, bias):
+    return np.asarray(l32, dtype=np.float32).copy()
+
+
+def _route_nan_first(l32, k):
+    l = np.asarray(l32, np.float32)
+    return ORIG["route"](np.where(np.isnan(l), np.float32(np.inf), l), k)
+
+
 ORIG = {n: getattr(M, n) for n in ("route", "batch_union", "moe_ffn_combine")}
 
 MUTATIONS = {
@@ -150,6 +176,10 @@ MUTATIONS = {
     "rms norm without sqrt": ("rms_norm", _rms_no_sqrt),
     "silu replaced by sigmoid": ("silu", _silu_as_sigmoid),
     "bf16 rounding wrong": ("round_bf16", _round_via_fp32),
+    "bf16 ties away from zero": ("round_bf16", _round_ties_away),
+    "router W_r read transposed": ("router_logits", _router_w_transposed),
+    "bias ignored": ("add_bias", _bias_ignored),
+    "NaN ranked first": ("route", _route_nan_first),
 }
 
 
