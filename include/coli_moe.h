@@ -216,6 +216,20 @@ coli_status coli_moe_layer_noalloc(const coli_moe_dims *dims, const coli_moe_wei
  * tokens (0 for unsupported dims). Host only. */
 size_t coli_moe_workspace_bytes(const coli_moe_dims *dims, int T_max);
 
+/* FFN form taken by coli_moe_layer and coli_moe_expert_ffn for these dims, T
+ * and flags (the rule under COLI_PATH_* above).  Host only: launches nothing
+ * and needs no device.
+ *   form  host pointer; out: one of the COLI_FORM_* values below, or 0 when
+ *         T == 0 (the calls are then no-ops whatever the flags)
+ * Returns the status the calls give for the same dims, T and flags before they
+ * look at pointers or the workspace: COLI_ERR_UNSUPPORTED for dims or batches
+ * outside the supported set, COLI_ERR_INVALID_ARG for T < 0, both COLI_PATH_*
+ * flags, dims == NULL or form == NULL. */
+#define COLI_FORM_DECODE_SPLITK   1  /* decode form, T <= 8 and I % 256 == 0: gate/up and down in one pass */
+#define COLI_FORM_DECODE_TWOPHASE 2  /* decode form, other batches: gate/up tiles, then down tiles, then combine */
+#define COLI_FORM_PREFILL         3  /* prefill form: tcgen05 grouped GEMM */
+coli_status coli_moe_ffn_form(const coli_moe_dims *dims, int T, uint32_t flags, int *form);
+
 /* Synchronises `stream`, then reads and clears the calling device's status
  * word.  *flags (host pointer, may be NULL) receives the COLI_FLAG_* bits.
  * Returns COLI_OK when no bit was set, COLI_ERR_NONFINITE when only the

@@ -19,10 +19,11 @@ COLI_OK, COLI_ERR_INVALID_ARG, COLI_ERR_UNSUPPORTED, COLI_ERR_WORKSPACE = 0, 1, 
 COLI_ERR_CUDA, COLI_ERR_NONFINITE, COLI_ERR_DEVICE = 4, 5, 6
 COLI_FLAG_NONFINITE, COLI_FLAG_BAD_ID, COLI_FLAG_TIMEOUT = 0x1, 0x2, 0x4
 COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
+COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
-           "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc")
+           "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form")
 COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -62,6 +63,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_launch_count": (U64, [I]),
         "coli_moe_set_stage_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
         "coli_moe_layer_noalloc": (I, [D, W, P, I, P, P, U32, P, P, P, P, P]),
+        "coli_moe_ffn_form": (I, [D, I, U32, ctypes.POINTER(I)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -102,6 +104,14 @@ def coli_moe_launch_count(reset: bool = False) -> int:
 
 def coli_moe_workspace_bytes(dims: coli_moe_dims, t_max: int) -> int:
     return _lib.coli_moe_workspace_bytes(ctypes.byref(dims), t_max)
+
+
+def coli_moe_ffn_form(dims: coli_moe_dims, T: int, flags: int = 0) -> int:
+    """The COLI_FORM_* value a layer call with these dims, T and flags takes
+    (0 for T == 0); raises ColiError where the call would fail on them."""
+    form = ctypes.c_int(0)
+    _check(_lib.coli_moe_ffn_form(ctypes.byref(dims), T, flags, ctypes.byref(form)), "coli_moe_ffn_form")
+    return form.value
 
 
 def coli_moe_route(logits, bias, topk_ids, topk_w, stream=None):

@@ -687,6 +687,23 @@ size_t coli_moe_workspace_bytes(const coli_moe_dims* dims, int T_max) {
   return layout(dims, T_max, nullptr).bytes;
 }
 
+coli_status coli_moe_ffn_form(const coli_moe_dims* dims, int T, uint32_t flags, int* form) {
+  if (!form) return COLI_ERR_INVALID_ARG;
+  *form = 0;
+  const coli_status st = check_dims(dims);
+  if (st != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  if (T == 0) return COLI_OK;
+  switch (choose_form(flags, T, dims)) {
+    case Form::kInvalid: return COLI_ERR_INVALID_ARG;
+    case Form::kUnsupported: return COLI_ERR_UNSUPPORTED;
+    case Form::kPrefill: *form = COLI_FORM_PREFILL; return COLI_OK;
+    case Form::kDecode: *form = use_splitk(dims, T) ? COLI_FORM_DECODE_SPLITK : COLI_FORM_DECODE_TWOPHASE; return COLI_OK;
+  }
+  return COLI_ERR_INVALID_ARG;
+}
+
 coli_status coli_moe_route(const float* logits, const float* bias, int T, int E, int k, int32_t* topk_ids,
                            float* topk_w, void* stream) {
   if (T < 0 || E < 1 || k < 1) return COLI_ERR_INVALID_ARG;

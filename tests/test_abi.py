@@ -153,3 +153,90 @@ def test_binding_constants_match_the_header(colimoe):
             assert getattr(colimoe._lib, name) == val, name
             found += 1
     assert found >= 7
+
+
+def _form_rule(T, E, k, inter=2048, code_bits=4, flags=0):
+    """The dispatch rule as include/coli_moe.h states it (COLI_PATH_* and
+    COLI_FORM_* comments)."""
+    fd, fp = bool(flags & 0x10), bool(flags & 0x20)
+    if T == 0:
+        return 0          # a no-op call, whatever the flags
+    if fd and fp:
+        return "invalid"
+    splitk = T <= 8 and inter % 256 == 0
+    if code_bits == 8:
+        return 1 if (splitk and not fp) else "unsupported"
+    P = T * k
+    prefill = fp or (not fd and T >= 32 and P >= 32 * min(E, P))
+    return 3 if prefill else (1 if splitk else 2)
+
+
+def test_ffn_form_follows_the_documented_rule(colimoe):
+    m = colimoe
+    errs = {m._lib.COLI_ERR_INVALID_ARG: "invalid", m._lib.COLI_ERR_UNSUPPORTED: "unsupported"}
+
+    def form(T, flags=0, **kw):
+        try:
+            return m.coli_moe_ffn_form(_dims(m, **kw), T, flags)
+        except m._lib.ColiError as e:
+            return errs[e.status]
+
+    for E, k in ((8, 1), (16, 2), (64, 8), (256, 8)):
+        for T in list(range(0, 70)) + [255, 256, 257, 511, 512, 1023, 1024, 1025, 4096]:
+            for flags in (0, 0x10, 0x20, 0x30):
+                assert form(T, flags, n_experts=E, top_k=k) == _form_rule(T, E, k, flags=flags), (E, k, T, flags)
+    for T in (1, 4, 8, 9, 64):
+        for flags in (0, 0x10, 0x20):
+            assert form(T, flags, inter=128) == _form_rule(T, 256, 8, inter=128, flags=flags)
+            assert form(T, flags, code_bits=8) == _form_rule(T, 256, 8, code_bits=8, flags=flags)
+    # the named cases: batch 1 splits K, batch 64 runs two phases, prefill 4096 takes tcgen05
+    assert (form(1), form(64), form(4096)) == (m._lib.COLI_FORM_DECODE_SPLITK, m._lib.COLI_FORM_DECODE_TWOPHASE,
+                                               m._lib.COLI_FORM_PREFILL)
+    assert form(-1) == "invalid" and form(4, group=16) == "unsupported" and form(1 << 22) == "unsupported"
+    lib, out = m._lib._lib, ctypes.c_int(7)
+    assert lib.coli_moe_ffn_form(None, 4, 0, ctypes.byref(out)) == m._lib.COLI_ERR_INVALID_ARG and out.value == 0
+    assert lib.coli_moe_ffn_form(ctypes.byref(_dims(m)), 4, 0, None) == m._lib.COLI_ERR_INVALID_ARG
+
+
+def test_bench_form_helpers_match_the_library(colimoe):
+    """bench.py picks each workload's roofline by the form it expects the
+    library to take: the library agrees for every workload."""
+    import bench
+    import synth
+    m = colimoe
+    for shape in synth.WORKLOADS.values():
+        d = m.dims_for(shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared, shape.group,
+                       shape.bits)
+        f = m.coli_moe_ffn_form(d, shape.tokens)
+        assert bench.splitk_form(shape) == (f == m._lib.COLI_FORM_DECODE_SPLITK), shape.name
+        assert bench.prefill_form(shape) == (f == m._lib.COLI_FORM_PREFILL), shape.name
+
+
+def _kw_cases(fn):
+    return next(list(mk.args[1]) for mk in fn.pytestmark if mk.name == "parametrize" and mk.args[0] == "kw")
+
+
+def test_gpu_tests_exercise_the_form_they_name(colimoe):
+    """The split-K and int8 parity cases take the split-K decode form and the
+    two-phase invariance cases the two-phase form (read from the tests' own
+    parametrisations, so a later edit cannot silently move them)."""
+    import tests.test_gpu_int8 as i8
+    import tests.test_gpu_splitk as sk
+    from tests.test_gpu_parity import _small_shape
+    m = colimoe
+
+    def form(shape, flags=0):
+        d = m.dims_for(shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.n_shared, shape.group,
+                       shape.bits)
+        return m.coli_moe_ffn_form(d, shape.tokens, flags)
+
+    for kw in _kw_cases(sk.test_splitk_small_shapes):
+        assert form(_small_shape(**kw)) == m._lib.COLI_FORM_DECODE_SPLITK, kw
+    for kw in _kw_cases(i8.test_int8_small_shapes):
+        assert form(_small_shape(bits=8, **kw)) == m._lib.COLI_FORM_DECODE_SPLITK, kw
+    for inter in (256, 512):
+        for T in (9, 64, 65):
+            shape = _small_shape(tokens=T, hidden=512, inter=inter, n_experts=8, top_k=2, n_shared=1)
+            assert form(shape) == m._lib.COLI_FORM_DECODE_TWOPHASE, (inter, T)
+    with pytest.raises(m._lib.ColiError):
+        form(_small_shape(bits=8, tokens=9, inter=256))
