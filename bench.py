@@ -63,7 +63,7 @@ def parse():
                    "glm52_layer_prefill_4096": 40, "glm52_stack16_decode_b4": 200,
                    "glm52_layer_prefill_512_e32": 50, "glm52_layer_decode_b1_gs64": 2000,
                    "glm52_layer_prefill_4096_gs64": 40,
-                   "glm52_layer_int8_decode_b1": 1000}.get(a.workload, 20)
+                   "glm52_layer_int8_decode_b1": 1000, "glm52_layer_prefill_4096_router": 40}.get(a.workload, 20)
     a.warmup = max(a.warmup, 3)
     return a
 
@@ -81,6 +81,9 @@ TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.724544e6 + 3.525376e6,
            ("glm52_layer_decode_b1_e16", "decode"): 191.724544e6 + 3.525376e6,
            ("glm52_layer_prefill_512_e32", "prefill"): 532.542208e6 + 16.592384e6,
            ("glm52_layer_prefill_4096", "prefill"):
+               _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2),
+           # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
+           ("glm52_layer_prefill_4096_router", "prefill"):
                _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)}
 
 

@@ -181,8 +181,12 @@ PREFILL_4096_GS64 = LayerShape("glm52_layer_prefill_4096_gs64", 6144, 2048, 256,
 # head, whose drafts are decoded in batches of 1..4): 37,748,736 + 2,359,296
 # bytes per expert.
 DECODE_B1_INT8 = LayerShape("glm52_layer_int8_decode_b1", 6144, 2048, 256, 8, 1, 1, bits=8)
+# The prefill layer with the router logits computed in the step (x . W_r^T for
+# 4096 tokens: 12.9 GFLOP in fp32) instead of given.
+PREFILL_4096_ROUTER = LayerShape("glm52_layer_prefill_4096_router", 6144, 2048, 256, 8, 1, 4096)
 WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16,
-                                 PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64, DECODE_B1_INT8)}
+                                 PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64, DECODE_B1_INT8,
+                                 PREFILL_4096_ROUTER)}
 
 
 class LayerInputs:
