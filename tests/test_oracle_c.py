@@ -8,6 +8,8 @@ independent means.  Both sides first pass the same pins: the hand-worked
 fixtures under ``tests/golden``, brute-force top-k and union, library
 conversions, and the dense SwiGLU identity.  CPU only (needs gcc).
 """
+import itertools
+
 import numpy as np
 import pytest
 import scipy.special
@@ -344,3 +346,30 @@ def test_layer_rejects_bad_arguments():
         cr.moe_layer(arr, x, 2, 3, 1, logits_in=np.zeros((2, 2), np.float32))     # k > E
     with pytest.raises(ValueError):
         cr.moe_layer(arr, x, 2, 1, 1)                                               # no logits, no router
+
+
+def _brute_topk_fast(l, k):
+    """All k-subsets S of range(E); keep those whose weakest member beats the
+    strongest non-member under (value descending, index ascending)."""
+    E = len(l)
+    rank = lambda e: (-l[e], e)  # noqa: E731  smaller is stronger
+    found = []
+    for S in itertools.combinations(range(E), k):
+        inside = set(S)
+        weakest = max(S, key=rank)
+        if all(rank(weakest) < rank(j) for j in range(E) if j not in inside):
+            found.append(set(S))
+    assert len(found) == 1
+    return found[0]
+
+
+def test_route_matches_brute_force_up_to_16_experts_both_oracles():
+    rng = np.random.default_rng(31)
+    for _ in range(40):
+        E = int(rng.integers(9, 17))
+        k = int(rng.integers(1, 9))
+        l = rng.integers(0, 4, size=(1, E)).astype(np.float32)
+        want = _brute_topk_fast(l[0].tolist(), k)
+        for ids in (cr.route(l, k)[0], oracle.route(l, k)[0]):
+            assert set(ids[0].tolist()) == want
+            assert [(-l[0, e], e) for e in ids[0]] == sorted((-l[0, e], e) for e in ids[0])
