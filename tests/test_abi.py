@@ -240,3 +240,27 @@ def test_gpu_tests_exercise_the_form_they_name(colimoe):
             assert form(shape) == m._lib.COLI_FORM_DECODE_TWOPHASE, (inter, T)
     with pytest.raises(m._lib.ColiError):
         form(_small_shape(bits=8, tokens=9, inter=256))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_layer_holder_checks_tensor_sizes(colimoe, bits):
+    """MoELayer accepts tensors sized for its dims (int4 or int8 codes) and
+    rejects a wrong size before any call; CPU tensors stand in for device ones."""
+    import torch
+    m = colimoe
+    H, I, E, S, G = 256, 256, 4, 1, 64
+    d = m.dims_for(H, I, E, 2, S, G, bits)
+    n = E + S
+    t = {"gate_q": torch.zeros(n, I, H * bits // 8, dtype=torch.uint8),
+         "up_q": torch.zeros(n, I, H * bits // 8, dtype=torch.uint8),
+         "down_q": torch.zeros(n, H, I * bits // 8, dtype=torch.uint8),
+         "gate_s": torch.zeros(n, I, H // G, dtype=torch.int16), "up_s": torch.zeros(n, I, H // G, dtype=torch.int16),
+         "down_s": torch.zeros(n, H, I // G, dtype=torch.int16)}
+    layer = m.MoELayer(d, t)
+    assert layer.weights.gate_q == t["gate_q"].data_ptr() and layer.weights.down_s == t["down_s"].data_ptr()
+    assert layer.weights.router_w is None
+    for name in t:
+        bad = dict(t)
+        bad[name] = t[name][:, :-1]
+        with pytest.raises(ValueError, match=name):
+            m.MoELayer(d, bad)
