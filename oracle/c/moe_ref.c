@@ -295,11 +295,18 @@ int coli_ref_union(int P, int E, const int32_t *flat, int32_t *unique, int32_t *
  * expert SwiGLU FFN, combine, the layer
  * ------------------------------------------------------------------------ */
 
+/* One pointer per expert and matrix: codes [I][H*bits/8] (gate, up) and
+ * [H][I*bits/8] (down), scales [I][H/group] and [H][I/group]. */
 typedef struct {
     int H, I, group, bits;
-    const uint8_t *gate_q, *up_q, *down_q;   /* [n_experts][I][H*bits/8], [..][I][..], [..][H][I*bits/8] */
-    const uint16_t *gate_s, *up_s, *down_s;  /* [n_experts][I][H/group], [..][I][..], [..][H][I/group] */
+    const uint8_t *const *gate_q, *const *up_q, *const *down_q;
+    const uint16_t *const *gate_s, *const *up_s, *const *down_s;
 } Experts;
+
+static int expert_present(const Experts *X, int e)
+{
+    return X->gate_q[e] && X->up_q[e] && X->down_q[e] && X->gate_s[e] && X->up_s[e] && X->down_s[e];
+}
 
 static double silu(double g) { return g / (1.0 + exp(-g)); }
 
@@ -309,10 +316,8 @@ static double silu(double g) { return g / (1.0 + exp(-g)); }
 static void expert_ffn(const Experts *X, int e, const double *x, double *hbuf, double *y)
 {
     const int H = X->H, I = X->I, G = X->group, B = X->bits;
-    const size_t gu_codes = (size_t)I * H * B / 8, gu_scales = (size_t)I * (H / G);
-    const size_t dn_codes = (size_t)H * I * B / 8, dn_scales = (size_t)H * (I / G);
-    const uint8_t *gq = X->gate_q + e * gu_codes, *uq = X->up_q + e * gu_codes, *dq = X->down_q + e * dn_codes;
-    const uint16_t *gs = X->gate_s + e * gu_scales, *us = X->up_s + e * gu_scales, *ds = X->down_s + e * dn_scales;
+    const uint8_t *gq = X->gate_q[e], *uq = X->up_q[e], *dq = X->down_q[e];
+    const uint16_t *gs = X->gate_s[e], *us = X->up_s[e], *ds = X->down_s[e];
     for (int i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
@@ -337,17 +342,16 @@ static void expert_ffn(const Experts *X, int e, const double *x, double *hbuf, d
  * experts (ids E..E+S-1) run on every token with weight 1, outside the
  * renormalisation.  Inputs: x bf16 [T][H]; router_w fp32 [E][H] or NULL when
  * logits_in fp32 [T][E] is given; bias fp32 [E] or NULL; residual bf16 [T][H]
- * or NULL; expert arrays with a leading axis of E+S.  Outputs (caller-owned):
- * l64 [T][E] (NULL allowed), l32 [T][E], ids [T][k], w [T][k], flags [T],
- * acc [T][H] (NULL allowed), out bf16 bits [T][H]. */
-int coli_ref_moe_layer(int T, int H, int I, int E, int k, int S, int group, int bits,
-                       const uint8_t *gate_q, const uint16_t *gate_s, const uint8_t *up_q, const uint16_t *up_s,
-                       const uint8_t *down_q, const uint16_t *down_s, const uint16_t *x, const float *router_w,
-                       const float *logits_in, const float *bias, const uint16_t *residual, double *l64,
-                       float *l32, int32_t *ids, double *w, int32_t *flags, double *acc_out, uint16_t *out)
+ * or NULL.  Outputs (caller-owned): l64 [T][E] (NULL allowed), l32 [T][E],
+ * ids [T][k], w [T][k], flags [T], acc [T][H] (NULL allowed), out bf16 bits
+ * [T][H]. */
+static int moe_layer(int T, int E, int k, int S, const Experts *X, const uint16_t *x, const float *router_w,
+                     const float *logits_in, const float *bias, const uint16_t *residual, double *l64, float *l32,
+                     int32_t *ids, double *w, int32_t *flags, double *acc_out, uint16_t *out)
 {
-    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || S < 0 || !container_ok(H, group, bits) ||
-        !container_ok(I, group, bits) || (!router_w && !logits_in))
+    const int H = X->H, I = X->I;
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || S < 0 || !container_ok(H, X->group, X->bits) ||
+        !container_ok(I, X->group, X->bits) || (!router_w && !logits_in))
         return COLI_REF_EARG;
     int rc;
     if (logits_in) {
@@ -373,14 +377,20 @@ int coli_ref_moe_layer(int T, int H, int I, int E, int k, int S, int group, int 
     int32_t U = 0;
     if ((rc = coli_ref_union(P, E, ids, unique, &U, seg, perm, pos)) != 0)
         goto done;
+    rc = COLI_REF_EARG;                         /* an expert the layer reads was not given */
+    for (int u = 0; u < U; ++u)
+        if (!expert_present(X, unique[u]))
+            goto done;
+    for (int s = 0; s < S && T > 0; ++s)
+        if (!expert_present(X, E + s))
+            goto done;
 
-    const Experts X = {H, I, group, bits, gate_q, up_q, down_q, gate_s, up_s, down_s};
     for (int u = 0; u < U; ++u)
         for (int at = seg[u]; at < seg[u + 1]; ++at) {
             int t = perm[at] / k, j = perm[at] % k;
             for (int c = 0; c < H; ++c)
                 xt[c] = bf16_value(x[(size_t)t * H + c]);
-            expert_ffn(&X, unique[u], xt, hb, y);
+            expert_ffn(X, unique[u], xt, hb, y);
             for (int c = 0; c < H; ++c)
                 acc[(size_t)t * H + c] += w[(size_t)t * k + j] * y[c];
         }
@@ -388,7 +398,7 @@ int coli_ref_moe_layer(int T, int H, int I, int E, int k, int S, int group, int 
         for (int c = 0; c < H; ++c)
             xt[c] = bf16_value(x[(size_t)t * H + c]);
         for (int s = 0; s < S; ++s) {
-            expert_ffn(&X, E + s, xt, hb, y);
+            expert_ffn(X, E + s, xt, hb, y);
             for (int c = 0; c < H; ++c)
                 acc[(size_t)t * H + c] += y[c];
         }
@@ -413,6 +423,57 @@ done:
     free(hb);
     free(y);
     return rc;
+}
+
+/* The layer with every expert's matrices in contiguous arrays with a leading
+ * axis of E+S: gate_q/up_q [E+S][I][H*bits/8], down_q [E+S][H][I*bits/8],
+ * gate_s/up_s [E+S][I][H/group], down_s [E+S][H][I/group]. */
+int coli_ref_moe_layer(int T, int H, int I, int E, int k, int S, int group, int bits,
+                       const uint8_t *gate_q, const uint16_t *gate_s, const uint8_t *up_q, const uint16_t *up_s,
+                       const uint8_t *down_q, const uint16_t *down_s, const uint16_t *x, const float *router_w,
+                       const float *logits_in, const float *bias, const uint16_t *residual, double *l64,
+                       float *l32, int32_t *ids, double *w, int32_t *flags, double *acc_out, uint16_t *out)
+{
+    if (E <= 0 || S < 0 || !container_ok(H, group, bits) || !container_ok(I, group, bits))
+        return COLI_REF_EARG;
+    const int n = E + S;
+    const size_t gu_codes = (size_t)I * H * bits / 8, gu_scales = (size_t)I * (H / group);
+    const size_t dn_codes = (size_t)H * I * bits / 8, dn_scales = (size_t)H * (I / group);
+    const uint8_t **q = malloc(sizeof(*q) * 3 * (size_t)n);
+    const uint16_t **sc = malloc(sizeof(*sc) * 3 * (size_t)n);
+    if (!q || !sc) {
+        free(q);
+        free(sc);
+        return COLI_REF_ENOMEM;
+    }
+    for (int e = 0; e < n; ++e) {
+        q[e] = gate_q + e * gu_codes;
+        q[n + e] = up_q + e * gu_codes;
+        q[2 * n + e] = down_q + e * dn_codes;
+        sc[e] = gate_s + e * gu_scales;
+        sc[n + e] = up_s + e * gu_scales;
+        sc[2 * n + e] = down_s + e * dn_scales;
+    }
+    const Experts X = {H, I, group, bits, q, q + n, q + 2 * n, sc, sc + n, sc + 2 * n};
+    int rc = moe_layer(T, E, k, S, &X, x, router_w, logits_in, bias, residual, l64, l32, ids, w, flags, acc_out, out);
+    free(q);
+    free(sc);
+    return rc;
+}
+
+/* The layer with one pointer per expert and matrix (arrays of E+S pointers);
+ * an expert the batch does not select may be NULL.  A NULL expert that the
+ * layer would read gives COLI_REF_EARG. */
+int coli_ref_moe_layer_experts(int T, int H, int I, int E, int k, int S, int group, int bits,
+                               const uint8_t *const *gate_q, const uint16_t *const *gate_s,
+                               const uint8_t *const *up_q, const uint16_t *const *up_s,
+                               const uint8_t *const *down_q, const uint16_t *const *down_s, const uint16_t *x,
+                               const float *router_w, const float *logits_in, const float *bias,
+                               const uint16_t *residual, double *l64, float *l32, int32_t *ids, double *w,
+                               int32_t *flags, double *acc_out, uint16_t *out)
+{
+    const Experts X = {H, I, group, bits, gate_q, up_q, down_q, gate_s, up_s, down_s};
+    return moe_layer(T, E, k, S, &X, x, router_w, logits_in, bias, residual, l64, l32, ids, w, flags, acc_out, out);
 }
 
 /* n = bf16( h / sqrt(mean(h^2) + 1e-6) ) per token, double inside.

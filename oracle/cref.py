@@ -169,5 +169,41 @@ def moe_layer(arrays: dict, x_bits, n_experts: int, top_k: int, n_shared: int, g
     return r
 
 
+def moe_layer_experts(fetch, hidden: int, inter: int, x_bits, n_experts: int, top_k: int, n_shared: int,
+                      group: int = 32, bits: int = 4, router_w=None, bias=None, logits_in=None,
+                      residual_bits=None, experts=None) -> dict:
+    """The layer with experts fetched on demand: ``fetch(kind, e)`` returns
+    (codes, scales) of expert e for kind 'gate', 'up' or 'down'.  The batch is
+    routed first (the C oracle's logits and Route) to learn which routed
+    experts it selects; only those and the shared experts are fetched, or the
+    ids in ``experts`` when given (the call fails if one it needs is missing).
+    Returns what ``moe_layer`` returns."""
+    x = _arr(x_bits, np.uint16)
+    T = x.shape[0]
+    E, k, n = n_experts, top_k, n_experts + n_shared
+    li = None if logits_in is None else _arr(logits_in, np.float32)
+    l32 = li if li is not None else router_logits(x, router_w)[1]
+    ids = route(l32, k, bias)[0]
+    need = sorted(set(ids.ravel().tolist()) | set(range(E, n))) if experts is None else sorted(experts)
+    held = {(kind, e): tuple(_arr(a, t) for a, t in zip(fetch(kind, e), (np.uint8, np.uint16)))
+            for kind in ("gate", "up", "down") for e in need}
+    ptrs = {}
+    for kind in ("gate", "up", "down"):
+        q, sc = (C.c_void_p * n)(), (C.c_void_p * n)()
+        for e in need:
+            q[e], sc[e] = held[(kind, e)][0].ctypes.data, held[(kind, e)][1].ctypes.data
+        ptrs[kind] = (q, sc)
+    rw = None if router_w is None else _arr(router_w, np.float32)
+    b = None if bias is None else _arr(bias, np.float32)
+    res = None if residual_bits is None else _arr(residual_bits, np.uint16)
+    r = dict(logits64=np.empty((T, E)), logits32=np.empty((T, E), np.float32), ids=np.empty((T, k), np.int32),
+             w=np.empty((T, k)), flags=np.empty(T, np.int32), acc=np.empty((T, hidden)),
+             out=np.empty((T, hidden), np.uint16))
+    _call("coli_ref_moe_layer_experts", T, hidden, inter, E, k, n_shared, group, bits, *ptrs["gate"], *ptrs["up"],
+          *ptrs["down"], _p(x), _p(rw), _p(li), _p(b), _p(res), _p(r["logits64"]), _p(r["logits32"]),
+          _p(r["ids"]), _p(r["w"]), _p(r["flags"]), _p(r["acc"]), _p(r["out"]))
+    return r
+
+
 if __name__ == "__main__":
     print("built", build(force=True))

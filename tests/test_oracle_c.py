@@ -373,3 +373,43 @@ def test_route_matches_brute_force_up_to_16_experts_both_oracles():
         for ids in (cr.route(l, k)[0], oracle.route(l, k)[0]):
             assert set(ids[0].tolist()) == want
             assert [(-l[0, e], e) for e in ids[0]] == sorted((-l[0, e], e) for e in ids[0])
+
+
+@pytest.mark.slow
+def test_c_oracle_agrees_with_numpy_oracle_at_glm_size():
+    """One token of the GLM-shaped layer (H 6144, I 2048, 256 experts, k 8, one
+    shared expert) with the Zipf bias and a residual: the C oracle fetches only
+    the experts the token selects."""
+    shape = synth.DECODE_B64
+    li = synth.LayerInputs(shape)
+    kinds = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
+    x = synth.activations(shape)[:1]
+    rw, bias = li.router_w(), li.bias()
+    assert bias is not None
+    rc = cr.moe_layer_experts(lambda kind, e: (li.expert_codes(kinds[kind][0], e), li.expert_scales(kinds[kind][1], e)),
+                              shape.hidden, shape.inter, x, shape.n_experts, shape.top_k, shape.n_shared, shape.group,
+                              shape.bits, router_w=rw, bias=bias, residual_bits=x)
+    W = oracle.ExpertWeights.from_synth(li)
+    rn = oracle.moe_layer(W, x, shape.n_experts, shape.top_k, shape.n_shared, router_w=rw, bias=bias, residual_bits=x)
+    assert np.array_equal(rc["logits32"], rn["logits32"]) and np.array_equal(rc["ids"], rn["ids"])
+    assert np.allclose(rc["w"], rn["w"], rtol=1e-14, atol=0)
+    _, acc_n = oracle.moe_ffn_combine(W, x, rn["ids"], rn["w"], shape.n_experts, shape.n_shared, residual_bits=x,
+                                      return_f64=True)
+    _assert_outputs_agree(rc["out"], rc["acc"], rn["out"], acc_n)
+
+
+def test_lazy_layer_matches_and_rejects_a_missing_selected_expert():
+    """The per-expert entry gives the contiguous entry's bits, and refuses to
+    run when an expert the batch selected was not given."""
+    rng = np.random.default_rng(80)
+    arr = _arrays(rng, 64, 32, 5, 32, 4)
+    x = synth.normal_bf16(81, 0, 1, (3, 64))
+    lg = rng.standard_normal((3, 4)).astype(np.float32)
+    fetch = lambda kind, e: (arr[kind][0][e], arr[kind][1][e])  # noqa: E731
+    r = cr.moe_layer_experts(fetch, 64, 32, x, 4, 2, 1, logits_in=lg)
+    full = cr.moe_layer(arr, x, 4, 2, 1, logits_in=lg)
+    assert np.array_equal(r["out"], full["out"]) and np.array_equal(r["acc"], full["acc"])
+    picked = set(r["ids"].ravel().tolist())
+    for missing in sorted(picked) + [4]:                 # a routed expert, then the shared one
+        with pytest.raises(ValueError):
+            cr.moe_layer_experts(fetch, 64, 32, x, 4, 2, 1, logits_in=lg, experts=(picked | {4}) - {missing})
