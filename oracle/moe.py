@@ -19,7 +19,9 @@ layer specification this library implements, and every place where it is a
 reading rather than a statement is marked READING.
 
 Parity pins live in ``tests/test_oracle_pins.py``; every function here is
-pinned there.
+pinned there.  ``oracle/c/moe_ref.c`` states the same layer again in plain C
+by other means, and ``tests/test_oracle_c.py`` checks the two against each
+other.
 """
 from __future__ import annotations
 
