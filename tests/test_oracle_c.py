@@ -413,3 +413,43 @@ def test_lazy_layer_matches_and_rejects_a_missing_selected_expert():
     for missing in sorted(picked) + [4]:                 # a routed expert, then the shared one
         with pytest.raises(ValueError):
             cr.moe_layer_experts(fetch, 64, 32, x, 4, 2, 1, logits_in=lg, experts=(picked | {4}) - {missing})
+
+
+def test_oracles_agree_on_random_small_layers():
+    """Property check over random shapes, containers, biases, residuals and
+    logit styles (computed, given with dense ties, given with NaN/inf)."""
+    from hypothesis import given, settings, HealthCheck
+    from hypothesis import strategies as st
+
+    @settings(max_examples=100, deadline=None, derandomize=True, suppress_health_check=list(HealthCheck))
+    @given(T=st.integers(0, 6), E=st.integers(1, 12), kfrac=st.floats(0, 1), S=st.integers(0, 2),
+           group=st.sampled_from([32, 64]), bits=st.sampled_from([4, 8]), hmul=st.integers(1, 2),
+           imul=st.integers(1, 2), logits=st.sampled_from(["router", "ties", "nonfinite"]),
+           use_bias=st.booleans(), use_res=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
+    def check(T, E, kfrac, S, group, bits, hmul, imul, logits, use_bias, use_res, seed):
+        rng = np.random.default_rng(seed)
+        k = 1 + int(kfrac * (E - 1))
+        H, I = 64 * hmul, 64 * imul
+        arr = _arrays(rng, H, I, E + S, group, bits)
+        x = synth.normal_bf16(seed % 1000, 3, 1, (T, H))
+        rw = lg = None
+        if logits == "router":
+            rw = (rng.standard_normal((E, H)) * 0.1).astype(np.float32)
+        else:
+            lg = rng.integers(-2, 3, size=(T, E)).astype(np.float32)
+            if logits == "nonfinite" and T:
+                lg[0, rng.integers(E)] = [np.nan, np.inf, -np.inf][int(rng.integers(3))]
+        bias = (rng.standard_normal(E) * 0.5).astype(np.float32) if use_bias else None
+        res = synth.normal_bf16(seed % 1000, 4, 1, (T, H)) if use_res else None
+        rc = cr.moe_layer(arr, x, E, k, S, group, bits, router_w=rw, logits_in=lg, bias=bias, residual_bits=res)
+        W = oracle.ExpertWeights.from_arrays(arr, group, bits)
+        rn = oracle.moe_layer(W, x, E, k, S, router_w=rw, logits_in=lg, bias=bias, residual_bits=res)
+        assert np.array_equal(rc["ids"], rn["ids"]) and np.array_equal(rc["flags"], rn["flags"])
+        assert np.array_equal(rc["logits32"], rn["logits32"], equal_nan=True)
+        if rn["flags"].any():
+            return                      # weights and outputs are not meaningful for flagged tokens
+        assert np.allclose(rc["w"], rn["w"], rtol=1e-14, atol=0)
+        _, acc_n = oracle.moe_ffn_combine(W, x, rn["ids"], rn["w"], E, S, residual_bits=res, return_f64=True)
+        _assert_outputs_agree(rc["out"], rc["acc"], rn["out"], acc_n)
+
+    check()

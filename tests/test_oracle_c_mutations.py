@@ -50,7 +50,7 @@ MUTATIONS = {  # name: (text in the source, replacement)
 
 def _pins():
     """The C oracle's pins, cheapest first; parametrised ones at fixed arguments."""
-    plain = [getattr(P, n) for n in dir(P) if n.startswith("test_") and "agrees" not in n and n not in (
+    plain = [getattr(P, n) for n in dir(P) if n.startswith("test_") and "agree" not in n and n not in (
         "test_dequant_group_index_and_rows", "test_batch_union_brute_force_and_inverse",
         "test_dense_identity_one_expert", "test_route_matches_brute_force_on_tie_dense_logits")]
     fixed = [lambda g=g, b=b: P.test_dequant_group_index_and_rows(g, b) for g, b in ((32, 4), (64, 4), (32, 8), (64, 8))]
