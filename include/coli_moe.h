@@ -212,8 +212,11 @@ coli_status coli_moe_layer_noalloc(const coli_moe_dims *dims, const coli_moe_wei
                                    float *logits_out, int32_t *topk_ids_out, float *topk_w_out,
                                    void *stream);
 
-/* Workspace bytes needed by coli_moe_layer / coli_moe_expert_ffn for up to T_max
- * tokens (0 for unsupported dims). Host only. */
+/* Workspace bytes that serve every coli_moe_layer / coli_moe_expert_ffn call of
+ * up to T_max tokens (0 for unsupported dims).  Not monotone in the form's own
+ * needs: the split-K decode form's partial sums at 8 tokens can take more than
+ * the two-phase form needs for larger batches, and the size returned for any
+ * T_max > 8 covers them.  Host only. */
 size_t coli_moe_workspace_bytes(const coli_moe_dims *dims, int T_max);
 
 /* FFN form taken by coli_moe_layer and coli_moe_expert_ffn for these dims, T

@@ -684,7 +684,15 @@ const char* coli_status_str(coli_status s) {
 
 size_t coli_moe_workspace_bytes(const coli_moe_dims* dims, int T_max) {
   if (check_dims(dims) != COLI_OK || T_max < 0) return 0;
-  return layout(dims, T_max, nullptr).bytes;
+  // Enough for every batch of up to T_max tokens.  The layout grows with T
+  // within each decode form, but the split-K form's partials at 8 tokens can
+  // outweigh what the two-phase form needs for somewhat larger batches.
+  size_t n = layout(dims, T_max, nullptr).bytes;
+  if (T_max > kSkMaxT) {
+    const size_t n_sk = layout(dims, kSkMaxT, nullptr).bytes;
+    if (n_sk > n) n = n_sk;
+  }
+  return n;
 }
 
 coli_status coli_moe_ffn_form(const coli_moe_dims* dims, int T, uint32_t flags, int* form) {

@@ -264,3 +264,41 @@ def test_layer_holder_checks_tensor_sizes(colimoe, bits):
         bad[name] = t[name][:, :-1]
         with pytest.raises(ValueError, match=name):
             m.MoELayer(d, bad)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(group=64), dict(code_bits=8), dict(hidden=1024, inter=512, n_experts=16),
+                                dict(hidden=256, inter=128, n_experts=16, top_k=2, n_shared=0)],
+                         ids=["glm", "glm_gs64", "glm_int8", "mid", "tiny_i128"])
+def test_workspace_for_t_max_covers_every_smaller_batch(colimoe, kw):
+    """A workspace of coli_moe_workspace_bytes(dims, T_max) bytes passes the
+    library's own workspace check for every batch of up to T_max tokens, in
+    the layer and the FFN call.  (On a machine without a GPU a call that passes
+    its checks stops at the device query with COLI_ERR_CUDA, before any launch.)"""
+    m = colimoe
+    lib = m._lib._lib
+    d, w = _dims(m, **kw), _weights(m)
+    int8 = kw.get("code_bits") == 8
+    f = _fake(0x500000)
+    t_maxes = list(range(0, 40)) + [63, 64, 65, 77, 78, 100, 129, 300]
+    for t_max in t_maxes:
+        n = m.coli_moe_workspace_bytes(d, t_max)
+        assert n > 0
+        for T in range(0, t_max + 1):
+            if int8 and T > 8:
+                break
+            st_layer = lib.coli_moe_layer(ctypes.byref(d), ctypes.byref(w), _fake(0x200000), T, None, None, 0,
+                                          _fake(0x300000), None, None, None, _fake(0x400000), n, None)
+            st_ffn = lib.coli_moe_expert_ffn(ctypes.byref(d), ctypes.byref(w), _fake(0x200000), T, f, f, f, f, f, f,
+                                             f, None, _fake(0x600000), 0, _fake(0x700000), n, None)
+            assert st_layer != m._lib.COLI_ERR_WORKSPACE and st_ffn != m._lib.COLI_ERR_WORKSPACE, (t_max, T)
+            assert st_layer in (m._lib.COLI_OK, m._lib.COLI_ERR_CUDA), st_layer
+    # and the size is not padded beyond the largest batch's need: one byte less fails for some T <= T_max
+    for t_max in (1, 8, 9, 64, 300):
+        n = m.coli_moe_workspace_bytes(d, t_max)
+        if int8 and t_max > 8:
+            continue
+        worst = [T for T in range(1, t_max + 1)
+                 if lib.coli_moe_layer(ctypes.byref(d), ctypes.byref(w), _fake(0x200000), T, None, None, 0,
+                                       _fake(0x300000), None, None, None, _fake(0x400000), n - 1, None)
+                 == m._lib.COLI_ERR_WORKSPACE]
+        assert worst, t_max
