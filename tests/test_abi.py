@@ -302,3 +302,40 @@ def test_workspace_for_t_max_covers_every_smaller_batch(colimoe, kw):
                                        _fake(0x300000), None, None, None, _fake(0x400000), n - 1, None)
                  == m._lib.COLI_ERR_WORKSPACE]
         assert worst, t_max
+
+
+def test_ffn_form_status_equals_the_calls_status(colimoe):
+    """For any dims, T and flags, coli_moe_ffn_form fails exactly when the
+    layer and FFN calls fail on them (same status); when it succeeds the calls
+    get past every check (to the device query, COLI_ERR_CUDA without a GPU)."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    m = colimoe
+    lib = m._lib._lib
+    w, f = _weights(m), _fake(0x500000)
+    big = 1 << 40
+
+    @settings(max_examples=400, deadline=None, derandomize=True, suppress_health_check=list(HealthCheck))
+    @given(hidden=st.sampled_from([128, 256, 512, 768, 1024, 6144, 6000]),
+           inter=st.sampled_from([64, 128, 256, 384, 512, 768, 2048]),
+           n_experts=st.sampled_from([1, 2, 16, 256, 1024, 1025]), top_k=st.sampled_from([1, 2, 8, 32, 33]),
+           n_shared=st.sampled_from([0, 1, 4, 5]), group=st.sampled_from([16, 32, 64, 128]),
+           code_bits=st.sampled_from([0, 4, 5, 8]), T=st.sampled_from([-1, 0, 1, 5, 8, 9, 64, 300, 4096]),
+           flags=st.sampled_from([0, 0x1, 0x10, 0x20, 0x30, 0x11, 0x21]))
+    def check(hidden, inter, n_experts, top_k, n_shared, group, code_bits, T, flags):
+        d = m.coli_moe_dims(hidden, inter, n_experts, top_k, n_shared, group, code_bits)
+        form = ctypes.c_int(-1)
+        st_form = lib.coli_moe_ffn_form(ctypes.byref(d), T, flags, ctypes.byref(form))
+        st_layer = lib.coli_moe_layer(ctypes.byref(d), ctypes.byref(w), _fake(0x200000), T, None, None, flags,
+                                      _fake(0x300000), None, None, None, _fake(0x400000), big, None)
+        st_ffn = lib.coli_moe_expert_ffn(ctypes.byref(d), ctypes.byref(w), _fake(0x200000), T, f, f, f, f, f, f, f,
+                                         None, _fake(0x600000), flags, _fake(0x700000), big, None)
+        if st_form != m._lib.COLI_OK:
+            assert st_layer == st_form and st_ffn == st_form, (st_form, st_layer, st_ffn)
+            assert form.value == 0
+        elif T == 0:
+            assert st_layer == st_ffn == m._lib.COLI_OK and form.value == 0
+        else:
+            assert st_layer == st_ffn == m._lib.COLI_ERR_CUDA and form.value in (1, 2, 3)
+
+    check()
