@@ -8,7 +8,8 @@ import ctypes
 
 import torch
 
-from ._lib import coli_moe_dims, coli_moe_layer, coli_moe_weights, coli_moe_workspace_bytes
+from ._lib import (COLI_ERR_INVALID_ARG, COLI_ERR_UNSUPPORTED, ColiError, coli_moe_dims, coli_moe_layer,
+                   coli_moe_weights, coli_moe_workspace_bytes)
 
 
 def dims_for(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int, group: int = 32,
@@ -41,7 +42,11 @@ class MoELayer:
                                         p(router_w), p(bias))
 
     def workspace(self, t_max: int, device="cuda") -> torch.Tensor:
+        """Scratch for any call of up to ``t_max`` tokens; raises ColiError for
+        dims the library does not support or a negative ``t_max``."""
         n = coli_moe_workspace_bytes(self.dims, t_max)
+        if n == 0:
+            raise ColiError(COLI_ERR_INVALID_ARG if t_max < 0 else COLI_ERR_UNSUPPORTED, "coli_moe_workspace_bytes")
         return torch.empty(n, dtype=torch.uint8, device=device)
 
     def forward(self, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, logits_in=None, residual=None,

@@ -339,3 +339,26 @@ def test_ffn_form_status_equals_the_calls_status(colimoe):
             assert st_layer == st_ffn == m._lib.COLI_ERR_CUDA and form.value in (1, 2, 3)
 
     check()
+
+
+def test_layer_holder_workspace_refuses_unsupported_dims(colimoe):
+    import torch
+    m = colimoe
+    H, I, E, S = 256, 256, 4, 1
+
+    def holder(group):
+        t = {"gate_q": torch.zeros(E + S, I, H // 2, dtype=torch.uint8),
+             "up_q": torch.zeros(E + S, I, H // 2, dtype=torch.uint8),
+             "down_q": torch.zeros(E + S, H, I // 2, dtype=torch.uint8),
+             "gate_s": torch.zeros(E + S, I, H // group, dtype=torch.int16),
+             "up_s": torch.zeros(E + S, I, H // group, dtype=torch.int16),
+             "down_s": torch.zeros(E + S, H, I // group, dtype=torch.int16)}
+        return m.MoELayer(m.dims_for(H, I, E, 2, S, group), t)
+
+    assert holder(32).workspace(4, device="cpu").numel() == m.coli_moe_workspace_bytes(holder(32).dims, 4)
+    with pytest.raises(m._lib.ColiError) as e:
+        holder(16).workspace(4, device="cpu")
+    assert e.value.status == m._lib.COLI_ERR_UNSUPPORTED
+    with pytest.raises(m._lib.ColiError) as e:
+        holder(32).workspace(-1, device="cpu")
+    assert e.value.status == m._lib.COLI_ERR_INVALID_ARG
