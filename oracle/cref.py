@@ -29,7 +29,7 @@ _lib = None
 def build(force: bool = False) -> str:
     """Compile the C oracle if its library is missing or older than the source."""
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
-        tmp = LIB + ".tmp"
+        tmp = f"{LIB}.{os.getpid()}.tmp"       # concurrent test processes each build their own, then rename
         r = subprocess.run([CC, *CFLAGS, SRC, "-o", tmp, "-lm"], capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"{CC} failed for the C oracle:\n{r.stdout}\n{r.stderr}")
