@@ -49,7 +49,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     for name, t in TARGETS.items():
         if not force and not _stale(t):
             continue
-        cmd = [NVCC, *ARCH, *COMMON, *(f"-I{d}" for d in t["inc"]), t["main"], "-o", t["out"] + ".tmp"]
+        tmp = f"{t['out']}.{os.getpid()}.tmp"     # concurrent builds each write their own, then rename
+        cmd = [NVCC, *ARCH, *COMMON, *(f"-I{d}" for d in t["inc"]), t["main"], "-o", tmp]
         if ptxas_info:
             cmd[1:1] = ["-Xptxas", "-v"]
         if verbose:
@@ -59,7 +60,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             raise RuntimeError(f"nvcc failed for {name}:\n{r.stdout}\n{r.stderr}")
         if verbose or ptxas_info:
             sys.stderr.write(r.stderr)
-        os.replace(t["out"] + ".tmp", t["out"])
+        os.replace(tmp, t["out"])
         built.append(t["out"])
     return built
 
