@@ -79,7 +79,17 @@ def status_str(s: int) -> str:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor argument (None -> NULL).  The library reads and
+    writes dense row-major device buffers, so only contiguous CUDA tensors pass:
+    a strided view would be read as if it were dense, and a host pointer would
+    reach a kernel."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (dense, row-major)")
+    if t.device.type != "cuda":
+        raise ValueError(f"tensor arguments must be in device memory, got a tensor on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):

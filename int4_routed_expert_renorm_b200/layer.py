@@ -36,6 +36,10 @@ class MoELayer:
                 raise ValueError(f"{name}: {self.t[name].numel()} elements, the dims need {shp}")
         self.router_w = router_w
         self.bias = bias
+        held = [self.t[name] for name in want] + [v for v in (router_w, bias) if v is not None]
+        if not all(v.is_contiguous() for v in held):
+            raise ValueError("weight tensors must be contiguous (dense, row-major)")
+        self._on_device = all(v.device.type == "cuda" for v in held)
         p = lambda x: None if x is None else ctypes.c_void_p(x.data_ptr())  # noqa: E731
         self.weights = coli_moe_weights(p(self.t["gate_q"]), p(self.t["up_q"]), p(self.t["down_q"]),
                                         p(self.t["gate_s"]), p(self.t["up_s"]), p(self.t["down_s"]),
@@ -51,6 +55,8 @@ class MoELayer:
 
     def forward(self, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, logits_in=None, residual=None,
                 flags: int = 0, logits_out=None, topk_ids_out=None, topk_w_out=None, stream=None):
+        if not self._on_device:
+            raise ValueError("the layer's weight tensors must be in device memory")
         coli_moe_layer(self.dims, self.weights, x, out, ws, logits_in=logits_in, residual=residual, flags=flags,
                        logits_out=logits_out, topk_ids_out=topk_ids_out, topk_w_out=topk_w_out, stream=stream)
         return out

@@ -362,3 +362,31 @@ def test_layer_holder_workspace_refuses_unsupported_dims(colimoe):
     with pytest.raises(m._lib.ColiError) as e:
         holder(32).workspace(-1, device="cpu")
     assert e.value.status == m._lib.COLI_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_and_strided_tensors(colimoe):
+    """Tensor arguments must be contiguous device buffers: a host tensor or a
+    strided view is refused before anything reaches the library."""
+    import torch
+    m = colimoe
+    lg = torch.zeros(4, 16)
+    ids, w = torch.zeros(4, 2, dtype=torch.int32), torch.zeros(4, 2)
+    with pytest.raises(ValueError, match="device memory"):
+        m.coli_moe_route(lg, None, ids, w)
+    with pytest.raises(ValueError, match="contiguous"):
+        m.coli_moe_route(torch.zeros(16, 4).t(), None, ids, w)
+    H, I, E, S, G = 256, 256, 4, 1, 32
+    t = {"gate_q": torch.zeros(E + S, I, H // 2, dtype=torch.uint8),
+         "up_q": torch.zeros(E + S, I, H // 2, dtype=torch.uint8),
+         "down_q": torch.zeros(E + S, H, I // 2, dtype=torch.uint8),
+         "gate_s": torch.zeros(E + S, I, H // G, dtype=torch.int16),
+         "up_s": torch.zeros(E + S, I, H // G, dtype=torch.int16),
+         "down_s": torch.zeros(E + S, H, I // G, dtype=torch.int16)}
+    d = m.dims_for(H, I, E, 2, S, G)
+    layer = m.MoELayer(d, t)                                  # host tensors are held, but never run
+    x = torch.zeros(2, H, dtype=torch.int16)
+    with pytest.raises(ValueError, match="device memory"):
+        layer.forward(x, torch.empty_like(x), torch.empty(16, dtype=torch.uint8))
+    bad = dict(t, down_s=torch.zeros(E + S, I // G, H, dtype=torch.int16).transpose(1, 2))
+    with pytest.raises(ValueError, match="contiguous"):
+        m.MoELayer(d, bad)
