@@ -79,3 +79,16 @@ def test_zipf_bias_is_a_log_rank_prior():
     ranks = np.rint(np.exp(-b.astype(np.float64) / 1.1)).astype(int)
     assert sorted(ranks.tolist()) == list(range(1, 257))
     assert np.allclose(b, (-1.1 * np.log(ranks)).astype(np.float32), rtol=0, atol=0)
+
+
+def test_expert_bytes_match_the_worked_sizes():
+    """Bytes of one expert (three matrices, codes + fp16 scales), the unit of
+    the roofline's algorithmic bytes: 18,874,368 B of int4 codes + 2,359,296 B
+    of group-32 scales at the GLM shape; 49,152 + 6,144 B for the tiny layer."""
+    assert synth.DECODE_B1.expert_bytes() == 18_874_368 + 2_359_296 == 21_233_664
+    assert synth.TINY.expert_bytes() == 49_152 + 6_144
+    assert synth.DECODE_B1_GS64.expert_bytes() == 18_874_368 + 1_179_648      # one scale per 64 codes
+    assert synth.DECODE_B1_INT8.expert_bytes() == 37_748_736 + 2_359_296      # one byte per code
+    # a GLM layer with its shared expert, and the 16-layer stack, in GB
+    assert round(257 * synth.DECODE_B1.expert_bytes() / 1e9, 3) == 5.457
+    assert round(16 * 257 * synth.STACK16_B4.expert_bytes() / 1e9, 1) == 87.3
