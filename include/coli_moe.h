@@ -219,6 +219,18 @@ coli_status coli_moe_layer_noalloc(const coli_moe_dims *dims, const coli_moe_wei
  * T_max > 8 covers them.  Host only. */
 size_t coli_moe_workspace_bytes(const coli_moe_dims *dims, int T_max);
 
+/* Where coli_moe_layer leaves the batch-union it computed (for tests and
+ * diagnostics; the pages have no counterpart): byte offsets, within the `ws`
+ * of a coli_moe_layer call with these dims and T, of the union step's outputs
+ * as coli_moe_union defines them,
+ *   off[0] unique_ids  int32 [min(E, T*k)]    off[3] perm      int32 [T*k]
+ *   off[1] n_unique    int32 [1]              off[4] pair_pos  int32 [T*k]
+ *   off[2] seg_off     int32 [min(E, T*k) + 1]
+ * They hold that call's union once it has run, until the next call that uses
+ * the same workspace.  off: host array of 5.  Host only; returns the status
+ * of the dims and T checks (COLI_ERR_INVALID_ARG for T < 0 or off == NULL). */
+coli_status coli_moe_union_offsets(const coli_moe_dims *dims, int T, size_t *off);
+
 /* FFN form taken by coli_moe_layer and coli_moe_expert_ffn for these dims, T
  * and flags (the rule under COLI_PATH_* above).  Host only: launches nothing
  * and needs no device.
@@ -239,6 +251,21 @@ coli_status coli_moe_ffn_form(const coli_moe_dims *dims, int T, uint32_t flags, 
  * NONFINITE bit was set, COLI_ERR_DEVICE for any other bit, COLI_ERR_CUDA if
  * the synchronisation failed.  Not capturable. */
 coli_status coli_moe_get_status(void *stream, uint32_t *flags);
+
+/* Test hook of the device-side bounded waits; the pages have no counterpart.
+ * Enqueues one tiny kernel whose single thread waits, with a limit of
+ * limit_ns nanoseconds of %globaltimer, first on a shared-memory barrier
+ * that nothing arrives on and then on a device counter that nothing
+ * increments -- the same wait routines every pipeline wait of the FFN kernels
+ * uses (there with a limit of 2 s).  Both waits give up, set
+ * COLI_FLAG_TIMEOUT in the status word and the kernel returns: the device
+ * stays usable.
+ *   limit_ns    0 < limit_ns <= 2e9, else COLI_ERR_INVALID_ARG
+ *   elapsed_ns  device pointer to 2 uint64 (8-byte aligned) receiving how
+ *               long each wait lasted before giving up, or NULL
+ * Read the result with coli_moe_get_status (COLI_ERR_DEVICE, flags
+ * COLI_FLAG_TIMEOUT). */
+coli_status coli_moe_test_wait_timeout(uint64_t limit_ns, uint64_t *elapsed_ns, void *stream);
 
 /* Static description of a status code. */
 const char *coli_status_str(coli_status s);

@@ -23,7 +23,8 @@ COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
-           "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form")
+           "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form",
+           "coli_moe_union_offsets", "coli_moe_test_wait_timeout")
 COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -64,6 +65,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_set_stage_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
         "coli_moe_layer_noalloc": (I, [D, W, P, I, P, P, U32, P, P, P, P, P]),
         "coli_moe_ffn_form": (I, [D, I, U32, ctypes.POINTER(I)]),
+        "coli_moe_union_offsets": (I, [D, I, ctypes.POINTER(Z)]),
+        "coli_moe_test_wait_timeout": (I, [U64, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -90,6 +93,34 @@ def _ptr(t):
     if t.device.type != "cuda":
         raise ValueError(f"tensor arguments must be in device memory, got a tensor on {t.device}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, n: int, esize: int, name: str, at_least: bool = False):
+    """Refuse a tensor whose size does not match what the C call will read or
+    write through its pointer (n elements of esize bytes; None passes)."""
+    if t is None:
+        return
+    if t.element_size() != esize:
+        raise ValueError(f"{name}: elements of {t.element_size()} bytes, the call needs {esize}")
+    if (t.numel() < n) if at_least else (t.numel() != n):
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {'at least ' if at_least else ''}{n}")
+
+
+def _tokens(x, H: int) -> int:
+    if x.dim() != 2 or x.shape[1] != H:
+        raise ValueError(f"x: shape {tuple(x.shape)}, the call needs [T, {H}]")
+    _need(x, x.shape[0] * H, 2, "x")
+    return x.shape[0]
+
+
+def _layer_sizes(dims, T: int, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out):
+    H, E, k = dims.hidden, dims.n_experts, dims.top_k
+    _need(out, T * H, 2, "out")
+    _need(residual, T * H, 2, "residual")
+    _need(logits_in, T * E, 4, "logits_in")
+    _need(logits_out, T * E, 4, "logits_out")
+    _need(topk_ids_out, T * k, 4, "topk_ids_out")
+    _need(topk_w_out, T * k, 4, "topk_w_out")
 
 
 def _stream(stream):
@@ -127,19 +158,37 @@ def coli_moe_ffn_form(dims: coli_moe_dims, T: int, flags: int = 0) -> int:
 def coli_moe_route(logits, bias, topk_ids, topk_w, stream=None):
     T, E = logits.shape
     k = topk_ids.shape[1]
+    _need(logits, T * E, 4, "logits")
+    _need(bias, E, 4, "bias")
+    _need(topk_ids, T * k, 4, "topk_ids")
+    _need(topk_w, T * k, 4, "topk_w")
     _check(_lib.coli_moe_route(_ptr(logits), _ptr(bias), T, E, k, _ptr(topk_ids), _ptr(topk_w), _stream(stream)),
            "coli_moe_route")
 
 
 def coli_moe_union(topk_ids, n_experts, unique_ids, n_unique, seg_off, perm, pair_pos, stream=None):
     T, k = topk_ids.shape
+    P = T * k
+    _need(topk_ids, P, 4, "topk_ids")
+    _need(unique_ids, min(n_experts, P), 4, "unique_ids", at_least=True)
+    _need(n_unique, 1, 4, "n_unique", at_least=True)
+    _need(seg_off, min(n_experts, P) + 1, 4, "seg_off", at_least=True)
+    _need(perm, P, 4, "perm", at_least=True)
+    _need(pair_pos, P, 4, "pair_pos", at_least=True)
     _check(_lib.coli_moe_union(_ptr(topk_ids), T, k, n_experts, _ptr(unique_ids), _ptr(n_unique), _ptr(seg_off),
                                _ptr(perm), _ptr(pair_pos), _stream(stream)), "coli_moe_union")
 
 
 def coli_moe_expert_ffn(dims, weights, x, topk_ids, topk_w, unique_ids, n_unique, seg_off, perm, pair_pos,
                         residual, out, ws, flags=0, stream=None):
-    T = x.shape[0]
+    T = _tokens(x, dims.hidden)
+    P, E = T * dims.top_k, dims.n_experts
+    _layer_sizes(dims, T, out, residual, None, None, topk_ids, topk_w)
+    _need(unique_ids, min(E, P), 4, "unique_ids", at_least=True)
+    _need(n_unique, 1, 4, "n_unique", at_least=True)
+    _need(seg_off, min(E, P) + 1, 4, "seg_off", at_least=True)
+    _need(perm, P, 4, "perm", at_least=True)
+    _need(pair_pos, P, 4, "pair_pos", at_least=True)
     _check(_lib.coli_moe_expert_ffn(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(topk_ids),
                                     _ptr(topk_w), _ptr(unique_ids), _ptr(n_unique), _ptr(seg_off), _ptr(perm),
                                     _ptr(pair_pos), _ptr(residual), _ptr(out), flags, _ptr(ws),
@@ -148,7 +197,8 @@ def coli_moe_expert_ffn(dims, weights, x, topk_ids, topk_w, unique_ids, n_unique
 
 def coli_moe_layer(dims, weights, x, out, ws, logits_in=None, residual=None, flags=0, logits_out=None,
                    topk_ids_out=None, topk_w_out=None, stream=None):
-    T = x.shape[0]
+    T = _tokens(x, dims.hidden)
+    _layer_sizes(dims, T, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
     _check(_lib.coli_moe_layer(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
                                _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
                                _ptr(topk_w_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
@@ -159,10 +209,26 @@ def coli_moe_layer_noalloc(dims, weights, x, out, logits_in=None, residual=None,
                            topk_ids_out=None, topk_w_out=None, stream=None):
     """coli_moe_layer with the library's own scratch instead of a workspace
     tensor, for callers that cannot allocate device memory (see the header)."""
-    T = x.shape[0]
+    T = _tokens(x, dims.hidden)
+    _layer_sizes(dims, T, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
     _check(_lib.coli_moe_layer_noalloc(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
                                        _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
                                        _ptr(topk_w_out), _stream(stream)), "coli_moe_layer_noalloc")
+
+
+def coli_moe_union_offsets(dims, T: int) -> list[int]:
+    """Byte offsets of unique_ids, n_unique, seg_off, perm and pair_pos inside
+    the workspace of a coli_moe_layer call with these dims and T."""
+    off = (ctypes.c_size_t * 5)()
+    _check(_lib.coli_moe_union_offsets(ctypes.byref(dims), T, off), "coli_moe_union_offsets")
+    return list(off)
+
+
+def coli_moe_test_wait_timeout(limit_ns: int, elapsed=None, stream=None):
+    """Test hook of the bounded device waits (see the header); elapsed: None or
+    a device int64 tensor of 2 elements receiving each wait's duration in ns."""
+    _need(elapsed, 2, 8, "elapsed")
+    _check(_lib.coli_moe_test_wait_timeout(limit_ns, _ptr(elapsed), _stream(stream)), "coli_moe_test_wait_timeout")
 
 
 def coli_moe_set_stage_events(events):

@@ -31,6 +31,33 @@ namespace {
 
 __device__ uint32_t g_status_word;
 
+// A counter nothing ever increments: the grid-counter wait of the timeout hook.
+__device__ int32_t g_never_counted;
+
+// Test hook of the bounded waits (coli_moe_test_wait_timeout): one thread waits
+// with a limit of limit_ns on an mbarrier nothing arrives on, then on a
+// counter nothing increments -- the same helpers every pipeline wait of the
+// FFN kernels uses.  Each wait gives up, sets COLI_FLAG_TIMEOUT and returns;
+// elapsed[0..1] (may be NULL) receive the time each one took.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, uint64_t* elapsed, uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  const uint64_t t0 = globaltimer();
+  const bool got_bar = mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  const uint64_t t1 = globaltimer();
+  abort_flag = 0;
+  const bool got_cnt = wait_counter(&g_never_counted, 1, &abort_flag, status, limit_ns);
+  const uint64_t t2 = globaltimer();
+  if (elapsed) {
+    elapsed[0] = got_bar ? 0 : t1 - t0;
+    elapsed[1] = got_cnt ? 0 : t2 - t1;
+  }
+}
+
 thread_local uint64_t t_launches = 0;
 
 // Stage events of the timing hook (coli_moe_set_stage_events); consumed by one call.
@@ -100,17 +127,17 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_PF_SMEM(2, 64)
     COLI_SET_PF_SMEM(1, 64)
 #undef COLI_SET_PF_SMEM
-#define COLI_SET_SK_SMEM(SG, GR, B)                                                                        \
-  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<SG, GR, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define COLI_SET_SK_SMEM(NT, GR, B)                                                                        \
+  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<NT, GR, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(SkCfg<GR, B>::SMEM)) == cudaSuccess;
-    COLI_SET_SK_SMEM(true, 32, 4)
-    COLI_SET_SK_SMEM(false, 32, 4)
-    COLI_SET_SK_SMEM(true, 64, 4)
-    COLI_SET_SK_SMEM(false, 64, 4)
-    COLI_SET_SK_SMEM(true, 32, 8)
-    COLI_SET_SK_SMEM(false, 32, 8)
-    COLI_SET_SK_SMEM(true, 64, 8)
-    COLI_SET_SK_SMEM(false, 64, 8)
+    COLI_SET_SK_SMEM(1, 32, 4)
+    COLI_SET_SK_SMEM(2, 32, 4)
+    COLI_SET_SK_SMEM(1, 64, 4)
+    COLI_SET_SK_SMEM(2, 64, 4)
+    COLI_SET_SK_SMEM(1, 32, 8)
+    COLI_SET_SK_SMEM(2, 32, 8)
+    COLI_SET_SK_SMEM(1, 64, 8)
+    COLI_SET_SK_SMEM(2, 64, 8)
 #undef COLI_SET_SK_SMEM
     ok &= cudaFuncSetAttribute(logits_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
           cudaSuccess;
@@ -199,6 +226,8 @@ struct Ws {
   uint16_t* xg;      // [P][H] expert input gathered into pair order (prefill form), directly followed by xq
   uint16_t* xq;      // [T][H] fragment-ordered expert input
   uint16_t* xn;      // [T][H] normalised input (prenorm)
+  uint8_t* xp;       // split-K form: [T][H/32][kPlaneRec] integer planes of the expert input
+  int32_t* xe;       // split-K form: [T] their grid exponents
   float* logits;     // [T][E]
   int32_t* ids;      // [T*k]
   float* w;          // [T*k]
@@ -252,6 +281,14 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
   ws.xg = static_cast<uint16_t*>(take((P + static_cast<size_t>(T)) * H * 2));
   ws.xq = ws.xg ? ws.xg + P * H : nullptr;
   ws.xn = static_cast<uint16_t*>(take(T * H * 2));
+  {
+    const size_t tsk = use_splitk(d, T) ? static_cast<size_t>(T) : 0;
+    // NULL when the batch takes another form: the front kernels then write no planes
+    uint8_t* xp = static_cast<uint8_t*>(take(tsk * (H / 32) * kPlaneRec));
+    int32_t* xe = static_cast<int32_t*>(take(tsk * 4));
+    ws.xp = tsk ? xp : nullptr;
+    ws.xe = tsk ? xe : nullptr;
+  }
   ws.logits = static_cast<float*>(take(T * E * 4));
   ws.ids = static_cast<int32_t*>(take(P * 4));
   ws.w = static_cast<float*>(take(P * 4));
@@ -340,6 +377,20 @@ bool launch_cooperative(FfnKernel kernel, size_t smem, const CUtensorMap* m, con
     e = cudaLaunchKernelEx(&cfg, kernel, m[0], m[1], m[2], m[3], m[4], m[5], a);
   }
   return e == cudaSuccess;
+}
+
+// The split-K kernel as a plain launch with programmatic dependent launch:
+// its grid is at most one CTA per SM and its shared memory admits one CTA
+// per SM, so every CTA becomes resident without a cooperative launch (a CTA
+// that finds its SM still busy with the routing kernel's one CTA starts when
+// that CTA ends; the routing kernel waits on nothing of this kernel).  The
+// plain launch lets the CTAs start their prologue and the shared experts'
+// weight stream while the routing kernel still runs, which a cooperative
+// launch does not.  Every wait in the kernel is bounded.
+bool launch_splitk(FfnKernel kernel, size_t smem, const CUtensorMap* m, const FfnArgs& a, int grid, int sms,
+                   cudaStream_t st) {
+  if (grid > sms) return false;
+  return launch(kernel, dim3(grid), dim3(kFfnThreads), smem, st, m[0], m[1], m[2], m[3], m[4], m[5], a);
 }
 
 template <int NT, bool SG, int KCD, int GR>
@@ -609,20 +660,24 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
                    CU_TENSOR_MAP_SWIZZLE_NONE))
       return COLI_ERR_CUDA;
     a.ypart = ws.ypair;
+    a.xp = ws.xp;
+    a.xe = ws.xe;
     const long tiles = blocks_ub * (I / kRowBlock);
     const int grid = static_cast<int>(tiles < di.sms ? tiles : di.sms);
+    // MMA n-tiles of four tokens each
+    const bool nt2 = T > 4;
     FfnKernel k;
     size_t smem;
     if (B == 4) {
-      k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32, 4> : ffn_splitk_kernel<true, 64, 4>)
-                 : (G == 32 ? ffn_splitk_kernel<false, 32, 4> : ffn_splitk_kernel<false, 64, 4>);
+      k = nt2 ? (G == 32 ? ffn_splitk_kernel<2, 32, 4> : ffn_splitk_kernel<2, 64, 4>)
+              : (G == 32 ? ffn_splitk_kernel<1, 32, 4> : ffn_splitk_kernel<1, 64, 4>);
       smem = G == 32 ? SkCfg<32, 4>::SMEM : SkCfg<64, 4>::SMEM;
     } else {
-      k = T == 1 ? (G == 32 ? ffn_splitk_kernel<true, 32, 8> : ffn_splitk_kernel<true, 64, 8>)
-                 : (G == 32 ? ffn_splitk_kernel<false, 32, 8> : ffn_splitk_kernel<false, 64, 8>);
+      k = nt2 ? (G == 32 ? ffn_splitk_kernel<2, 32, 8> : ffn_splitk_kernel<2, 64, 8>)
+              : (G == 32 ? ffn_splitk_kernel<1, 32, 8> : ffn_splitk_kernel<1, 64, 8>);
       smem = G == 32 ? SkCfg<32, 8>::SMEM : SkCfg<64, 8>::SMEM;
     }
-    if (!launch_cooperative(k, smem, maps, a, grid, st)) return COLI_ERR_CUDA;
+    if (!launch_splitk(k, smem, maps, a, grid, di.sms, st)) return COLI_ERR_CUDA;
     rec.mark_through(6, 7);
     rec.mark(8);
     return COLI_OK;
@@ -695,6 +750,25 @@ size_t coli_moe_workspace_bytes(const coli_moe_dims* dims, int T_max) {
   return n;
 }
 
+coli_status coli_moe_union_offsets(const coli_moe_dims* dims, int T, size_t* off) {
+  if (!off) return COLI_ERR_INVALID_ARG;
+  const coli_status st = check_dims(dims);
+  if (st != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  // the layout of a workspace based at address 0 gives the offsets (256-byte
+  // aligned, so any workspace the calls accept has the same ones)
+  uint8_t* const base = reinterpret_cast<uint8_t*>(uintptr_t(256));
+  const Ws w = layout(dims, T, base);
+  auto rel = [&](const void* p) { return static_cast<size_t>(static_cast<const uint8_t*>(p) - base); };
+  off[0] = rel(w.unique);
+  off[1] = rel(w.n_unique);
+  off[2] = rel(w.seg_off);
+  off[3] = rel(w.perm);
+  off[4] = rel(w.pair_pos);
+  return COLI_OK;
+}
+
 coli_status coli_moe_ffn_form(const coli_moe_dims* dims, int T, uint32_t flags, int* form) {
   if (!form) return COLI_ERR_INVALID_ARG;
   *form = 0;
@@ -765,7 +839,8 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   cudaStream_t s = as_stream(stream);
   const StageRecorder rec(s);
   rec.mark(0);
-  if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq))
+  if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq,
+              lay.xp, lay.xe))
     return COLI_ERR_CUDA;
   rec.mark_through(1, 4);
   if (form == Form::kPrefill)
@@ -813,12 +888,15 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   if (fused_front) {
     const float* wr = logits_in ? nullptr : w->router_w;
     const int grid = logits_in ? T : E;
-    if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq))
+    if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq,
+                lay.xp, lay.xe))
       return COLI_ERR_CUDA;
     rec.mark_through(1, 2);
     if (!logits_in) lg = lo;
   } else {
-    if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, H, prenorm ? 1 : 0, lay.xn, lay.xq)) return COLI_ERR_CUDA;
+    if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, H, prenorm ? 1 : 0, lay.xn, lay.xq,
+                static_cast<uint8_t*>(nullptr), static_cast<int32_t*>(nullptr)))
+      return COLI_ERR_CUDA;
     rec.mark(1);
     if (!logits_in) {
       const uint16_t* xr = prenorm ? lay.xn : x;
@@ -895,6 +973,16 @@ coli_status coli_moe_layer_noalloc(const coli_moe_dims* dims, const coli_moe_wei
   }
   return coli_moe_layer(dims, w, x, T, logits_in, residual, flags, out, logits_out, topk_ids_out, topk_w_out, ptr,
                         COLI_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+coli_status coli_moe_test_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > kWaitLimitNs) return COLI_ERR_INVALID_ARG;
+  if (elapsed_ns && !aligned(elapsed_ns, 8)) return COLI_ERR_INVALID_ARG;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  return launch(wait_timeout_kernel, dim3(1), dim3(32), 0, as_stream(stream), limit_ns, elapsed_ns, di.status)
+             ? COLI_OK
+             : COLI_ERR_CUDA;
 }
 
 coli_status coli_moe_get_status(void* stream, uint32_t* flags) {

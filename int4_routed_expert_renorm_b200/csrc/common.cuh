@@ -60,17 +60,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Returns false
 // (and leaves the barrier alone) if `abort_flag` was raised by another warp or
-// if the wait ran past kWaitLimitNs, in which case it raises `abort_flag` and
-// sets COLI_FLAG_TIMEOUT in the status word.
+// if the wait ran past limit_ns (kWaitLimitNs unless a test passes a shorter
+// limit), in which case it raises `abort_flag` and sets COLI_FLAG_TIMEOUT in
+// the status word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         atomicOr(status, COLI_FLAG_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -88,6 +89,37 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// L2 cache policies (createpolicy): data read once and not shared with other
+// CTAs goes in with evict_first, so that it does not push out what the kernel
+// reads again later; data written now and read back at the end of the kernel
+// goes in with evict_last.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// tma_load_2d with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                                                 int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// One fp32 store to global memory (L2) with an L2 cache policy.
+__device__ __forceinline__ void st_f32_hint(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
 }
 
 // Contiguous bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
@@ -153,6 +185,82 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t b) { return __half2
 __device__ __forceinline__ int frag_pos(int i) {
   const int p = i & 7;
   return (i & ~7) | (p < 4 ? 2 * p : 2 * (p - 4) + 1);
+}
+
+// ---------------------------------------------------------------------------
+// Integer activation planes of the decode form for batches of up to 8 tokens.
+//
+// The expert input of one token (and each 128-row slice of h of one pair) is
+// put on a fixed-point grid of its own: v -> q = rint(v * 2^e), with e the
+// power of two that brings the largest |v| into [2^13, 2^14).  Every value
+// whose magnitude is at least 2^-6 of that largest one lands on the grid
+// exactly (a bf16 value has 8 significant bits); the smaller ones are rounded
+// to the nearest grid point, the grid step being at most max|v| * 2^-13.
+// |q| < 2^14 is then written as
+// two signed bytes, q = 256 * hi + lo with lo in [-128, 127] and hi in
+// [-64, 64]: the "low" and "high" planes, the B operands of an integer MMA
+// (mma.sync m16n8k32, u8/s8 x s8 -> s32) against the int4 (or int8) codes.
+//
+// Record of one 32-wide K group of one token: 72 bytes,
+//   [0, 32)   low plane, [32, 64) high plane: lane c (0..3) of an MMA quad
+//             owns elements 8c .. 8c+7 of the group, stored as the 4 even
+//             ones then the 4 odd ones (the order in which an int4 code word
+//             of 8 nibbles splits into its low and high nibbles);
+//   [64, 72)  two int32: the MMA accumulator's start value for the low and
+//             the high column, kPlaneMagic - 8 * (sum of the low plane) and
+//             -8 * (sum of the high plane).  The -8 * sum terms cancel the +8
+//             that turns a two's-complement int4 code into an unsigned byte;
+//             kPlaneMagic (1.5 * 2^23 as an fp32 bit pattern) makes the
+//             combined integer 256 * d_hi + d_lo readable as the float
+//             1.5 * 2^23 + value, exactly, for |value| < 2^22.
+// A token's records for all K follow each other: H / 32 records.
+constexpr int kPlaneRec = 72;
+constexpr int kPlaneMagic = 0x4B400000;
+constexpr float kPlaneMagicF = 12582912.0f;
+
+// floor(log2 m) for a finite m > 0 (subnormals included).
+__device__ __forceinline__ int ilog2f(float m) {
+  int e2;
+  frexpf(m, &e2);
+  return e2 - 1;
+}
+
+// The grid exponent for a largest magnitude m (0 when m == 0): max|v| * 2^e
+// lies in [2^13, 2^14).
+__device__ __forceinline__ int plane_exponent(float m) { return m > 0.f ? 13 - ilog2f(m) : 0; }
+
+// 2^k for |k| <= 126.
+__device__ __forceinline__ float pow2i(int k) { return __int_as_float((k + 127) << 23); }
+
+// 2^e as two factors (each exact for |e| <= 252).
+__device__ __forceinline__ void pow2_split(int e, float& f1, float& f2) {
+  const int a = e / 2;
+  f1 = pow2i(a);
+  f2 = pow2i(e - a);
+}
+
+// Eight values v[0..7] (elements 8c .. 8c+7 of a group) on the grid 2^-e
+// (factors f1 * f2 = 2^e): the lane's 8 bytes of each plane and its partial
+// plane sums.
+__device__ __forceinline__ void planes8(const float (&v)[8], float f1, float f2, uint2& lo, uint2& hi, int& slo,
+                                        int& shi) {
+  int l[8], h[8];
+  slo = 0;
+  shi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int q = __float2int_rn((v[i] * f1) * f2);
+    l[i] = ((q + 128) & 255) - 128;
+    h[i] = (q - l[i]) >> 8;
+    slo += l[i];
+    shi += h[i];
+  }
+  auto pack = [](int a, int b, int c, int d) {
+    return (static_cast<uint32_t>(a) & 0xffu) | ((static_cast<uint32_t>(b) & 0xffu) << 8) |
+           ((static_cast<uint32_t>(c) & 0xffu) << 16) | (static_cast<uint32_t>(d) << 24);
+  };
+  lo = make_uint2(pack(l[0], l[2], l[4], l[6]), pack(l[1], l[3], l[5], l[7]));
+  hi = make_uint2(pack(h[0], h[2], h[4], h[6]), pack(h[1], h[3], h[5], h[7]));
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32,

@@ -49,6 +49,8 @@ constexpr int kFusedCombineMaxT = 4;
 
 struct FfnArgs {
   const uint16_t* xq;        // fragment-ordered expert input [T][H]
+  const uint8_t* xp;         // split-K form: integer planes of the expert input [T][H/32][kPlaneRec]
+  const int32_t* xe;         // split-K form: grid exponent of each token's planes [T]
   uint16_t* hq;              // h, fragment-ordered [P+S*T][I]
   float* ypair;              // y [P+S*T][H]
   float* ypart;              // split-K form: y partials [P+S*T][I/128][H]
@@ -457,21 +459,12 @@ __device__ __forceinline__ void warp_combine_rows(const FfnArgs& a, int rb, int 
   }
 }
 
-// Padded row of one token's 128-element h slice in shared memory (split-K form).
-constexpr int kSkHRow = 128 * 2 + 64;
-
-// Consumers: one tile.  Returns false on a timeout.  HSMEM (gate/up of the
-// split-K form): h of the tile's 128 rows goes to the shared-memory slice
-// buffer `hbuf` ([token][kSkHRow bytes], fragment order) once every consumer
-// warp has released the previous unit's slice (h_free), and is announced on
-// h_ready; nothing is written to global memory.
-template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP, bool HSMEM = false, int BITS = 4>
+// Consumers: one tile.  Returns false on a timeout.
+template <int KC, int NT, int NMAT, bool SINGLE, int NS, int STAGE, int GROUP, int BITS = 4>
 __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, const TileInfo& ti, int K, int R,
                                              uint8_t* smem, float* red, uint64_t* full, uint64_t* empty,
                                              uint64_t* red_full, uint64_t* red_empty, int& s, uint32_t& ph,
-                                             uint32_t& rph, volatile int* abort_flag, int warp, int lane,
-                                             uint16_t* hbuf = nullptr, uint64_t* h_free = nullptr,
-                                             uint64_t* h_ready = nullptr, uint32_t lu = 0) {
+                                             uint32_t& rph, volatile int* abort_flag, int warp, int lane) {
   using C = StageCfg<KC, NT, NMAT, GROUP, BITS>;
   const int rw = warp & (kRowWarps - 1);   // 16-row slice
   const int half = warp / kRowWarps;       // which half of each stage's groups
@@ -599,58 +592,41 @@ __device__ __forceinline__ bool consume_tile(const FfnArgs& a, const Meta& m, co
   mbar_arrive(&red_empty[rw]);
   rph ^= 1u;
   // epilogue: d0 (row g, col 2c), d1 (row g, col 2c+1), d2 (row g+8, col 2c), d3 (row g+8, col 2c+1)
-  if constexpr (HSMEM) {
-    static_assert(NMAT == 2 && NT == 1, "h slices in shared memory are for 8-token gate/up tiles");
-    if (lu > 0 && !mbar_wait(h_free, (lu - 1) & 1u, abort_flag, a.status)) return false;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = 2 * c + (q & 1);
-      if (i < ti.ntok && !(SINGLE && (q & 1))) {
-        const float gv = acc0[0][q], uv = acc1[0][q];
-        const float hv = gv / (1.0f + expf(-gv)) * uv;
-        hbuf[i * (kSkHRow / 2) + frag_pos(rl0 + ((q & 2) ? 8 : 0))] = float_to_bf16_bits(hv);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(h_ready);
-    return true;
-  } else {
-  #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      if (nt < nnt) {
-  #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = ti.i0 + nt * 8 + 2 * c + (q & 1);
-          if (i < ti.cnt && !(SINGLE && (q & 1))) {
-            const size_t orow = static_cast<size_t>(ti.base + i);
-            const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
-            if (NMAT == 2) {
-              const float gv = acc0[nt][q], uv = acc1[nt][q];
-              const float hv = gv / (1.0f + expf(-gv)) * uv;
-              a.hq[orow * R + frag_pos(r)] = float_to_bf16_bits(hv);
-            } else {
-              a.ypair[orow * R + r] = acc0[nt][q];
-            }
+  for (int nt = 0; nt < NT; ++nt) {
+    if (nt < nnt) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = ti.i0 + nt * 8 + 2 * c + (q & 1);
+        if (i < ti.cnt && !(SINGLE && (q & 1))) {
+          const size_t orow = static_cast<size_t>(ti.base + i);
+          const int r = ti.rb * kRowBlock + rl0 + ((q & 2) ? 8 : 0);
+          if (NMAT == 2) {
+            const float gv = acc0[nt][q], uv = acc1[nt][q];
+            const float hv = gv / (1.0f + expf(-gv)) * uv;
+            a.hq[orow * R + frag_pos(r)] = float_to_bf16_bits(hv);
+          } else {
+            a.ypair[orow * R + r] = acc0[nt][q];
           }
         }
       }
     }
-    // publish: every lane's stores, then one increment per warp
-    __threadfence();
-    __syncwarp();
-    if (NMAT == 2) {
-      if (lane == 0) atomicAdd(a.tb_done + ti.tbg, 1);
-    } else if (a.T <= kFusedCombineMaxT) {
-      int old = 0;
-      if (lane == 0) old = atomicAdd(a.rb_done + ti.rb, 1);
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old + 1 == m.total_blocks * kRowWarps) {   // last warp of this row block
-        __threadfence();
-        warp_combine_rows(a, ti.rb, lane);
-      }
-    }
-    return true;
   }
+  // publish: every lane's stores, then one increment per warp
+  __threadfence();
+  __syncwarp();
+  if (NMAT == 2) {
+    if (lane == 0) atomicAdd(a.tb_done + ti.tbg, 1);
+  } else if (a.T <= kFusedCombineMaxT) {
+    int old = 0;
+    if (lane == 0) old = atomicAdd(a.rb_done + ti.rb, 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old + 1 == m.total_blocks * kRowWarps) {   // last warp of this row block
+      __threadfence();
+      warp_combine_rows(a, ti.rb, lane);
+    }
+  }
+  return true;
 }
 
 // The persistent FFN kernel (gate/up tiles, then down tiles).  Launched

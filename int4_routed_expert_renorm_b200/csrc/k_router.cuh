@@ -11,12 +11,74 @@ namespace coli {
 
 constexpr float kRmsEps = 1e-6f;
 
+// Eight consecutive expert-input values of a token from its bf16 row: x, or
+// with pre-norm n = bf16(x * r).
+__device__ __forceinline__ void input8(const uint16_t* __restrict__ xr, int i, int prenorm, float r, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(xr + i);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+  if (prenorm) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = bf16_bits_to_float(float_to_bf16_bits(v[k] * r));
+  }
+}
+
+// Integer planes of one token's expert input (common.cuh): the largest |v|
+// over the row sets the grid exponent (*xe), then the H/32 plane records go
+// to xp_row.  Called by every thread of a block of 256 (H % 256 == 0, so each
+// warp covers whole groups); `mx` is 8 floats of shared memory.
+__device__ __forceinline__ void token_planes(const uint16_t* __restrict__ xr, int H, int prenorm, float r,
+                                             uint8_t* __restrict__ xp_row, int32_t* __restrict__ xe, float* mx) {
+  float m = 0.f;
+  for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+    float v[8];
+    input8(xr, i, prenorm, r, v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();   // mx may still be read from the previous token
+  if ((threadIdx.x & 31) == 0) mx[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, mx[w]);
+  const int e = plane_exponent(m);
+  if (threadIdx.x == 0) *xe = e;
+  float f1, f2;
+  pow2_split(e, f1, f2);
+  const int c = threadIdx.x & 3;
+  for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+    float v[8];
+    input8(xr, i, prenorm, r, v);
+    uint2 lo, hi;
+    int slo, shi;
+    planes8(v, f1, f2, lo, hi, slo, shi);
+    uint8_t* rec = xp_row + static_cast<size_t>(i >> 5) * kPlaneRec;
+    *reinterpret_cast<uint2*>(rec + 8 * c) = lo;
+    *reinterpret_cast<uint2*>(rec + 32 + 8 * c) = hi;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      slo += __shfl_xor_sync(0xffffffffu, slo, o);
+      shi += __shfl_xor_sync(0xffffffffu, shi, o);
+    }
+    if (c == 0) *reinterpret_cast<int2*>(rec + 64) = make_int2(kPlaneMagic - 8 * slo, -8 * shi);
+  }
+}
+
 // One block per token.  Writes the fragment-ordered copy `xq` of the layer's
-// expert input and, with prenorm, the natural-order normalised copy `xn`:
+// expert input, its integer planes `xp` / grid exponents `xe` when xp is not
+// NULL (the split-K decode form), and, with prenorm, the natural-order
+// normalised copy `xn`:
 //   n = bf16( x * (1 / sqrt(mean(x^2) + 1e-6)) ), the sum of squares in fp32
 // in a fixed order.  H % 8 == 0.
 __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int H, int prenorm,
-                                                   uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
+                                                   uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
+                                                   uint8_t* __restrict__ xp, int32_t* __restrict__ xe) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -69,6 +131,10 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
     o.z = e[2] | (static_cast<uint32_t>(e[6]) << 16);
     o.w = e[3] | (static_cast<uint32_t>(e[7]) << 16);
     *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
+  }
+  if (xp) {
+    __shared__ float mx[8];
+    token_planes(xr, H, prenorm, r, xp + static_cast<size_t>(t) * (H / 32) * kPlaneRec, xe + t, mx);
   }
 }
 
@@ -141,14 +207,16 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
 }
 
 // Small-batch front end (T <= 8): router logits, plus
-// the fragment-ordered copy of the expert input written by the blocks whose
-// index matches a token (block b writes tokens b, b + gridDim.x, ...).  With
+// the fragment-ordered copy of the expert input (and, when xp is not NULL, its
+// integer planes and grid exponents) written by the blocks whose index
+// matches a token (block b writes tokens b, b + gridDim.x, ...).  With
 // prenorm every block normalises its tokens itself (n = bf16(x * r) with
 // r = 1/sqrt(mean(x^2) + 1e-6) summed in the same order as prep_kernel), so
 // the logits see exactly the normalised input the experts see.
 __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                                                     int T, int E, int H, int prenorm, float* __restrict__ logits,
-                                                    uint16_t* __restrict__ xn, uint16_t* __restrict__ xq) {
+                                                    uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
+                                                    uint8_t* __restrict__ xp, int32_t* __restrict__ xe) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[8][8];
@@ -222,6 +290,10 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
       o.z = q8[2] | (static_cast<uint32_t>(q8[6]) << 16);
       o.w = q8[3] | (static_cast<uint32_t>(q8[7]) << 16);
       *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
+    }
+    if (xp) {
+      __shared__ float mx[8];
+      token_planes(xr, H, prenorm, r, xp + static_cast<size_t>(t) * (H / 32) * kPlaneRec, xe + t, mx);
     }
   }
   if (!wr) return;

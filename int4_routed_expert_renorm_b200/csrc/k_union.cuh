@@ -422,7 +422,9 @@ __device__ __forceinline__ void warp_bitonic_sort128(int (&key)[4], int lane) {
 }
 
 // ids: T*k routed experts (shared memory); writes the union outputs, the plan
-// and zeroes the FFN counters, like block_union + block_plan.  Called by warp 0.
+// and zeroes the FFN counters (when tb_done / rb_done are not NULL), like
+// block_union + block_plan.  Called by one warp; the outputs may be in global
+// or shared memory.
 __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, int T, int S, int tokb,
                                                 int32_t* __restrict__ unique_ids, int32_t* __restrict__ n_unique,
                                                 int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
@@ -523,8 +525,10 @@ __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, in
     plan[1] = total;
     plan[2 + n_seg] = total;
   }
-  for (int i = lane; i < total; i += 32) tb_done[i] = 0;
-  for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
+  if (tb_done)
+    for (int i = lane; i < total; i += 32) tb_done[i] = 0;
+  if (rb_done)
+    for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
 }
 
 // The same for T*k <= 32, one key per lane: a 32-wide bitonic sort (15
@@ -595,8 +599,10 @@ __device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, 
     plan[1] = total;
     plan[2 + n_seg] = total;
   }
-  for (int i = lane; i < total; i += 32) tb_done[i] = 0;
-  for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
+  if (tb_done)
+    for (int i = lane; i < total; i += 32) tb_done[i] = 0;
+  if (rb_done)
+    for (int i = lane; i < n_rb; i += 32) rb_done[i] = 0;
 }
 
 // Route + union + plan for T*k <= 128: warp w routes tokens w, w + nwarps, ...;

@@ -390,3 +390,58 @@ def test_binding_refuses_host_and_strided_tensors(colimoe):
     bad = dict(t, down_s=torch.zeros(E + S, I // G, H, dtype=torch.int16).transpose(1, 2))
     with pytest.raises(ValueError, match="contiguous"):
         m.MoELayer(d, bad)
+
+
+def test_binding_refuses_tensors_of_the_wrong_size(colimoe):
+    """Every tensor argument must have exactly the elements (and element size)
+    the C call reads or writes through its pointer: a short or mistyped tensor
+    is refused with ValueError before anything reaches the library (these are
+    host tensors, which would be refused later anyway; the size check comes
+    first)."""
+    import torch
+    m = colimoe
+    H, I, E, k, S, T = 256, 256, 8, 2, 1, 3
+    d = m.dims_for(H, I, E, k, S)
+    w = m.coli_moe_weights()
+    x = torch.zeros(T, H, dtype=torch.int16)
+    out = torch.zeros(T, H, dtype=torch.int16)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    good = dict(logits_in=torch.zeros(T, E), residual=torch.zeros(T, H, dtype=torch.int16),
+                logits_out=torch.zeros(T, E), topk_ids_out=torch.zeros(T, k, dtype=torch.int32),
+                topk_w_out=torch.zeros(T, k))
+    bad = dict(logits_in=torch.zeros(T, E - 1), residual=torch.zeros(T - 1, H, dtype=torch.int16),
+               logits_out=torch.zeros(T, E, dtype=torch.float64), topk_ids_out=torch.zeros(T, k + 1, dtype=torch.int32),
+               topk_w_out=torch.zeros(T * k - 1))
+    for name in bad:
+        kw = dict(good, **{name: bad[name]})
+        with pytest.raises(ValueError, match=name):
+            m.coli_moe_layer(d, w, x, out, ws, **kw)
+        with pytest.raises(ValueError, match=name):
+            m.coli_moe_layer_noalloc(d, w, x, out, **kw)
+    with pytest.raises(ValueError, match="x"):
+        m.coli_moe_layer(d, w, torch.zeros(T, H + 8, dtype=torch.int16), out, ws)
+    with pytest.raises(ValueError, match="x"):
+        m.coli_moe_layer(d, w, torch.zeros(T, H, dtype=torch.float32), out, ws)
+    with pytest.raises(ValueError, match="out"):
+        m.coli_moe_layer(d, w, x, torch.zeros(T, H - 1, dtype=torch.int16), ws)
+    # expert FFN: the union arrays
+    P, U = T * k, min(E, T * k)
+    i32 = lambda n: torch.zeros(n, dtype=torch.int32)  # noqa: E731
+    args = dict(topk_ids=i32(P), topk_w=torch.zeros(P), unique_ids=i32(U), n_unique=i32(1), seg_off=i32(U + 1),
+                perm=i32(P), pair_pos=i32(P))
+    for name, short in (("topk_ids", i32(P - 1)), ("topk_w", torch.zeros(P + 1)), ("unique_ids", i32(U - 1)),
+                        ("n_unique", i32(0)), ("seg_off", i32(U)), ("perm", i32(P - 1)), ("pair_pos", i32(P - 1))):
+        a = dict(args, **{name: short})
+        with pytest.raises(ValueError, match=name):
+            m.coli_moe_expert_ffn(d, w, x, a["topk_ids"], a["topk_w"], a["unique_ids"], a["n_unique"],
+                                  a["seg_off"], a["perm"], a["pair_pos"], None, out, ws)
+    # route and union
+    lg, ids, tw = torch.zeros(T, E), torch.zeros(T, k, dtype=torch.int32), torch.zeros(T, k)
+    with pytest.raises(ValueError, match="bias"):
+        m.coli_moe_route(lg, torch.zeros(E - 1), ids, tw)
+    with pytest.raises(ValueError, match="topk_w"):
+        m.coli_moe_route(lg, None, ids, torch.zeros(T, k, dtype=torch.float16))
+    with pytest.raises(ValueError, match="pair_pos"):
+        m.coli_moe_union(ids, E, i32(U), i32(1), i32(U + 1), i32(P), i32(P - 1))
+    with pytest.raises(ValueError, match="seg_off"):
+        m.coli_moe_union(ids, E, i32(U), i32(1), i32(U), i32(P), i32(P))

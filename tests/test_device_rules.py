@@ -33,6 +33,9 @@ def test_no_trap_and_no_device_assert():
 
 
 def test_every_open_loop_checks_the_wait_limit():
+    """An open loop compares %globaltimer with kWaitLimitNs, or with a
+    `limit_ns` parameter of its function (checked below to default to
+    kWaitLimitNs), within a few lines."""
     open_loop = re.compile(r"for\s*\([^;)]*;\s*;[^)]*\)|while\s*\(\s*(true|1)\s*\)|\bdo\s*\{")
     found = 0
     for p in SOURCES:
@@ -41,8 +44,26 @@ def test_every_open_loop_checks_the_wait_limit():
             if open_loop.search(ln):
                 found += 1
                 window = "\n".join(lines[i:i + 12])
-                assert "kWaitLimitNs" in window and "globaltimer()" in window, f"{p}:{i + 1}: {ln.strip()}"
+                assert ("kWaitLimitNs" in window or "limit_ns" in window) and "globaltimer()" in window, \
+                    f"{p}:{i + 1}: {ln.strip()}"
     assert found >= 3      # the mbarrier wait, the token-block counter wait, the grid-wide counter wait
+
+
+def test_wait_limit_parameters_default_to_the_limit():
+    """Every `limit_ns` parameter of a wait routine defaults to kWaitLimitNs,
+    so only a caller that names a limit waits less.  The one caller that does
+    is the timeout test hook's kernel, whose host entry refuses any limit
+    above kWaitLimitNs before launching it."""
+    n = 0
+    for p in SOURCES:
+        code = _code(p)
+        for m in re.finditer(r"(\w+)\s*\(([^()]*?)uint64_t\s+limit_ns\b([^,)]*)", code):
+            if m.group(1) in ("wait_timeout_kernel", "coli_moe_test_wait_timeout"):
+                assert "limit_ns > kWaitLimitNs" in code, p
+                continue
+            n += 1
+            assert m.group(3).replace(" ", "") == "=kWaitLimitNs", f"{p}: {m.group(1)}: limit_ns{m.group(3)}"
+    assert n >= 2
 
 
 def test_while_loops_are_bounded_forms():
