@@ -4,9 +4,8 @@ CPU oracle, through the C ABI.
 The form is forced with COLI_PATH_PREFILL on shapes the oracle computes in
 full: one-stage and multi-stage K, token blocks split near-equally once a
 segment passes 160 tokens, experts with a single token, shared experts,
-residual and pre-norm.  At the full prefill size (4096 tokens, 256 experts)
-sampled tokens are compared with the oracle and every token with the decode
-form, an independent implementation (mma.sync) of the same FFN.
+residual and pre-norm.  The full prefill chunk (4096 tokens, 256 experts) is
+compared with the C oracle on many tokens in ``tests/test_gpu_fullsize.py``.
 """
 import numpy as np
 import pytest
@@ -76,7 +75,7 @@ def test_prefill_form_at_decode_batch_sizes(lib, T):
 
 def test_prefill_and_decode_forms_agree_small(lib):
     """Same routed batch through both forms: identical routing, outputs within
-    twice the layer tolerance of each other (each is within it of the oracle)."""
+    the layer tolerance of each other."""
     shape = _small_shape(tokens=96, hidden=512, inter=256, n_experts=8, n_shared=1)
     layer = device_layer(shape, seed=10)
     li = synth.LayerInputs(shape, seed=10)
@@ -86,7 +85,7 @@ def test_prefill_and_decode_forms_agree_small(lib):
     _, gd = check_layer(lib, shape, layer, W, x, rw=li.router_w(), flags=DECODE)
     assert np.array_equal(gp["ids"], gd["ids"])
     a, b = oracle.bf16_bits_to_f64(gp["out"]), oracle.bf16_bits_to_f64(gd["out"])
-    assert np.abs(a - b).max() <= 2 * OUT_REL_TOL * np.abs(b).max()
+    assert np.abs(a - b).max() <= OUT_REL_TOL * np.abs(b).max()
 
 
 @pytest.fixture(scope="module")
@@ -103,21 +102,3 @@ def test_glm_decode_b1_prefill_form(lib, glm_layer_pf):
     err, g = check_layer(lib, shape, glm_layer_pf, oracle_weights(shape), synth.activations(shape),
                          rw=li.router_w(), flags=PREFILL)
     print(f"decode b1 through the prefill form: max rel err {err:.3e}")
-
-
-def test_glm_prefill_4096_forms(lib, glm_layer_pf):
-    """Full prefill chunk: sampled tokens against the oracle (prefill form), and
-    every token of the prefill form against the decode form."""
-    shape = synth.PREFILL_4096
-    li = synth.LayerInputs(shape)
-    x = synth.activations(shape)
-    lg = li.logits()
-    err, gp = check_layer(lib, shape, glm_layer_pf, oracle_weights(shape), x, sample=[0, 5, 1777, 2048, 4095],
-                          logits_in=lg, flags=PREFILL)
-    gd = run_gpu_layer(lib, glm_layer_pf, x, logits_in=lg, flags=DECODE)
-    assert gd["flags"] == 0
-    assert np.array_equal(gp["ids"], gd["ids"])
-    a, b = oracle.bf16_bits_to_f64(gp["out"]), oracle.bf16_bits_to_f64(gd["out"])
-    diff = np.abs(a - b).max() / np.abs(b).max()
-    print(f"prefill 4096: sampled max rel err {err:.3e}; prefill vs decode form over all tokens {diff:.3e}")
-    assert diff <= 2 * OUT_REL_TOL

@@ -5,13 +5,12 @@ Every layer is checked on the GPU's own hidden state: the oracle normalises
 it, routes from its own logits and runs the layer, and the GPU layer output
 must match within the layer tolerance (routing bit-exact outside near-ties).
 On the reduced shape the oracle also runs the whole chain from the same
-input, and the final hidden states are compared.  At the GLM-5.2 shape the
-first and last layers are checked (the oracle materialises every expert a
-batch touches in float64).
+input, and the final hidden states are compared, within the same 1e-2 of the
+largest magnitude.  Every layer of the GLM-5.2-shaped stack is checked in
+``tests/test_gpu_fullsize.py``.
 """
 import numpy as np
 import pytest
-import torch
 
 import oracle
 import synth
@@ -41,26 +40,4 @@ def test_stack16_reduced_shape(lib):
     err = np.abs(got - want).max() / np.abs(want).max()
     print(f"stack of {L} (reduced shape): final hidden state max rel err {err:.3e}")
     assert np.isfinite(got).all()
-    assert err <= 2 * OUT_REL_TOL
-
-
-def test_stack16_glm_first_and_last_layer(lib):
-    shape = synth.STACK16_B4
-    h0 = synth.activations(shape)
-    h = h0
-    for l in range(shape.layers):
-        layer = device_layer(shape, seed=0, layer=l)
-        li = synth.LayerInputs(shape, 0, l)
-        if l in (0, shape.layers - 1):
-            err, g = check_layer(lib, shape, layer, oracle_weights(shape, seed=0, layer=l), h, rw=li.router_w(),
-                                 residual_bits=h, flags=PRENORM, max_ambiguous=1)
-            print(f"stack layer {l}: max rel err {err:.3e}")
-            h = g["out"]
-        else:
-            x = torch.from_numpy(np.ascontiguousarray(h).view(np.int16)).cuda()
-            out = torch.empty_like(x)
-            layer.forward(x, out, layer.workspace(x.shape[0]), residual=x, flags=PRENORM)
-            h = out.cpu().numpy().view(np.uint16)
-        del layer
-        torch.cuda.empty_cache()
-    assert np.isfinite(oracle.bf16_bits_to_f64(h)).all()
+    assert err <= OUT_REL_TOL

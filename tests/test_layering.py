@@ -41,8 +41,14 @@ def test_product_python_never_imports_the_oracle():
 
 
 def test_bench_imports_the_oracle_only_in_its_cpu_leg():
+    """bench.py imports the oracle only in the functions of its CPU leg:
+    oracle_sample and the per-process worker it runs, _oracle_tokens."""
     found = _oracle_imports(_parse(os.path.join(ROOT, "bench.py")))
-    assert found and all(fn == "oracle_sample" for _, fn in found)
+    assert found and all(fn in ("oracle_sample", "_oracle_tokens") for _, fn in found)
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    # every use of the worker besides its definition lies inside oracle_sample
+    assert src.count("_oracle_tokens") == len(re.findall(r"_oracle_tokens", src[src.index("def oracle_sample"):
+                                                                             src.index("def rank_batches")])) + 1
 
 
 def test_entry_imports_the_oracle_only_to_build_it_and_in_smoke():

@@ -6,8 +6,11 @@ owns every device allocation, or a real-time loop whose memory is fixed up
 front.  It uses scratch that the library keeps in device memory instead of a
 caller workspace.  These tests call it through the C ABI twice in a row, with
 different inputs, and compare each result with coli_moe_layer's on the same
-inputs, within the layer's output tolerance (the two run the same kernels,
-so the outputs are in fact identical).  This file is collected last.
+inputs: within the layer's output tolerance, and bit for bit, since the two
+run the same kernels on the same data and scratch left over from an earlier
+call must change nothing.  A third call with a larger batch, which takes
+another FFN form, checks the same after the shared scratch was last used by
+a different form.  This file is collected last.
 """
 import numpy as np
 import pytest
@@ -44,11 +47,13 @@ def test_noalloc_matches_workspace_call_glm_decode():
     import int4_routed_expert_renorm_b200 as m
     shape = synth.DECODE_B1
     layer = device_layer(shape)
-    for batch in (0, 1):                       # two calls in a row
-        x = synth.activations(shape, 0, batch)
+    # two batch-1 calls in a row (split-K form), then 9 tokens (two-phase form)
+    for batch, T in ((0, 1), (1, 1), (2, 9)):
+        x = np.concatenate([synth.activations(shape, 0, 10 * batch + t) for t in range(T)])
         o_ws, o_na, i_ws, i_na = _both(m, layer, x)
         assert np.array_equal(i_ws, i_na)
         assert _close(o_ws, o_na)
+        assert np.array_equal(o_ws, o_na)
     del layer
     torch.cuda.empty_cache()
 
@@ -57,11 +62,12 @@ def test_noalloc_matches_workspace_call_prenorm_residual():
     import int4_routed_expert_renorm_b200 as m
     shape = synth.LayerShape("small", 256, 128, 16, 2, 1, 5)
     layer = device_layer(shape, seed=7)
-    for batch in (0, 1):
-        x = synth.normal_bf16(7, batch, synth.X_IN, (5, 256))
+    for batch, T in ((0, 5), (1, 5), (2, 40)):
+        x = synth.normal_bf16(7, batch, synth.X_IN, (T, 256))
         o_ws, o_na, i_ws, i_na = _both(m, layer, x, residual_bits=x, flags=m._lib.COLI_LAYER_PRENORM)
         assert np.array_equal(i_ws, i_na)
         assert _close(o_ws, o_na)
+        assert np.array_equal(o_ws, o_na)
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
