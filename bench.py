@@ -156,48 +156,98 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the oracle leg (CPU)
 
-def oracle_sample(shape: synth.LayerShape, seconds: float):
-    """Time the CPU oracle, as it stands, on a bounded sample of the workload.
+_KINDS = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
 
-    Weights of the experts the sample touches are generated beforehand (not
-    timed); the timed call is oracle.moe_layer (logits, route, union, FFN,
-    combine).  Returns (tokens/s, cores, description)."""
-    import oracle
-    from threadpoolctl import threadpool_limits
+
+def _oracle_tokens(name: str, batch: int, toks: list[int]) -> tuple[float, int]:
+    """Time the plain-C oracle (oracle/c/moe_ref.c, -O2, one thread) on tokens
+    `toks` of input batch `batch` of a workload, one token per call, each on
+    the first layer of the workload: the weights of the experts a token
+    selects are generated beforehand (untimed); the timed call is the C
+    oracle's whole layer (logits or given logits, route, union, expert FFN,
+    combine; pre-norm for the stack).  Returns (seconds, calls)."""
+    import oracle.cref as cr
+    cr.build()
+    shape = synth.WORKLOADS[name]
     li = synth.LayerInputs(shape, 0, 0)
     rw = None if shape.logits_in else li.router_w()
     bias = li.bias()
-    per_tok = 1 if shape.tokens == 1 else 4
-    layers_timed = 1
-    scale = shape.layers  # the stack: one layer is timed and the time is scaled by the layer count
-    tok_done, elapsed, batches = 0, 0.0, 0
-    with threadpool_limits(1):
-        while elapsed < seconds and batches < 8:
-            x = synth.activations(shape, 0, batches)[:per_tok]
-            lg = None
-            if shape.logits_in:
-                lg = synth.normal_f32(0, 1000 + batches, synth.LOGITS_IN, (shape.tokens, shape.n_experts), 1.0)[:per_tok]
-            # pre-generate the touched experts' codes/scales (untimed)
-            lpre = lg if lg is not None else oracle.router_logits(x if not shape.prenorm else oracle.rms_norm(x), rw)[1]
-            ids, _, _ = oracle.route(oracle.add_bias(lpre, bias), shape.top_k)
-            need = sorted(set(ids.ravel().tolist()) | set(range(shape.n_experts, shape.n_total)))
-            kinds = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
-            pre = {(k, e): (li.expert_codes(q, e), li.expert_scales(s, e)) for k, (q, s) in kinds.items() for e in need}
-            W = oracle.ExpertWeights(lambda k, e: pre[(k, e)][0], lambda k, e: pre[(k, e)][1], shape.group,
-                                     bits=shape.bits)
-            xin = x
-            t0 = time.perf_counter()
-            if shape.prenorm:
-                xin = oracle.rms_norm(x)
-            oracle.moe_layer(W, xin, shape.n_experts, shape.top_k, shape.n_shared, router_w=rw, bias=bias,
-                             logits_in=lg, residual_bits=x if shape.prenorm else None)
-            elapsed += (time.perf_counter() - t0) * scale * layers_timed
-            tok_done += x.shape[0]
-            batches += 1
-    desc = (f"{batches} batches x {per_tok} token(s) of {shape.name}"
-            + (f"; one layer timed, x{shape.layers} for the stack" if shape.layers > 1 else "")
-            + "; numpy float64, BLAS limited to 1 thread; touched experts' weights generated untimed")
-    return tok_done / elapsed, 1, desc
+    x = synth.activations(shape, 0, batch)
+    lg = None
+    if shape.logits_in:
+        lg = synth.normal_f32(0, 1000 + batch, synth.LOGITS_IN, (shape.tokens, shape.n_experts), 1.0)
+    elapsed = 0.0
+    for t in toks:
+        xt = x[t:t + 1]
+        xin = cr.rms_norm(xt) if shape.prenorm else xt
+        lt = None if lg is None else lg[t:t + 1]
+        l32 = lt if lt is not None else cr.router_logits(xin, rw)[1]
+        ids = cr.route(l32, shape.top_k, bias)[0]
+        need = sorted(set(ids.ravel().tolist()) | set(range(shape.n_experts, shape.n_total)))
+        held = {(kind, e): (li.expert_codes(q, e), li.expert_scales(sc, e)) for kind, (q, sc) in _KINDS.items()
+                for e in need}
+        t0 = time.perf_counter()
+        xin = cr.rms_norm(xt) if shape.prenorm else xt
+        cr.moe_layer_experts(lambda kind, e: held[(kind, e)], shape.hidden, shape.inter, xin, shape.n_experts,
+                             shape.top_k, shape.n_shared, shape.group, shape.bits, router_w=rw, bias=bias,
+                             logits_in=lt, residual_bits=xt if shape.prenorm else None, experts=need)
+        elapsed += time.perf_counter() - t0
+    return elapsed, len(toks)
+
+
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample(shape: synth.LayerShape, seconds: float):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload.
+
+    The plain-C oracle, one token per call.  Decode and stack workloads: one
+    core, tokens taken in turn from the rotating input batches until about
+    `seconds` of oracle time.  Prefill workloads (thousands of tokens): one
+    process per host core (spawned, so no CUDA state is inherited), each
+    timing its own share of tokens; throughput = all tokens over the longest
+    worker's oracle time.  The stack times one layer per token and scales by
+    the layer count.  Returns (tokens/s, cores, calls, description)."""
+    per_call = 4.0 if shape.hidden >= 4096 else 0.001      # rough C-oracle seconds per token (GLM shape)
+    ncores = os.cpu_count() or 1
+    parallel = shape.tokens >= 512 and ncores > 1
+    if not parallel:
+        n = max(1, min(64, int(seconds / per_call)))
+        toks = [(i // shape.tokens, i % shape.tokens) for i in range(n)]   # (batch, token) in turn
+        if shape.tokens > 1:     # spread the sample over the batch's tokens
+            step = max(1, shape.tokens // max(1, n))
+            toks = [(i // shape.tokens, (i * step) % shape.tokens) for i in range(n)]
+        el, calls = 0.0, 0
+        for b in sorted({bt for bt, _ in toks}):
+            e, c = _oracle_tokens(shape.name, b, [t for bb, t in toks if bb == b])
+            el += e
+            calls += c
+        el *= shape.layers
+        cores = 1
+        desc = (f"{calls} calls of 1 token each of {shape.name} (rotating input batches); plain C oracle "
+                f"(gcc -O2, -ffp-contract=off), 1 thread")
+    else:
+        import multiprocessing as mp
+        per_worker = max(1, int(seconds / per_call))
+        tok_lists = [[(w * per_worker + i) * 131 % shape.tokens for i in range(per_worker)] for w in range(ncores)]
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(ncores) as pool:
+            res = pool.starmap(_oracle_tokens, [(shape.name, 0, tl) for tl in tok_lists])
+        el = max(e for e, _ in res)
+        calls = sum(c for _, c in res)
+        cores = ncores
+        desc = (f"{calls} calls of 1 token each of {shape.name}, {per_worker} per process on {ncores} processes "
+                f"(spawned), throughput = tokens / longest process; plain C oracle (gcc -O2, -ffp-contract=off)")
+    desc += (f"{'; one layer timed, x' + str(shape.layers) + ' for the stack' if shape.layers > 1 else ''}"
+             f"; touched experts' weights generated untimed; host: {ncores} cores, {cpu_model()}")
+    return calls / el, cores, calls, desc
 
 
 # ---- replicas over ranks (the path has no exchange step) -------------------
@@ -224,18 +274,26 @@ def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> f
     return world * tokens_per_step * steps / (ms / 1e3)
 
 
+def workload_config(shape, rotating: int) -> dict:
+    """The `config` of both arms' bench lines: the workload and how it was fed."""
+    return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "inter": shape.inter,
+            "experts": shape.n_experts, "top_k": shape.top_k, "shared": shape.n_shared, "layers": shape.layers,
+            "group": shape.group, "code_bits": shape.bits, "rotating_batches": rotating,
+            "l2": "GPU arm: L2 flushed before every step (256 MiB write, then 256 MiB read), outside the timed events"}
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     shape = synth.WORKLOADS[a.workload]
-    v, cores, desc = oracle_sample(shape, max(5.0, a.cpu_seconds))
-    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": shape.tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
+    v, cores, calls, desc = oracle_sample(shape, max(5.0, a.cpu_seconds))
+    # a step here is one timed oracle call (one token; for the stack, one
+    # token through all layers)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus, "steps": calls, "warmup": 0,
+            "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden,
-                       "inter": shape.inter, "experts": shape.n_experts, "top_k": shape.top_k,
-                       "shared": shape.n_shared, "layers": shape.layers},
+            "config": workload_config(shape, a.batches),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -491,27 +549,34 @@ def main():
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e):
             e2e_step(0)
-    for i in range(K2):
-        bi = i % NB
-        flush_l2()
-        es[i].record()
-        xd.copy_(xh[bi], non_blocking=True)
-        if ld is not None:
-            ld.copy_(lh[bi], non_blocking=True)
-        if g_e2e is not None:
-            g_e2e.replay()
-        else:
-            e2e_step(bi)
-        oh.copy_(od, non_blocking=True)
-        ee[i].record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(es[i].elapsed_time(ee[i]) for i in range(K2)), world, "cuda")
-    e2e = {"value": job_throughput(world, T, K2, e2e_ms), "unit": UNIT,
-           "h2d_bytes_per_step": T * H * 2 + (T * E * 4 if shape.logits_in else 0), "d2h_bytes_per_step": T * H * 2}
+    def e2e_run(graph):
+        for i in range(K2):
+            bi = i % NB
+            flush_l2()
+            es[i].record()
+            xd.copy_(xh[bi], non_blocking=True)
+            if ld is not None:
+                ld.copy_(lh[bi], non_blocking=True)
+            if graph is not None:
+                graph.replay()
+            else:
+                e2e_step(bi)
+            oh.copy_(od, non_blocking=True)
+            ee[i].record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(sum(es[i].elapsed_time(ee[i]) for i in range(K2)), world, "cuda")
+        return job_throughput(world, T, K2, ms)
+
+    io = {"h2d_bytes_per_step": T * H * 2 + (T * E * 4 if shape.logits_in else 0), "d2h_bytes_per_step": T * H * 2}
+    e2e = {"value": e2e_run(g_e2e), "unit": UNIT, **io,
+           "how": "CUDA graph of the layer call(s) replayed each step" if g_e2e is not None else "eager calls"}
+    # the same through eager calls: the host side of every call (argument
+    # checks, tensor-map encoding, launches) inside the timed region
+    e2e_eager = {"value": e2e_run(None), "unit": UNIT, **io, "how": "eager calls"} if g_e2e is not None else None
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        v, cores, desc = oracle_sample(shape, a.cpu_seconds)
+        v, cores, calls, desc = oracle_sample(shape, a.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
@@ -519,13 +584,10 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": a.warmup,
             "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "ffn_form": form, "cuda_graph": use_graph,
-            "config": {"workload": shape.name, "tokens": T, "hidden": H, "inter": I, "experts": E, "top_k": k,
-                       "shared": S, "layers": shape.layers, "union_per_batch": U,
-                       "union_per_layer": u_stack or None, "l2": "flushed before every step (256 MiB write, then 256 MiB read), outside the timed events",
-                       "rotating_batches": NB},
+            "config": workload_config(shape, NB), "union_per_batch": U, "union_per_layer": u_stack or None,
             "int4_bytes_per_step": bytes_step, "int4_gbs": int4_gbs, "int4_frac_of_hbm": int4_gbs / hbm,
             "roofline": roof, "stage_ms": stage_ms,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "cpu_baseline": cpu, "e2e": e2e, "e2e_eager": e2e_eager, "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
