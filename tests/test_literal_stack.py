@@ -1,4 +1,4 @@
-"""Why the 16-layer stack carries a pre-norm (DESIGN reading R8), pinned.
+"""Why the 16-layer stack carries a weightless pre-norm, pinned.
 
 Taken literally -- h_{l+1} = bf16(h_l + MoE_l(h_l)), with no normalisation --
 the stack of GLM-shaped layers with the stated weight and input
