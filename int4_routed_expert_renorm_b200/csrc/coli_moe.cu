@@ -119,13 +119,13 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_SMEM(2, false, 256, 64)
     COLI_SET_SMEM(4, false, 256, 64)
 #undef COLI_SET_SMEM
-#define COLI_SET_PF_SMEM(NMAT, GR)                                                                      \
-  ok &= cudaFuncSetAttribute(ffn_prefill_kernel<NMAT, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define COLI_SET_PF_SMEM(NMAT, GR, DN)                                                                      \
+  ok &= cudaFuncSetAttribute(ffn_prefill_kernel<NMAT, GR, DN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(PfCfg<NMAT>::SMEM)) == cudaSuccess;
-    COLI_SET_PF_SMEM(2, 32)
-    COLI_SET_PF_SMEM(1, 32)
-    COLI_SET_PF_SMEM(2, 64)
-    COLI_SET_PF_SMEM(1, 64)
+    COLI_SET_PF_SMEM(2, 32, false)
+    COLI_SET_PF_SMEM(2, 32, true)
+    COLI_SET_PF_SMEM(2, 64, false)
+    COLI_SET_PF_SMEM(2, 64, true)
 #undef COLI_SET_PF_SMEM
 #define COLI_SET_SK_SMEM(NT, GR, B)                                                                        \
   ok &= cudaFuncSetAttribute(ffn_splitk_kernel<NT, GR, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -496,7 +496,7 @@ bool pf_weight_maps(const uint8_t* q, const uint16_t* s, uint64_t rows_total, in
                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int NMAT, int GR>
+template <int NMAT, int GR, bool DN>
 bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -509,7 +509,7 @@ bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ++t_launches;
-  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT, GR>, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a) ==
+  return cudaLaunchKernelEx(&cfg, ffn_prefill_kernel<NMAT, GR, DN>, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a) ==
          cudaSuccess;
 }
 
@@ -574,14 +574,15 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   };
   a.s0 = w->gate_s;
   a.s1 = w->up_s;
-  if (!(G == 32 ? launch_prefill<2, 32>(mg, a, grid_for(I / kRowBlock), st)
-                : launch_prefill<2, 64>(mg, a, grid_for(I / kRowBlock), st)))
+  if (!(G == 32 ? launch_prefill<2, 32, false>(mg, a, grid_for(I / kRowBlock), st)
+                : launch_prefill<2, 64, false>(mg, a, grid_for(I / kRowBlock), st)))
     return COLI_ERR_CUDA;
   rec.mark(6);
   a.s0 = w->down_s;
   a.s1 = w->down_s;
-  if (!(G == 32 ? launch_prefill<1, 32>(md, a, grid_for(H / kRowBlock), st)
-                : launch_prefill<1, 64>(md, a, grid_for(H / kRowBlock), st)))
+  // two 128-row blocks of W_down per tile (H is a multiple of 256)
+  if (!(G == 32 ? launch_prefill<2, 32, true>(md, a, grid_for(H / (2 * kRowBlock)), st)
+                : launch_prefill<2, 64, true>(md, a, grid_for(H / (2 * kRowBlock)), st)))
     return COLI_ERR_CUDA;
   rec.mark(7);
   {
@@ -887,7 +888,7 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   const bool fused_front = T <= 8;
   if (fused_front) {
     const float* wr = logits_in ? nullptr : w->router_w;
-    const int grid = logits_in ? T : E;
+    const int grid = (logits_in ? 0 : E) + T;
     if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq,
                 lay.xp, lay.xe))
       return COLI_ERR_CUDA;

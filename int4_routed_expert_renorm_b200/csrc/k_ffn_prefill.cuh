@@ -19,6 +19,11 @@
 //     releases A buffers and token stages with tcgen05.commit;
 //   * the same 16 warps read the accumulators back (tcgen05.ld) and write
 //     h = bf16(silu(g) * u) (gate/up launch) or y in fp32 (down launch).
+// A tile of the gate/up launch holds the same 128 rows of both matrices; a
+// tile of the down launch holds two neighbouring 128-row blocks of W_down.
+// Either way two weight blocks share each token tile, which halves the
+// token-tile traffic per MMA (one block per tile would need ~60 B/cycle of
+// TMA per SM for a 160-token tile, above what the TMA engine delivers).
 // The activations are gathered into pair order first, so a token tile is a
 // plain row range of a 2-D tensor map.  Both operands use the same
 // permutation of K inside every 8-element block (x0 x4 x1 x5 ...), which
@@ -50,8 +55,9 @@ struct PfArgs {
   int H, I, T, k, E, S, P;
 };
 
-// Shared-memory / TMEM plan of one launch.  NMAT = 2: gate and up share the
-// token tile; NMAT = 1: down.
+// Shared-memory / TMEM plan of one launch.  NMAT weight blocks per tile share
+// the token tile: gate and up, or two row blocks of down (NMAT = 1: one down
+// row block).
 template <int NMAT>
 struct PfCfg {
   static constexpr int CODE_SLOT = kRowBlock * 128;                 // codes of one matrix, 4 chunks
@@ -166,7 +172,7 @@ struct PfTile {
 
 // Tile t of a launch with `mb` row blocks.  plan/unique/seg_off are the
 // shared-memory copies.
-template <int NMAT>
+template <bool DOWN>
 __device__ __forceinline__ PfTile pf_decode(const PfArgs& a, const int32_t* blk_off, int n_seg, const int32_t* uniq,
                                             const int32_t* seg, int U, int mb, int t) {
   PfTile ti;
@@ -188,7 +194,7 @@ __device__ __forceinline__ PfTile pf_decode(const PfArgs& a, const int32_t* blk_
     ti.e = a.E + (lo - U);
     cnt = a.T;
     obase = a.P + (lo - U) * a.T;
-    sbase = NMAT == 2 ? a.P : obase;   // every shared segment reads the token-order rows
+    sbase = DOWN ? obase : a.P;   // gate/up: every shared segment reads the token-order rows
   }
   const int start = static_cast<int>(static_cast<int64_t>(cnt) * j / nb);
   const int end = static_cast<int>(static_cast<int64_t>(cnt) * (j + 1) / nb);
@@ -256,7 +262,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // one per 32-wide K half.  GROUP 64: one scale per chunk; a stage's 4 scales
 // are half of a 16-byte box of 8 (the scale map's box), so two consecutive
 // stages load the same box and each reads its own half (K a multiple of 512).
-template <int NMAT, int GROUP>
+// DOWN: the down projection (NMAT row blocks of W_down per tile, y out);
+// otherwise gate/up (NMAT = 2, h out).
+template <int NMAT, int GROUP, bool DOWN>
 __global__ void __launch_bounds__(kPfThreads, 1)
     ffn_prefill_kernel(const __grid_constant__ CUtensorMap mq0, const __grid_constant__ CUtensorMap mq1,
                        const __grid_constant__ CUtensorMap ms0, const __grid_constant__ CUtensorMap ms1,
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&mq0);
-    if (NMAT == 2) prefetch_tensormap(&mq1);
+    if (NMAT == 2 && !DOWN) prefetch_tensormap(&mq1);
   }
   if (warp == 2 && lane == 0) {
     prefetch_tensormap(&mb128);
@@ -328,9 +336,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  const int K = NMAT == 2 ? a.H : a.I;
-  const int R = NMAT == 2 ? a.I : a.H;
-  const int mbk = R / kRowBlock;
+  const int K = DOWN ? a.I : a.H;
+  const int R = DOWN ? a.H : a.I;
+  constexpr int ROWS = DOWN ? NMAT * kRowBlock : kRowBlock;   // weight rows a tile spans
+  const int mbk = R / ROWS;
   const int nk = K / 64;
   const int cps = (K % 256 == 0) ? 4 : 2;            // 64-wide chunks per code stage
   const bool one_stage = GROUP == 32 && (K == cps * 64);   // scales then move by one 1-D copy
@@ -344,25 +353,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t cst = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
-        const int row0 = ti.e * R + ti.rblk * kRowBlock;
+        const PfTile ti = pf_decode<DOWN>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
+        const int row0 = ti.e * R + ti.rblk * ROWS;
+        // weight block m: gate / up rows row0 (maps 0 / 1), or down rows row0 + 128 m (map 0)
+        const int row1 = DOWN ? row0 + kRowBlock : row0;
+        const CUtensorMap* q1 = DOWN ? &mq0 : &mq1;
+        const CUtensorMap* s1 = DOWN ? &ms0 : &ms1;
+        const uint16_t* s1p = DOWN ? a.s0 : a.s1;
         for (int kb = 0; ok && kb < nk; kb += cps) {
           const int cs = static_cast<int>(cst % C::NSC);
           if (!(ok = mbar_wait(&code_empty[cs], ((cst / C::NSC) & 1u) ^ 1u, abort_flag, a.status))) break;
           uint8_t* dst = cst_base + cs * C::CSTAGE;
           mbar_arrive_expect_tx(&code_full[cs], NMAT * kRowBlock * cps * 36);
           tma_load_2d(dst, &mq0, &code_full[cs], kb * 32, row0);
-          if (NMAT == 2) tma_load_2d(dst + C::CODE_SLOT, &mq1, &code_full[cs], kb * 32, row0);
+          if (NMAT == 2) tma_load_2d(dst + C::CODE_SLOT, q1, &code_full[cs], kb * 32, row1);
           uint8_t* sdst = dst + NMAT * C::CODE_SLOT;
           if (one_stage) {
             bulk_load(sdst, a.s0 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4, &code_full[cs]);
             if (NMAT == 2)
-              bulk_load(sdst + C::SC_SLOT, a.s1 + static_cast<size_t>(row0) * (K / 32), kRowBlock * cps * 4,
+              bulk_load(sdst + C::SC_SLOT, s1p + static_cast<size_t>(row1) * (K / 32), kRowBlock * cps * 4,
                         &code_full[cs]);
           } else {
             const int sx = GROUP == 32 ? kb * 2 : (kb & ~7);
             tma_load_2d(sdst, &ms0, &code_full[cs], sx, row0);
-            if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, &ms1, &code_full[cs], sx, row0);
+            if (NMAT == 2) tma_load_2d(sdst + C::SC_SLOT, s1, &code_full[cs], sx, row1);
           }
           ++cst;
         }
@@ -381,7 +395,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t bit = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
+        const PfTile ti = pf_decode<DOWN>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
         for (int kb = 0; ok && kb < nk; ++kb) {
           const int s = static_cast<int>(bit % C::NSB);
           if (!(ok = mbar_wait(&slot_empty[s], ((bit / C::NSB) & 1u) ^ 1u, abort_flag, a.status))) break;
@@ -411,7 +425,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t it = 0, bit = 0, tt = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
+        const PfTile ti = pf_decode<DOWN>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
         const uint32_t idesc = idesc_bf16_m128(ti.npad);
         const int ab = static_cast<int>(tt % C::ACC_BUFS);
         const uint32_t dbase = tbase + ab * NMAT * kPfMaxN;
@@ -466,7 +480,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!warp_wait(&acc_full[ab], (ett / C::ACC_BUFS) & 1u, abort_flag, a.status)) return false;
       tc_fence_after();
       const uint32_t dbase = tbase + lane_bits + ab * NMAT * kPfMaxN;
-      const int grow = et.rblk * kRowBlock + r;     // output row within the expert
+      const int grow = et.rblk * ROWS + r;          // output row within the expert (weight block 0)
       const int hpos = frag_pos(grow);
       for (int c8 = dw >> 2; c8 < (et.npad >> 3); c8 += kPfDqWarps / 4) {
         uint32_t d0[8], d1[8];
@@ -477,12 +491,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int n = 0; n < 8; ++n) {
           const int i = c8 * 8 + n;
           if (i < et.ntok) {
-            if (NMAT == 2) {
+            if (!DOWN) {
               const float gv = __uint_as_float(d0[n]), uv = __uint_as_float(d1[n]);
               const float hv = gv / (1.0f + expf(-gv)) * uv;
               a.hq[static_cast<size_t>(et.orow + i) * a.I + hpos] = float_to_bf16_bits(hv);
             } else {
-              a.ypair[static_cast<size_t>(et.orow + i) * a.H + grow] = __uint_as_float(d0[n]);
+              float* yrow = a.ypair + static_cast<size_t>(et.orow + i) * a.H + grow;
+              yrow[0] = __uint_as_float(d0[n]);
+              if (NMAT == 2) yrow[kRowBlock] = __uint_as_float(d1[n]);
             }
           }
         }
@@ -499,7 +515,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     uint32_t pend_tt = 0;
     bool has_pend = false;
     for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-      const PfTile ti = pf_decode<NMAT>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
+      const PfTile ti = pf_decode<DOWN>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
       for (int kb = 0; kb < nk; ++kb, ++it) {
         if (C::ACC_BUFS > 1 && has_pend && kb == (kDefer < nk ? kDefer : nk - 1)) {
           if (!(ok = epilogue(pend, pend_tt))) break;

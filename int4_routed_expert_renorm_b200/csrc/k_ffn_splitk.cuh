@@ -610,21 +610,32 @@ __device__ __forceinline__ bool wait_counter(const int32_t* cnt, int target, vol
 // range of output units (token t, 4 rows r..r+3), one unit per warp at a
 // time.  Lane quad q (lanes 4q .. 4q+3) takes pair slot j = j0 + q of the
 // unit's k routed and S shared pairs, 8 slots per round; lane p of the quad
-// adds the slices p, p+4, ... of the pair's I/128 partials in order, the quad
-// adds (p0 + p1) + (p2 + p3); then the routed y's are weighted in slot order,
-// the shared y's and the residual added, and the sum rounded once to bf16.
-// Two rounds' loads are in flight before the first is reduced.  pos_s / w_s:
+// adds the slices p, p+4, p+8, p+12 of the pair's I/128 partials in order,
+// the quad adds (p0 + p1) + (p2 + p3) (with more than 16 slices, each block
+// of 16 so, and the blocks' sums in turn); then the routed y's are weighted
+// in slot order, the shared y's and the residual added, and the sum rounded
+// once to bf16.  Every load of a lane (two slot rounds x four slices) is in
+// flight before the first add: one L2 round trip per unit.  pos_s / w_s:
 // shared-memory copies of pair_pos and topk_w.  No barrier: warps work on
 // different units.
+// dry: one unit per warp from the start of the output, nothing stored.  The
+// code runs once per launch, after the weight stream has evicted it from L2,
+// so its first execution would fetch every instruction from DRAM; a dry pass
+// at the start of the kernel, while the warps wait for their first stage,
+// brings it into the SM's instruction cache (the loads read this workspace's
+// partials, whatever they hold).
 __device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* pos_s, const float* w_s, int warp,
-                                               int lane) {
+                                               int lane, bool dry = false) {
   const int q4 = a.H / 4;
   const long units = static_cast<long>(a.T) * q4;
-  const int u0 = static_cast<int>(units * blockIdx.x / gridDim.x);
-  const int u1 = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
+  const int u0 = dry ? 0 : static_cast<int>(units * blockIdx.x / gridDim.x);
+  const int u1 = dry ? (units < kFfnConsumerWarps ? static_cast<int>(units) : kFfnConsumerWarps)
+                     : static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
   const int nj = a.k + a.S;
   const int nsl = a.I / kRowBlock;
   const int quad = lane >> 2, p = lane & 3;
+  auto f4add = [](float4 x, float4 y) { return make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w); };
+  float4 ysl[2];
   for (int u = u0 + warp; u < u1; u += kFfnConsumerWarps) {
     const int t = u / q4, r = (u - t * q4) * 4;
     // the residual load goes out first and lands while the partials come in
@@ -632,58 +643,77 @@ __device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* 
     if (a.residual && lane == 0) rv = __ldg(reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j0 = 0; j0 < nj; j0 += 16) {
-      float4 y[2];
+      for (int s0 = 0; s0 < nsl; s0 += 16) {
+        // every load of this lane (2 pair slots x 4 slices) goes out before any add
+        float4 v[2][4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = j0 + 8 * h + quad;
-        y[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j < nj) {
-          const int row = j < a.k ? pos_s[t * a.k + j] : a.P + (j - a.k) * a.T + t;
+        for (int h = 0; h < 2; ++h) {
+          const int j = j0 + 8 * h + quad;
+          const int row = j < a.k ? pos_s[t * a.k + (j < nj ? j : 0)] : a.P + (j - a.k) * a.T + t;
           const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
-#pragma unroll 4
-          for (int sl = p; sl < nsl; sl += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * a.H));
-            y[h].x += v.x;
-            y[h].y += v.y;
-            y[h].z += v.z;
-            y[h].w += v.w;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int sl = s0 + p + 4 * i;
+            v[h][i] = (j < nj && sl < nsl)
+                          ? __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * a.H))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
-      }
+        float4 y[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2; ++h) {
+          y[h] = v[h][0];
 #pragma unroll
-        for (int m = 1; m <= 2; m <<= 1) {
-          y[h].x += __shfl_xor_sync(0xffffffffu, y[h].x, m);
-          y[h].y += __shfl_xor_sync(0xffffffffu, y[h].y, m);
-          y[h].z += __shfl_xor_sync(0xffffffffu, y[h].z, m);
-          y[h].w += __shfl_xor_sync(0xffffffffu, y[h].w, m);
+          for (int i = 1; i < 4; ++i) {
+            y[h].x += v[h][i].x;
+            y[h].y += v[h][i].y;
+            y[h].z += v[h][i].z;
+            y[h].w += v[h][i].w;
+          }
+#pragma unroll
+          for (int m = 1; m <= 2; m <<= 1) {
+            y[h].x += __shfl_xor_sync(0xffffffffu, y[h].x, m);
+            y[h].y += __shfl_xor_sync(0xffffffffu, y[h].y, m);
+            y[h].z += __shfl_xor_sync(0xffffffffu, y[h].z, m);
+            y[h].w += __shfl_xor_sync(0xffffffffu, y[h].w, m);
+          }
         }
-        // slot order: the 8 quads of this round, one after another
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = j0 + 8 * h + jj;
-          if (j >= nj) break;
-          float4 yj;
-          yj.x = __shfl_sync(0xffffffffu, y[h].x, 4 * jj);
-          yj.y = __shfl_sync(0xffffffffu, y[h].y, 4 * jj);
-          yj.z = __shfl_sync(0xffffffffu, y[h].z, 4 * jj);
-          yj.w = __shfl_sync(0xffffffffu, y[h].w, 4 * jj);
-          if (j < a.k) {
-            const float w = w_s[t * a.k + j];
-            acc.x = fmaf(w, yj.x, acc.x);
-            acc.y = fmaf(w, yj.y, acc.y);
-            acc.z = fmaf(w, yj.z, acc.z);
-            acc.w = fmaf(w, yj.w, acc.w);
-          } else {
-            acc.x += yj.x;
-            acc.y += yj.y;
-            acc.z += yj.z;
-            acc.w += yj.w;
+        if (s0 + 16 < nsl) {
+          // more than 16 slices: keep this block's sums per slot and go on
+          // (I > 2048; the order stays fixed: slice blocks in turn)
+          for (int h = 0; h < 2; ++h) ysl[h] = s0 == 0 ? y[h] : f4add(ysl[h], y[h]);
+          continue;
+        }
+        if (s0 > 0)
+          for (int h = 0; h < 2; ++h) y[h] = f4add(ysl[h], y[h]);
+        // slot order: the 8 quads of each round, one after another
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = j0 + 8 * h + jj;
+            if (j >= nj) break;
+            float4 yj;
+            yj.x = __shfl_sync(0xffffffffu, y[h].x, 4 * jj);
+            yj.y = __shfl_sync(0xffffffffu, y[h].y, 4 * jj);
+            yj.z = __shfl_sync(0xffffffffu, y[h].z, 4 * jj);
+            yj.w = __shfl_sync(0xffffffffu, y[h].w, 4 * jj);
+            if (j < a.k) {
+              const float w = w_s[t * a.k + j];
+              acc.x = fmaf(w, yj.x, acc.x);
+              acc.y = fmaf(w, yj.y, acc.y);
+              acc.z = fmaf(w, yj.z, acc.z);
+              acc.w = fmaf(w, yj.w, acc.w);
+            } else {
+              acc.x += yj.x;
+              acc.y += yj.y;
+              acc.z += yj.z;
+              acc.w += yj.w;
+            }
           }
         }
       }
     }
-    if (lane == 0) {
+    if (lane == 0 && !dry) {
       if (a.residual) {
         acc.x += __uint_as_float(rv.x << 16);
         acc.y += __uint_as_float(rv.x & 0xffff0000u);
@@ -786,18 +816,20 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   pdl_wait();
   pdl_trigger();
   {
-    const int n_seg = __ldg(a.plan);
-    const int U = __ldg(a.n_unique);
+    // every array in one round of loads, up to its allocated size (the union
+    // of P pairs has at most Umax = min(E, P) experts), not to the sizes the
+    // routing kernel reports, so no load waits on another
     const int P = a.T * a.k;
-    for (int i = threadIdx.x; i < n_seg + 3; i += blockDim.x) mplan[i] = __ldg(a.plan + i);
-    for (int i = threadIdx.x; i < U; i += blockDim.x) muniq[i] = __ldg(a.unique_ids + i);
-    for (int i = threadIdx.x; i <= U; i += blockDim.x) mseg[i] = __ldg(a.seg_off + i);
+    const int Umax = P < a.E ? P : a.E;
+    if (threadIdx.x == 0) *n_unique_s = __ldg(a.n_unique);
+    for (int i = threadIdx.x; i < Umax + a.S + 3; i += blockDim.x) mplan[i] = __ldg(a.plan + i);
+    for (int i = threadIdx.x; i < Umax; i += blockDim.x) muniq[i] = __ldg(a.unique_ids + i);
+    for (int i = threadIdx.x; i <= Umax; i += blockDim.x) mseg[i] = __ldg(a.seg_off + i);
     for (int i = threadIdx.x; i < P; i += blockDim.x) {
       perm_s[i] = __ldg(a.perm + i);
       pos_s[i] = __ldg(a.pair_pos + i);
       w_s[i] = __ldg(a.topk_w + i);
     }
-    if (threadIdx.x == 0) *n_unique_s = U;
   }
   __syncthreads();
   Meta m;
@@ -842,6 +874,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   }
 
   // ---------------- consumers ----------------
+  splitk_combine(a, pos_s, w_s, warp, lane, true);
   int s = 0;
   uint32_t ph = 0, rph = 0, lu = 0;
   for (int t = blockIdx.x; t < m.tiles_gu; t += gridDim.x, ++lu) {

@@ -206,10 +206,11 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
   }
 }
 
-// Small-batch front end (T <= 8): router logits, plus
-// the fragment-ordered copy of the expert input (and, when xp is not NULL, its
-// integer planes and grid exponents) written by the blocks whose index
-// matches a token (block b writes tokens b, b + gridDim.x, ...).  With
+// Small-batch front end (T <= 8), one launch of E + T blocks (T when the
+// logits are given, wr == NULL): block e < E computes the router logits of
+// expert e for every token; block E + t writes token t's fragment-ordered
+// copy of the expert input (and, when xp is not NULL, its integer planes and
+// grid exponent), so that no block does both.  With
 // prenorm every block normalises its tokens itself (n = bf16(x * r) with
 // r = 1/sqrt(mean(x^2) + 1e-6) summed in the same order as prep_kernel), so
 // the logits see exactly the normalised input the experts see.
@@ -219,6 +220,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
                                                     uint8_t* __restrict__ xp, int32_t* __restrict__ xe) {
   pdl_wait();
   pdl_trigger();
+  const int nlog = wr ? E : 0;   // blocks [0, nlog): logits of expert b; then one block per token
   __shared__ float red[8][8];
   __shared__ float rs[64];
   const int e = blockIdx.x;
@@ -261,8 +263,9 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
     }
     __syncthreads();
   }
-  // fragment-ordered (and normalised) copies of this block's tokens
-  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+  // fragment-ordered (and normalised) copy and integer planes of this block's token
+  if (static_cast<int>(blockIdx.x) >= nlog) {
+    const int t = blockIdx.x - nlog;
     const uint16_t* xr = x + static_cast<size_t>(t) * H;
     const float r = prenorm ? rs[t] : 1.0f;
     for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
       token_planes(xr, H, prenorm, r, xp + static_cast<size_t>(t) * (H / 32) * kPlaneRec, xe + t, mx);
     }
   }
-  if (!wr) return;
+  if (static_cast<int>(blockIdx.x) >= nlog) return;
   // logits of expert e for every token, 8 tokens at a time.  Each lane issues
   // all its W_r loads (and a token's x loads) before any arithmetic, so the
   // DRAM round trips overlap instead of following one another.

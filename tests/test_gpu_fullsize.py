@@ -145,3 +145,28 @@ def test_stack16_every_layer_teacher_forced(lib):
     errs = [_rel_err(out, ref) for (_, _, out), ref in zip(per_layer, refs)]
     print("stack 16 x b4, per-layer max rel err: " + " ".join(f"{e:.2e}" for e in errs))
     assert max(errs) <= OUT_REL_TOL
+
+
+def test_prefill_4096_with_router_logits(lib):
+    """The prefill chunk with its router logits computed in the step (the tiled
+    fp32 logits kernel at T = 4096, H = 6144): every logit within the derived
+    fp32 bound of the oracle's float64 value, routing from those logits bit-exact,
+    and 32 tokens of output against the C oracle."""
+    shape = synth.PREFILL_4096_ROUTER
+    li = synth.LayerInputs(shape)
+    rw = li.router_w()
+    x = synth.activations(shape)
+    layer = device_layer(synth.DECODE_B1)          # the same layer's weights and router
+    out, lo, ids = _gpu_layer(lib, layer, x)
+    del layer
+    torch.cuda.empty_cache()
+    l64, _ = oracle.router_logits(x, rw)
+    tol = logits_tol(x, rw)
+    assert np.all(np.abs(lo - l64) <= tol), np.abs(lo - l64).max()
+    assert np.array_equal(ids, oracle.route(lo, shape.top_k)[0])
+    toks = np.unique(np.concatenate([[0, shape.tokens - 1], np.random.default_rng(7).integers(0, shape.tokens, 30)]))
+    ref, _ = layer_outputs(shape, 0, 0, x[toks], lo[toks])
+    err = _rel_err(out[toks], ref)
+    print(f"prefill 4096 with router logits: {len(toks)} tokens, max rel err {err:.3e}, "
+          f"max logit error {np.abs(lo - l64).max():.2e}")
+    assert err <= OUT_REL_TOL
