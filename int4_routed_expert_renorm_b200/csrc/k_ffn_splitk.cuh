@@ -484,7 +484,7 @@ __device__ __forceinline__ bool load_h_planes(const FfnArgs& a, const TileInfo& 
 #pragma unroll
     for (int j = 0; j < kSkHGroups; ++j) {
       hbv[j][nt] = *reinterpret_cast<const uint2*>(hb.hp + (sb * kSkHGroups + j) * kPlaneRec + (g & 1) * 32 + 8 * c);
-      hcv[j][nt] = *reinterpret_cast<const int2*>(hb.hp + (sc * kSkHGroups + j) * kPlaneRec + 64);
+      if (NT == 1) hcv[j][nt] = *reinterpret_cast<const int2*>(hb.hp + (sc * kSkHGroups + j) * kPlaneRec + 64);
     }
     he[nt] = hb.he[sc];
   }
@@ -562,8 +562,12 @@ __device__ __forceinline__ bool consume_down_slice(const FfnArgs& a, const TileI
           for (int nt = 0; nt < NT; ++nt) {
             if (NT == 1 || nt < nnt) {
               int d[4];
-              mma_i8<BITS>(d, fa, hbv[j][nt], BITS == 4 ? hcv[j][nt].x : kPlaneMagic,
-                           BITS == 4 ? hcv[j][nt].y : kPlaneMagic);
+              // two n-tiles: the start values come from the plane records in
+              // shared memory (unchanged until every warp has left this
+              // unit's down stages), which saves 16 registers
+              const int2 cv = NT == 1 ? hcv[j][nt]
+                                      : *reinterpret_cast<const int2*>(hb.hp + ((nt * 4 + c) * kSkHGroups + j) * kPlaneRec + 64);
+              mma_i8<BITS>(d, fa, hbv[j][nt], BITS == 4 ? cv.x : kPlaneMagic, BITS == 4 ? cv.y : kPlaneMagic);
               acc_group<BITS>(acc[nt][0], acc[nt][1], d, s0[j], s1[j]);
             }
           }
@@ -618,19 +622,12 @@ __device__ __forceinline__ bool wait_counter(const int32_t* cnt, int target, vol
 // flight before the first add: one L2 round trip per unit.  pos_s / w_s:
 // shared-memory copies of pair_pos and topk_w.  No barrier: warps work on
 // different units.
-// dry: one unit per warp from the start of the output, nothing stored.  The
-// code runs once per launch, after the weight stream has evicted it from L2,
-// so its first execution would fetch every instruction from DRAM; a dry pass
-// at the start of the kernel, while the warps wait for their first stage,
-// brings it into the SM's instruction cache (the loads read this workspace's
-// partials, whatever they hold).
 __device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* pos_s, const float* w_s, int warp,
-                                               int lane, bool dry = false) {
+                                               int lane) {
   const int q4 = a.H / 4;
   const long units = static_cast<long>(a.T) * q4;
-  const int u0 = dry ? 0 : static_cast<int>(units * blockIdx.x / gridDim.x);
-  const int u1 = dry ? (units < kFfnConsumerWarps ? static_cast<int>(units) : kFfnConsumerWarps)
-                     : static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
+  const int u0 = static_cast<int>(units * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
   const int nj = a.k + a.S;
   const int nsl = a.I / kRowBlock;
   const int quad = lane >> 2, p = lane & 3;
@@ -713,7 +710,7 @@ __device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* 
         }
       }
     }
-    if (lane == 0 && !dry) {
+    if (lane == 0) {
       if (a.residual) {
         acc.x += __uint_as_float(rv.x << 16);
         acc.y += __uint_as_float(rv.x & 0xffff0000u);
@@ -792,7 +789,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   // routing: CTA b < S * I/128 starts with row block b % (I/128) of shared
   // expert E + b / (I/128), for all T tokens.  Those weights are no output of
   // an earlier kernel, so their first stages stream in while the kernel still
-  // waits for the routing.
+  // waits for its inputs.
   int pre = 0;
   const int nrb_gu = a.I / kRowBlock;
   if (warp == kFfnConsumerWarps) {
@@ -874,7 +871,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   }
 
   // ---------------- consumers ----------------
-  splitk_combine(a, pos_s, w_s, warp, lane, true);
   int s = 0;
   uint32_t ph = 0, rph = 0, lu = 0;
   for (int t = blockIdx.x; t < m.tiles_gu; t += gridDim.x, ++lu) {

@@ -58,7 +58,7 @@ __device__ __forceinline__ int block_union(const int32_t* ids, int P, int E, int
     if (e >= 0 && lane == __ffs(peers) - 1) myhist[e] += __popc(peers);
     __syncwarp();
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, COLI_FLAG_BAD_ID);
   __syncthreads();
 
   // per-expert totals and per-(warp, expert) offsets within the expert
@@ -444,7 +444,7 @@ __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, in
       pair_pos[p] = -1;
     }
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, COLI_FLAG_BAD_ID);
   warp_bitonic_sort128(key, lane);
   // segment starts: a valid key whose expert differs from the previous key's
   const int prev_last = __shfl_up_sync(0xffffffffu, key[3], 1);
@@ -548,7 +548,7 @@ __device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, 
     else key = (e << 8) | lane;
     pair_pos[lane] = -1;
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, COLI_FLAG_BAD_ID);
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, COLI_FLAG_BAD_ID);
 #pragma unroll
   for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
