@@ -43,12 +43,11 @@
 //     on a CTA barrier; one thread per CTA then increments a grid counter;
 //     once all CTAs have (a bounded grid-wide wait -- the grid is at most
 //     one CTA per SM and one CTA fills an SM's shared memory, so every CTA is
-//     resident), each CTA combines
-//     a contiguous range of (token, 4 rows), a warp per unit: y of every
-//     routed and shared pair as the sum of its I/128 partials in a fixed
-//     order (four lanes each add every fourth slice in turn, then their sums
-//     pairwise), then the routed y's weighted in slot order, the shared y's
-//     and the residual, rounded once to bf16.
+//     resident), each CTA combines a contiguous range of (token, 4 rows):
+//     y of every routed and shared pair as the sum of its I/128 partials in
+//     slice order (a thread per pair and unit), then the routed y's weighted
+//     in slot order, the shared y's and the residual (a thread per unit),
+//     rounded once to bf16.
 // Every token's arithmetic is the same whatever else is in the batch (its own
 // grid, exact integer products, fixed orders everywhere), so the form is
 // batch-invariant.
@@ -104,6 +103,8 @@ struct SkCfg {
   static_assert(D::CODE % 1024 == 0, "swizzled boxes need 1 KiB alignment");
   static_assert(GU::W_BYTES % 16 == 0 && SLOT % 16 == 0, "bulk copies need 16-byte alignment");
   static_assert(META_BYTES % 16 == 0 && H_BYTES % 16 == 0 && HP_BYTES % 16 == 0, "shared regions stay aligned");
+  // the combine stages its pairs' y (k + S <= 36 per 4-row unit) in the stage ring
+  static_assert(NS * STAGE >= 36 * 16, "combine staging");
 };
 
 // Integer MMA of one 32-wide group: d = A * B + C with C = {c_lo, c_hi} in
@@ -611,106 +612,78 @@ __device__ __forceinline__ bool wait_counter(const int32_t* cnt, int target, vol
 }
 
 // The CTA's share of the output after every partial is in: a contiguous
-// range of output units (token t, 4 rows r..r+3), one unit per warp at a
-// time.  Lane quad q (lanes 4q .. 4q+3) takes pair slot j = j0 + q of the
-// unit's k routed and S shared pairs, 8 slots per round; lane p of the quad
-// adds the slices p, p+4, p+8, p+12 of the pair's I/128 partials in order,
-// the quad adds (p0 + p1) + (p2 + p3) (with more than 16 slices, each block
-// of 16 so, and the blocks' sums in turn); then the routed y's are weighted
-// in slot order, the shared y's and the residual added, and the sum rounded
-// once to bf16.  Every load of a lane (two slot rounds x four slices) is in
-// flight before the first add: one L2 round trip per unit.  pos_s / w_s:
-// shared-memory copies of pair_pos and topk_w.  No barrier: warps work on
-// different units.
-__device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* pos_s, const float* w_s, int warp,
-                                               int lane) {
+// range of output units (token t, 4 rows r..r+3), in chunks that fit the
+// idle stage ring.  Pass 1, one thread per (unit, pair slot j): y of the
+// slot's pair (routed slot j < k, then the shared experts) as the sum of its
+// I/128 partials in slice order, every load in flight before the first add,
+// into the ring.  After a CTA barrier, pass 2, one thread per unit: the
+// routed y's weighted in slot order, then the shared y's and the residual,
+// rounded once to bf16.  pos / w: shared-memory copies of pair_pos and
+// topk_w.  `cbar` (count: consumer warps) separates the passes; returns
+// false on a timeout.
+__device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* pos, const float* w,
+                                               uint8_t* ring, int ring_bytes, uint64_t* cbar, uint32_t& cph,
+                                               volatile int* abort_flag, int warp, int lane) {
+  const int tid = warp * 32 + lane;
+  const int nthr = kFfnConsumerWarps * 32;
   const int q4 = a.H / 4;
   const long units = static_cast<long>(a.T) * q4;
   const int u0 = static_cast<int>(units * blockIdx.x / gridDim.x);
   const int u1 = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
   const int nj = a.k + a.S;
   const int nsl = a.I / kRowBlock;
-  const int quad = lane >> 2, p = lane & 3;
-  auto f4add = [](float4 x, float4 y) { return make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w); };
-  float4 ysl[2];
-  for (int u = u0 + warp; u < u1; u += kFfnConsumerWarps) {
-    const int t = u / q4, r = (u - t * q4) * 4;
-    // the residual load goes out first and lands while the partials come in
-    uint2 rv = make_uint2(0u, 0u);
-    if (a.residual && lane == 0) rv = __ldg(reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < nj; j0 += 16) {
+  const int ch = ring_bytes / (nj * 16);
+  float4* ysum = reinterpret_cast<float4*>(ring);
+  for (int cu = u0; cu < u1; cu += ch) {
+    const int cn = (u1 - cu) < ch ? (u1 - cu) : ch;
+    for (int task = tid; task < cn * nj; task += nthr) {
+      const int ui = task / nj, j = task - ui * nj;
+      const int u = cu + ui;
+      const int t = u / q4, r = (u - t * q4) * 4;
+      const int row = j < a.k ? pos[t * a.k + j] : a.P + (j - a.k) * a.T + t;
+      const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
+      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int s0 = 0; s0 < nsl; s0 += 16) {
-        // every load of this lane (2 pair slots x 4 slices) goes out before any add
-        float4 v[2][4];
+        float4 v[16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int j = j0 + 8 * h + quad;
-          const int row = j < a.k ? pos_s[t * a.k + (j < nj ? j : 0)] : a.P + (j - a.k) * a.T + t;
-          const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
+        for (int i = 0; i < 16; ++i)
+          v[i] = s0 + i < nsl ? __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(s0 + i) * a.H))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int sl = s0 + p + 4 * i;
-            v[h][i] = (j < nj && sl < nsl)
-                          ? __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * a.H))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-        float4 y[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          y[h] = v[h][0];
-#pragma unroll
-          for (int i = 1; i < 4; ++i) {
-            y[h].x += v[h][i].x;
-            y[h].y += v[h][i].y;
-            y[h].z += v[h][i].z;
-            y[h].w += v[h][i].w;
-          }
-#pragma unroll
-          for (int m = 1; m <= 2; m <<= 1) {
-            y[h].x += __shfl_xor_sync(0xffffffffu, y[h].x, m);
-            y[h].y += __shfl_xor_sync(0xffffffffu, y[h].y, m);
-            y[h].z += __shfl_xor_sync(0xffffffffu, y[h].z, m);
-            y[h].w += __shfl_xor_sync(0xffffffffu, y[h].w, m);
-          }
-        }
-        if (s0 + 16 < nsl) {
-          // more than 16 slices: keep this block's sums per slot and go on
-          // (I > 2048; the order stays fixed: slice blocks in turn)
-          for (int h = 0; h < 2; ++h) ysl[h] = s0 == 0 ? y[h] : f4add(ysl[h], y[h]);
-          continue;
-        }
-        if (s0 > 0)
-          for (int h = 0; h < 2; ++h) y[h] = f4add(ysl[h], y[h]);
-        // slot order: the 8 quads of each round, one after another
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = j0 + 8 * h + jj;
-            if (j >= nj) break;
-            float4 yj;
-            yj.x = __shfl_sync(0xffffffffu, y[h].x, 4 * jj);
-            yj.y = __shfl_sync(0xffffffffu, y[h].y, 4 * jj);
-            yj.z = __shfl_sync(0xffffffffu, y[h].z, 4 * jj);
-            yj.w = __shfl_sync(0xffffffffu, y[h].w, 4 * jj);
-            if (j < a.k) {
-              const float w = w_s[t * a.k + j];
-              acc.x = fmaf(w, yj.x, acc.x);
-              acc.y = fmaf(w, yj.y, acc.y);
-              acc.z = fmaf(w, yj.z, acc.z);
-              acc.w = fmaf(w, yj.w, acc.w);
-            } else {
-              acc.x += yj.x;
-              acc.y += yj.y;
-              acc.z += yj.z;
-              acc.w += yj.w;
-            }
-          }
+        for (int i = 0; i < 16; ++i) {
+          y.x += v[i].x;
+          y.y += v[i].y;
+          y.z += v[i].z;
+          y.w += v[i].w;
         }
       }
+      ysum[task] = y;
     }
-    if (lane == 0) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    if (!mbar_wait(cbar, cph, abort_flag, a.status)) return false;
+    cph ^= 1u;
+    for (int ui = tid; ui < cn; ui += nthr) {
+      const int u = cu + ui;
+      const int t = u / q4, r = (u - t * q4) * 4;
+      uint2 rv = make_uint2(0u, 0u);
+      if (a.residual) rv = __ldg(reinterpret_cast<const uint2*>(a.residual + static_cast<size_t>(t) * a.H + r));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < a.k; ++j) {
+        const float wj = w[t * a.k + j];
+        const float4 y = ysum[ui * nj + j];
+        acc.x = fmaf(wj, y.x, acc.x);
+        acc.y = fmaf(wj, y.y, acc.y);
+        acc.z = fmaf(wj, y.z, acc.z);
+        acc.w = fmaf(wj, y.w, acc.w);
+      }
+      for (int s = 0; s < a.S; ++s) {
+        const float4 y = ysum[ui * nj + a.k + s];
+        acc.x += y.x;
+        acc.y += y.y;
+        acc.z += y.z;
+        acc.w += y.w;
+      }
       if (a.residual) {
         acc.x += __uint_as_float(rv.x << 16);
         acc.y += __uint_as_float(rv.x & 0xffff0000u);
@@ -722,7 +695,13 @@ __device__ __forceinline__ void splitk_combine(const FfnArgs& a, const int32_t* 
       o.y = float_to_bf16_bits(acc.z) | (static_cast<uint32_t>(float_to_bf16_bits(acc.w)) << 16);
       *reinterpret_cast<uint2*>(a.out + static_cast<size_t>(t) * a.H + r) = o;
     }
+    // the next chunk overwrites ysum: everyone is done with this one
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    if (!mbar_wait(cbar, cph, abort_flag, a.status)) return false;
+    cph ^= 1u;
   }
+  return true;
 }
 
 // The split-K FFN kernel.  At most one CTA per SM, all resident (the final
@@ -895,7 +874,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     if (wait_counter(a.rb_done, static_cast<int>(gridDim.x), abort_flag, a.status)) mbar_arrive(gbar);
   }
   if (!mbar_wait(gbar, 0, abort_flag, a.status)) return;
-  splitk_combine(a, pos_s, w_s, warp, lane);
+  // (the combine's CTA barriers are cbar's next phases)
+  uint32_t cph = 1;
+  splitk_combine(a, pos_s, w_s, smem, NS * STAGE, cbar, cph, abort_flag, warp, lane);
 }
 
 }  // namespace coli

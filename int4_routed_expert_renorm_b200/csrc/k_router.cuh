@@ -141,11 +141,12 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
 // Router logits l[t,e] = sum_h x[t,h] * W_r[e,h] in fp32, for batches of more
 // than 8 tokens.  Block = 8 warps, 8 experts (one per warp) and up to `tt`
 // tokens whose bf16 rows the block first copies into shared memory (read once
-// per block instead of once per expert).  Lane l of a warp multiplies the
-// elements 4l + 128i .. +3 (i = 0, 1, ...) of its expert's W_r row (float4
-// loads, four in flight) with every token's, in that order, then the lanes
-// are added in a fixed tree: each (token, expert) is summed the same way
-// whatever the batch.  H % 128 == 0; dynamic shared memory tt * H * 2 bytes.
+// per block instead of once per expert).  Each (token, expert) is summed in
+// front_kernel's order, so that a token's logits are the same bits in a batch
+// of any size: H in eight ranges of H/8; in range w, lane l adds the elements
+// w*H/8 + 4l + 128j (j ascending, float4 loads of W_r, four in flight); the
+// lanes of each range are added in a fixed tree, and the eight range sums in
+// turn.  H % 128 == 0; dynamic shared memory tt * H * 2 bytes.
 __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __restrict__ x,
                                                           const float* __restrict__ wr, int T, int E, int H, int tt,
                                                           float* __restrict__ logits) {
@@ -155,14 +156,23 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
   const int t0 = blockIdx.y * tt;
   const int nt = min(tt, T - t0);
   const int e = blockIdx.x * 8 + warp;
-  // the expert's first W_r loads do not depend on the previous kernel
   const float* wrow = wr + static_cast<size_t>(e < E ? e : 0) * H;
-  float4 wq[4];
+  const int hw = H >> 3;                 // one range
+  const int nch = (hw + 511) / 512;      // chunks of four float4 per lane and range
+  const int nall = 8 * nch;
+  // chunk c: range c / nch, this lane's elements h0 + 4 lane + 512 (c % nch) + 128 u
+  auto load_chunk = [&](int c, float4 (&wv)[4]) {
+    const int w8 = c / nch, k = c - w8 * nch;
+    const int h0 = w8 * hw, h1 = h0 + hw;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int h = lane * 4 + u * 128;
-    wq[u] = (e < E && h < H) ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+    for (int u = 0; u < 4; ++u) {
+      const int h = h0 + lane * 4 + 512 * k + 128 * u;
+      wv[u] = (e < E && h < h1) ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // the expert's first W_r loads do not depend on the previous kernel
+  float4 wq[4];
+  load_chunk(0, wq);
   pdl_wait();
   pdl_trigger();
   const int n16 = nt * H / 8;
@@ -170,18 +180,22 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
     xs_raw[i] = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0) * H + static_cast<size_t>(i) * 8);
   __syncthreads();
   if (e >= E) return;
-  float acc[8];
+  float acc[8], tot[8];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-  for (int h0 = 0; h0 < H; h0 += 512) {
+  for (int q = 0; q < 8; ++q) acc[q] = tot[q] = 0.f;
+  for (int c = 0; c < nall; ++c) {
+    const int w8 = c / nch, k = c - w8 * nch;
+    const int h0 = w8 * hw, h1 = h0 + hw;
+    float4 cur[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) cur[u] = wq[u];
+    // the next chunk's loads go out before this chunk's arithmetic
+    if (c + 1 < nall) load_chunk(c + 1, wq);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int h = h0 + lane * 4 + u * 128;
-      const float4 w = wq[u];
-      // next round's load of this slot goes out before the arithmetic
-      const int hn = h + 512;
-      wq[u] = hn < H ? __ldg(reinterpret_cast<const float4*>(wrow + hn)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      if (h < H) {
+      const int h = h0 + lane * 4 + 512 * k + 128 * u;
+      if (h < h1) {
+        const float4 w = cur[u];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           if (q < nt) {
@@ -196,14 +210,21 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
         }
       }
     }
+    if (k == nch - 1) {
+      // end of a range: its lane tree, then onto the running sum
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float v = acc[q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        tot[q] += v;
+        acc[q] = 0.f;
+      }
+    }
   }
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    float v = acc[q];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && q < nt) logits[static_cast<size_t>(t0 + q) * E + e] = v;
-  }
+  for (int q = 0; q < 8; ++q)
+    if (lane == 0 && q < nt) logits[static_cast<size_t>(t0 + q) * E + e] = tot[q];
 }
 
 // Small-batch front end (T <= 8), one launch of E + T blocks (T when the

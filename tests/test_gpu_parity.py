@@ -279,6 +279,38 @@ def test_glm_decode_b1_full(lib, glm_layer):
 
 # ---------------------------------------------------------------- batch invariance
 
+@pytest.mark.parametrize("prenorm", [False, True], ids=["plain", "prenorm"])
+def test_router_logits_do_not_depend_on_the_batch_glm(lib, glm_layer, prenorm):
+    """Batches of up to 8 tokens get their router logits from front_kernel,
+    larger ones from logits_tile_kernel.  Both sum every (token, expert) dot
+    product in the same order, so a token's logits, and with them its
+    routing, are the same bits in a batch of 12 as alone."""
+    shape = synth.DECODE_B1
+    x = np.concatenate([synth.activations(shape, 0, b) for b in range(12)])
+    flags = lib._lib.COLI_LAYER_PRENORM if prenorm else 0
+    gb = run_gpu_layer(lib, glm_layer, x, flags=flags)
+    assert gb["flags"] == 0
+    for t in (0, 5, 11):
+        g1 = run_gpu_layer(lib, glm_layer, x[t:t + 1], flags=flags)
+        assert np.array_equal(g1["logits"][0], gb["logits"][t]), t
+        assert np.array_equal(g1["ids"][0], gb["ids"][t]) and np.array_equal(g1["w"][0], gb["w"][t]), t
+
+
+@pytest.mark.parametrize("hidden", [256, 512, 768, 1280])
+def test_router_logits_do_not_depend_on_the_batch_small(lib, hidden):
+    """The same across H whose eighth is not a multiple of 128 (some lanes of
+    each range idle, ragged last chunk)."""
+    shape = _small_shape(tokens=20, hidden=hidden, inter=128, n_experts=24, top_k=3)
+    layer = device_layer(shape, seed=14)
+    x = synth.normal_bf16(14, 5, synth.X_IN, (20, hidden))
+    gb = run_gpu_layer(lib, layer, x)
+    for t in range(0, 20, 3):
+        g1 = run_gpu_layer(lib, layer, x[t:t + 1])
+        assert np.array_equal(g1["logits"][0], gb["logits"][t]), t
+    g8 = run_gpu_layer(lib, layer, x[:8])
+    assert np.array_equal(g8["logits"], gb["logits"][:8])
+
+
 @pytest.mark.parametrize("T", [2, 4, 8])
 def test_decode_batch_invariance(lib, glm_layer, T):
     """A token's output in a batch of T (draft + verify tokens decoded in one
