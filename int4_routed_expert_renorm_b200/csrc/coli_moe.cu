@@ -901,10 +901,17 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
     rec.mark(1);
     if (!logits_in) {
       const uint16_t* xr = prenorm ? lay.xn : x;
-      const int tt = logits_tokens_per_block(H);
-      if (!launch(logits_tile_kernel, dim3((E + 7) / 8, (T + tt - 1) / tt), dim3(256),
-                  static_cast<size_t>(tt) * H * 2, s, xr, w->router_w, T, E, H, tt, lo))
-        return COLI_ERR_CUDA;
+      if (T >= kLogitsMmaMinT) {
+        // prefill-sized batches: tensor cores (bf16 pieces of W_r)
+        if (!launch(logits_mma_kernel, dim3((E + kLgBN - 1) / kLgBN, (T + kLgBM - 1) / kLgBM), dim3(256), 0, s,
+                    xr, w->router_w, T, E, H, lo))
+          return COLI_ERR_CUDA;
+      } else {
+        const int tt = logits_tokens_per_block(H);
+        if (!launch(logits_tile_kernel, dim3((E + 7) / 8, (T + tt - 1) / tt), dim3(256),
+                    static_cast<size_t>(tt) * H * 2, s, xr, w->router_w, T, E, H, tt, lo))
+          return COLI_ERR_CUDA;
+      }
       lg = lo;
     }
     rec.mark(2);

@@ -227,6 +227,159 @@ __global__ void __launch_bounds__(256) logits_tile_kernel(const uint16_t* __rest
     if (lane == 0 && q < nt) logits[static_cast<size_t>(t0 + q) * E + e] = tot[q];
 }
 
+// Router logits for batches of more than kLogitsMmaMinT - 1 tokens (prefill
+// chunks), on the tensor cores.  W_r (fp32) is split on the fly into three
+// bf16 pieces, w = w1 + w2 + w3 (w1 = bf16(w), w2 = bf16(w - w1), w3 =
+// bf16(w - w1 - w2); each difference is exact in fp32, so the pieces carry all
+// 24 bits of w), and l[t,e] = sum over the pieces of x . w_i^T with
+// mma.sync m16n8k16 (bf16 x bf16, exact products, fp32 accumulation).  Each
+// 256-wide K chunk is accumulated in a fresh accumulator (16 k-steps x 3
+// pieces) and added to the running fp32 sum in chunk order, so every (token,
+// expert) is summed the same way whatever the batch.  CTA = 64 tokens x 64
+// experts, 8 warps as 2 x 4 (32 tokens x 16 experts each); K in chunks of 32,
+// double-buffered in shared memory (rows padded to 40 bf16: conflict-free
+// fragment loads).  H % 256 == 0.
+constexpr int kLogitsMmaMinT = 65;
+constexpr int kLgBM = 64, kLgBN = 64, kLgBK = 32, kLgStr = 40;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The three bf16 pieces of four fp32 values, packed two per word.
+__device__ __forceinline__ void split3(float4 v, uint2 (&p)[3]) {
+  const float f[4] = {v.x, v.y, v.z, v.w};
+  uint16_t q[3][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t b1 = float_to_bf16_bits(f[i]);
+    const float r1 = f[i] - bf16_bits_to_float(b1);
+    const uint16_t b2 = float_to_bf16_bits(r1);
+    const float r2 = r1 - bf16_bits_to_float(b2);
+    q[0][i] = b1;
+    q[1][i] = b2;
+    q[2][i] = float_to_bf16_bits(r2);
+  }
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    p[j].x = q[j][0] | (static_cast<uint32_t>(q[j][1]) << 16);
+    p[j].y = q[j][2] | (static_cast<uint32_t>(q[j][3]) << 16);
+  }
+}
+
+__global__ void __launch_bounds__(256) logits_mma_kernel(const uint16_t* __restrict__ x,
+                                                         const float* __restrict__ wr, int T, int E, int H,
+                                                         float* __restrict__ logits) {
+  __shared__ __align__(16) uint16_t xs[2][kLgBM * kLgStr];
+  __shared__ __align__(16) uint16_t ws[2][3][kLgBN * kLgStr];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int t0 = blockIdx.y * kLgBM, e0 = blockIdx.x * kLgBN;
+  const int wm = warp & 1, wn = warp >> 1;
+  // global loads of one K chunk: x row tid / 4, 8 bf16 at column 8 (tid % 4);
+  // W_r rows tid / 8 and 32 + tid / 8, 4 fp32 at column 4 (tid % 8)
+  const int xr = tid >> 2, xq = tid & 3;
+  const int wrw = tid >> 3, wq = tid & 7;
+  const bool xin = t0 + xr < T;
+  const bool win0 = e0 + wrw < E, win1 = e0 + wrw + 32 < E;
+  const uint16_t* xp = x + static_cast<size_t>(xin ? t0 + xr : 0) * H + 8 * xq;
+  const float* wp0 = wr + static_cast<size_t>(win0 ? e0 + wrw : 0) * H + 4 * wq;
+  const float* wp1 = wr + static_cast<size_t>(win1 ? e0 + wrw + 32 : 0) * H + 4 * wq;
+  uint4 xv;
+  float4 wv0, wv1;
+  auto load = [&](int kc) {
+    const int k0 = kc * kLgBK;
+    xv = xin ? *reinterpret_cast<const uint4*>(xp + k0) : make_uint4(0u, 0u, 0u, 0u);
+    wv0 = win0 ? __ldg(reinterpret_cast<const float4*>(wp0 + k0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv1 = win1 ? __ldg(reinterpret_cast<const float4*>(wp1 + k0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  auto store = [&](int b) {
+    *reinterpret_cast<uint4*>(&xs[b][xr * kLgStr + 8 * xq]) = xv;
+    uint2 p0[3], p1[3];
+    split3(wv0, p0);
+    split3(wv1, p1);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      *reinterpret_cast<uint2*>(&ws[b][j][wrw * kLgStr + 4 * wq]) = p0[j];
+      *reinterpret_cast<uint2*>(&ws[b][j][(wrw + 32) * kLgStr + 4 * wq]) = p1[j];
+    }
+  };
+  pdl_wait();
+  pdl_trigger();
+  const int nk = H / kLgBK;
+  constexpr int kChunk = 256 / kLgBK;     // K chunks per fresh accumulator
+  float tot[2][2][4], acc[2][2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tot[mt][nt][i] = acc[mt][nt][i] = 0.f;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int kc = 0; kc < nk; ++kc) {
+    const int b = kc & 1;
+    if (kc + 1 < nk) load(kc + 1);
+#pragma unroll
+    for (int ks = 0; ks < kLgBK / 16; ++ks) {
+      const int kk = ks * 16 + 2 * c;
+      uint32_t a[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint16_t* r0 = &xs[b][(32 * wm + 16 * mt + g) * kLgStr + kk];
+        const uint16_t* r8 = r0 + 8 * kLgStr;
+        a[mt][0] = *reinterpret_cast<const uint32_t*>(r0);
+        a[mt][1] = *reinterpret_cast<const uint32_t*>(r8);
+        a[mt][2] = *reinterpret_cast<const uint32_t*>(r0 + 8);
+        a[mt][3] = *reinterpret_cast<const uint32_t*>(r8 + 8);
+      }
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint16_t* wrow = &ws[b][j][(16 * wn + 8 * nt + g) * kLgStr + kk];
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wrow);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wrow + 8);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(acc[mt][nt], a[mt], b0, b1);
+        }
+      }
+    }
+    if ((kc + 1) % kChunk == 0) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            tot[mt][nt][i] += acc[mt][nt][i];
+            acc[mt][nt][i] = 0.f;
+          }
+    }
+    if (kc + 1 < nk) store(b ^ 1);
+    __syncthreads();
+  }
+  // d0, d1: token row g, experts 2c, 2c + 1; d2, d3: token row g + 8
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + 32 * wm + 16 * mt + g + 8 * h;
+        const int e = e0 + 16 * wn + 8 * nt + 2 * c;
+        if (t < T) {
+          if (e < E) logits[static_cast<size_t>(t) * E + e] = tot[mt][nt][2 * h];
+          if (e + 1 < E) logits[static_cast<size_t>(t) * E + e + 1] = tot[mt][nt][2 * h + 1];
+        }
+      }
+}
+
 // Small-batch front end (T <= 8), one launch of E + T blocks (T when the
 // logits are given, wr == NULL): block e < E computes the router logits of
 // expert e for every token; block E + t writes token t's fragment-ordered

@@ -167,6 +167,8 @@ def test_prefill_4096_with_router_logits(lib):
     toks = np.unique(np.concatenate([[0, shape.tokens - 1], np.random.default_rng(7).integers(0, shape.tokens, 30)]))
     ref, _ = layer_outputs(shape, 0, 0, x[toks], lo[toks])
     err = _rel_err(out[toks], ref)
+    xa = np.abs(synth.bf16_bits_to_f32(x).astype(np.float64)) @ np.abs(rw.astype(np.float64)).T
     print(f"prefill 4096 with router logits: {len(toks)} tokens, max rel err {err:.3e}, "
-          f"max logit error {np.abs(lo - l64).max():.2e}")
+          f"max logit error {np.abs(lo - l64).max():.2e} "
+          f"({(np.abs(lo - l64) / (2.0 ** -24 * xa)).max():.2f} x 2^-24 sum|x w|)")
     assert err <= OUT_REL_TOL

@@ -311,6 +311,28 @@ def test_router_logits_do_not_depend_on_the_batch_small(lib, hidden):
     assert np.array_equal(g8["logits"], gb["logits"][:8])
 
 
+@pytest.mark.parametrize("kw", [dict(tokens=70, hidden=512, n_experts=24, top_k=3),
+                                dict(tokens=130, hidden=768, n_experts=100, top_k=8, n_shared=1)],
+                         ids=lambda kw: "-".join(f"{k}{v}" for k, v in kw.items()))
+def test_router_logits_tensor_core_path(lib, kw):
+    """Batches of 65 tokens or more get their router logits from the tensor
+    cores (three bf16 pieces of W_r): every logit within the fp32 bound of the
+    float64 oracle, routing and output checked as everywhere (tile edges: T
+    and E not multiples of 64); and a token's logits are the same bits in a
+    batch of 65 as in the larger one."""
+    shape = _small_shape(**kw)
+    layer = device_layer(shape, seed=15)
+    li = synth.LayerInputs(shape, seed=15)
+    x = synth.normal_bf16(15, 5, synth.X_IN, (shape.tokens, shape.hidden))
+    err, g = check_layer(lib, shape, layer, oracle_weights(shape, seed=15), x, rw=li.router_w(), max_ambiguous=2)
+    l64, _ = oracle.router_logits(x, li.router_w())
+    xa = np.abs(synth.bf16_bits_to_f32(x).astype(np.float64)) @ np.abs(li.router_w().astype(np.float64)).T
+    print(f"tensor-core logits: max error {np.abs(g['logits'] - l64).max():.2e}, "
+          f"in units of 2^-24 sum|x w|: {(np.abs(g['logits'] - l64) / (2.0 ** -24 * xa)).max():.2f}")
+    g65 = run_gpu_layer(lib, layer, x[:65])
+    assert np.array_equal(g65["logits"], g["logits"][:65])
+
+
 @pytest.mark.parametrize("T", [2, 4, 8])
 def test_decode_batch_invariance(lib, glm_layer, T):
     """A token's output in a batch of T (draft + verify tokens decoded in one
