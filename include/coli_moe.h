@@ -86,6 +86,9 @@ typedef enum {
 #define COLI_FLAG_NONFINITE 0x1u  /* a logit was NaN or +inf, or a selected logit was -inf */
 #define COLI_FLAG_BAD_ID    0x2u  /* an expert id outside [0, E) reached the union */
 #define COLI_FLAG_TIMEOUT   0x4u  /* a bounded pipeline wait expired; outputs are undefined */
+#define COLI_FLAG_RANGE     0x8u  /* the prefill form met an expert input or h value of magnitude
+                                   * 65536 or more, which its fp16 operands cannot hold; outputs
+                                   * are undefined */
 
 /* Layer flags (coli_moe_layer / coli_moe_expert_ffn). */
 #define COLI_LAYER_PRENORM       0x1u  /* route and run the experts on n = bf16(x * rsqrt(mean(x^2) + 1e-6)) */

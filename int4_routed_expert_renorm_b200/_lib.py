@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(PKG, "libcolimoe.so")
 # COLI_* constants of include/coli_moe.h
 COLI_OK, COLI_ERR_INVALID_ARG, COLI_ERR_UNSUPPORTED, COLI_ERR_WORKSPACE = 0, 1, 2, 3
 COLI_ERR_CUDA, COLI_ERR_NONFINITE, COLI_ERR_DEVICE = 4, 5, 6
-COLI_FLAG_NONFINITE, COLI_FLAG_BAD_ID, COLI_FLAG_TIMEOUT = 0x1, 0x2, 0x4
+COLI_FLAG_NONFINITE, COLI_FLAG_BAD_ID, COLI_FLAG_TIMEOUT, COLI_FLAG_RANGE = 0x1, 0x2, 0x4, 0x8
 COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
 COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 

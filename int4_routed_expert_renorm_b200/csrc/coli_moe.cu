@@ -841,7 +841,7 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   const StageRecorder rec(s);
   rec.mark(0);
   if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, dims->hidden, 0, static_cast<uint16_t*>(nullptr), lay.xq,
-              lay.xp, lay.xe))
+              lay.xp, lay.xe, form == Form::kPrefill ? 1 : 0, di.status))
     return COLI_ERR_CUDA;
   rec.mark_through(1, 4);
   if (form == Form::kPrefill)
@@ -890,13 +890,14 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
     const float* wr = logits_in ? nullptr : w->router_w;
     const int grid = (logits_in ? 0 : E) + T;
     if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq,
-                lay.xp, lay.xe))
+                lay.xp, lay.xe, form == Form::kPrefill ? 1 : 0, di.status))
       return COLI_ERR_CUDA;
     rec.mark_through(1, 2);
     if (!logits_in) lg = lo;
   } else {
     if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, H, prenorm ? 1 : 0, lay.xn, lay.xq,
-                static_cast<uint8_t*>(nullptr), static_cast<int32_t*>(nullptr)))
+                static_cast<uint8_t*>(nullptr), static_cast<int32_t*>(nullptr), form == Form::kPrefill ? 1 : 0,
+                di.status))
       return COLI_ERR_CUDA;
     rec.mark(1);
     if (!logits_in) {

@@ -177,6 +177,20 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
+// fp16 bits of a bf16 value: exact unless |v| < 2^-17 (rounded to fp16's
+// subnormal grid) or |v| >= 65536 (infinity; `range` is set).
+__device__ __forceinline__ uint16_t bf16_to_f16_bits(uint16_t b, bool& range) {
+  const float f = bf16_bits_to_float(b);
+  range |= fabsf(f) >= 65536.0f && fabsf(f) != INFINITY;
+  return __half_as_ushort(__float2half_rn(f));
+}
+
+// The same for eight values in place.
+__device__ __forceinline__ void to_f16_8(uint16_t (&e)[8], bool& range) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) e[q] = bf16_to_f16_bits(e[q], range);
+}
+
 // Position of natural element i (within a row) in the fragment-ordered copy of
 // an activation row: every block of 8 elements is stored as
 // x0 x4 x1 x5 x2 x6 x3 x7, so that one 16-byte load gives the bf16 pairs

@@ -6,19 +6,24 @@
 // (segment, token block of <= 160 tokens, 128 weight rows); segments are the
 // union's experts followed by the shared ones.  Per tile and 64-wide K chunk:
 //   * the producer warp copies the chunk's codes and fp16 group scales
-//     (2-D tensor maps, 4 chunks per copy) and the token rows (bf16, 128B
+//     (2-D tensor maps, 4 chunks per copy) and the token rows (fp16, 128B
 //     swizzle) into two shared-memory rings;
 //   * 16 dequantisation warps, one weight row per thread, turn the codes into
-//     bf16 q*s (one mask-and-magic LOP3, one bf16x2 subtract, one bf16x2
-//     multiply per pair of codes) and store them straight into tensor memory
-//     with tcgen05.st: the weights are the MMA's A operand *in TMEM*, so they
-//     never pass through shared memory;
+//     fp16 q*s (one mask-and-magic LOP3, one f16x2 subtract, one f16x2
+//     multiply per pair of codes: q exact, q*s rounded once to 11 bits) and
+//     store them straight into tensor memory with tcgen05.st: the weights are
+//     the MMA's A operand *in TMEM*, so they never pass through shared memory;
 //   * one thread issues tcgen05.mma (kind::f16, M = 128 weight rows, N =
 //     the tile's tokens rounded up to 16, K = 16) from A in TMEM and the
 //     token tile in shared memory into fp32 accumulators in TMEM, and
 //     releases A buffers and token stages with tcgen05.commit;
 //   * the same 16 warps read the accumulators back (tcgen05.ld) and write
-//     h = bf16(silu(g) * u) (gate/up launch) or y in fp32 (down launch).
+//     h = bf16(silu(g) * u) (gate/up launch; stored as the fp16 of that bf16
+//     value, which is exact) or y in fp32 (down launch).
+// Both MMA operands are fp16 (kind::f16 takes one type for A and B): the
+// expert input rows are the fp16 copies of their bf16 values (exact from
+// 2^-17 up; COLI_FLAG_RANGE marks a value of 65536 or more, which fp16
+// cannot hold), and h likewise.
 // A tile of the gate/up launch holds the same 128 rows of both matrices; a
 // tile of the down launch holds two neighbouring 128-row blocks of W_down.
 // Either way two weight blocks share each token tile, which halves the
@@ -126,10 +131,10 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
          (static_cast<uint64_t>(2) << 61);
 }
 
-// Instruction descriptor of kind::f16: bf16 A and B (both K-major), fp32
-// accumulate, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_bf16_m128(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | ((128u >> 4) << 24);
+// Instruction descriptor of kind::f16: fp16 A and B (both K-major; type
+// fields 0), fp32 accumulate, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_f16_m128(int n) {
+  return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
@@ -152,12 +157,24 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// bf16x2 a * b, rounded to nearest even (a * b + (-0) is exactly a * b).
-__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+// Two code nibbles (e_i, e_{i+4}) of word w -> exact f16x2 (q_i, q_{i+4}):
+// (w >> sh) & 0x000F000F keeps one nibble per 16-bit half; XOR with 0x6408
+// puts it under the exponent of 1024 and flips bit 3, giving 1024 + (n ^ 8)
+// = 1032 + q; subtracting 1032 leaves q.
+__device__ __forceinline__ uint32_t dq_pair_f16(uint32_t w, int sh) {
+  uint32_t r, q;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(w >> sh), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(r), "r"(0x64086408u));
+  return q;
+}
+
+// f16x2 a * b, rounded to nearest even.
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(0x80008000u));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+
 
 // ------------------------------------------------------------- tile plan --
 
@@ -426,7 +443,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const PfTile ti = pf_decode<DOWN>(a, blk_off, n_seg, uniq, seg, U, mbk, t);
-        const uint32_t idesc = idesc_bf16_m128(ti.npad);
+        const uint32_t idesc = idesc_f16_m128(ti.npad);
         const int ab = static_cast<int>(tt % C::ACC_BUFS);
         const uint32_t dbase = tbase + ab * NMAT * kPfMaxN;
         if (!(ok = mbar_wait(&acc_empty[ab], ((tt / C::ACC_BUFS) & 1u) ^ 1u, abort_flag, a.status))) break;
@@ -474,6 +491,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     uint32_t it = 0, tt = 0;
     uint32_t scl[NMAT][4];                    // this row's fp16 scales of the current code stage
     bool ok = true;
+    bool range = false;                       // an h value fp16 cannot hold
     // epilogue of one tile: accumulators -> h (gate/up) or y (down)
     auto epilogue = [&](const PfTile& et, uint32_t ett) -> bool {
       const int ab = static_cast<int>(ett % C::ACC_BUFS);
@@ -494,7 +512,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!DOWN) {
               const float gv = __uint_as_float(d0[n]), uv = __uint_as_float(d1[n]);
               const float hv = gv / (1.0f + expf(-gv)) * uv;
-              a.hq[static_cast<size_t>(et.orow + i) * a.I + hpos] = float_to_bf16_bits(hv);
+              a.hq[static_cast<size_t>(et.orow + i) * a.I + hpos] = bf16_to_f16_bits(float_to_bf16_bits(hv), range);
             } else {
               float* yrow = a.ypair + static_cast<size_t>(et.orow + i) * a.H + grow;
               yrow[0] = __uint_as_float(d0[n]);
@@ -566,14 +584,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const uint32_t sw = ci == 0 ? scl[m][0] : ci == 1 ? scl[m][1] : ci == 2 ? scl[m][2] : scl[m][3];
             sh = sw >> (g * 16);
           }
-          const uint16_t sb = float_to_bf16_bits(half_bits_to_float(static_cast<uint16_t>(sh & 0xFFFFu)));
-          const uint32_t s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
+          const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
           const uint32_t wd[4] = {cw[m].x, cw[m].y, cw[m].z, cw[m].w};
           uint32_t v[16];
 #pragma unroll
           for (int w = 0; w < 4; ++w)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[4 * w + i] = bmul2(dq_pair(wd[w], 4 * i), s2);
+            for (int i = 0; i < 4; ++i) v[4 * w + i] = hmul2(dq_pair_f16(wd[w], 4 * i), s2);
           tmem_st16(tbase + lane_bits + C::ACOL + b * 32 * NMAT + m * 32 + g * 16, v);
         }
         tmem_wait_st();
@@ -592,6 +609,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ++tt;
     }
     if (ok && has_pend) ok = epilogue(pend, pend_tt);
+    if (range) atomicOr(a.status, COLI_FLAG_RANGE);
   }
   tc_fence_before();
   __syncthreads();

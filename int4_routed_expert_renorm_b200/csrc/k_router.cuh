@@ -71,20 +71,23 @@ __device__ __forceinline__ void token_planes(const uint16_t* __restrict__ xr, in
 }
 
 // One block per token.  Writes the fragment-ordered copy `xq` of the layer's
-// expert input, its integer planes `xp` / grid exponents `xe` when xp is not
-// NULL (the split-K decode form), and, with prenorm, the natural-order
-// normalised copy `xn`:
+// expert input (bf16; with xq_f16, for the prefill form, the fp16 copies of
+// those bf16 values, COLI_FLAG_RANGE for one of magnitude 65536 or more), its
+// integer planes `xp` / grid exponents `xe` when xp is not NULL (the split-K
+// decode form), and, with prenorm, the natural-order normalised copy `xn`:
 //   n = bf16( x * (1 / sqrt(mean(x^2) + 1e-6)) ), the sum of squares in fp32
 // in a fixed order.  H % 8 == 0.
 __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int H, int prenorm,
                                                    uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
-                                                   uint8_t* __restrict__ xp, int32_t* __restrict__ xe) {
+                                                   uint8_t* __restrict__ xp, int32_t* __restrict__ xe, int xq_f16,
+                                                   uint32_t* __restrict__ status) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
   const uint16_t* xr = x + static_cast<size_t>(t) * H;
   __shared__ float red[8];
   float r = 1.0f;
+  bool range = false;
   if (prenorm) {
     float ss = 0.f;
     for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
@@ -124,7 +127,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
       o.w = e[6] | (static_cast<uint32_t>(e[7]) << 16);
       *reinterpret_cast<uint4*>(xn + static_cast<size_t>(t) * H + i) = o;
     }
-    // fragment order x0 x4 x1 x5 x2 x6 x3 x7
+    // fragment order x0 x4 x1 x5 x2 x6 x3 x7 (fp16 copies for the prefill form)
+    if (xq_f16) to_f16_8(e, range);
     uint4 o;
     o.x = e[0] | (static_cast<uint32_t>(e[4]) << 16);
     o.y = e[1] | (static_cast<uint32_t>(e[5]) << 16);
@@ -132,6 +136,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
     o.w = e[3] | (static_cast<uint32_t>(e[7]) << 16);
     *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
   }
+  if (range) atomicOr(status, COLI_FLAG_RANGE);
   if (xp) {
     __shared__ float mx[8];
     token_planes(xr, H, prenorm, r, xp + static_cast<size_t>(t) * (H / 32) * kPlaneRec, xe + t, mx);
@@ -391,7 +396,8 @@ __global__ void __launch_bounds__(256) logits_mma_kernel(const uint16_t* __restr
 __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                                                     int T, int E, int H, int prenorm, float* __restrict__ logits,
                                                     uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
-                                                    uint8_t* __restrict__ xp, int32_t* __restrict__ xe) {
+                                                    uint8_t* __restrict__ xp, int32_t* __restrict__ xe, int xq_f16,
+                                                    uint32_t* __restrict__ status) {
   pdl_wait();
   pdl_trigger();
   const int nlog = wr ? E : 0;   // blocks [0, nlog): logits of expert b; then one block per token
@@ -442,6 +448,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
     const int t = blockIdx.x - nlog;
     const uint16_t* xr = x + static_cast<size_t>(t) * H;
     const float r = prenorm ? rs[t] : 1.0f;
+    bool range = false;
     for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
       const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
       uint16_t q8[8];
@@ -461,6 +468,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
         o.w = q8[6] | (static_cast<uint32_t>(q8[7]) << 16);
         *reinterpret_cast<uint4*>(xn + static_cast<size_t>(t) * H + i) = o;
       }
+      if (xq_f16) to_f16_8(q8, range);
       uint4 o;
       o.x = q8[0] | (static_cast<uint32_t>(q8[4]) << 16);
       o.y = q8[1] | (static_cast<uint32_t>(q8[5]) << 16);
@@ -468,6 +476,7 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
       o.w = q8[3] | (static_cast<uint32_t>(q8[7]) << 16);
       *reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * H + i) = o;
     }
+    if (range) atomicOr(status, COLI_FLAG_RANGE);
     if (xp) {
       __shared__ float mx[8];
       token_planes(xr, H, prenorm, r, xp + static_cast<size_t>(t) * (H / 32) * kPlaneRec, xe + t, mx);

@@ -54,6 +54,23 @@ def test_prefill_form_hot_expert_and_prenorm(lib):
                 flags=PREFILL | lib._lib.COLI_LAYER_PRENORM, max_ambiguous=3)
 
 
+def test_prefill_form_flags_inputs_fp16_cannot_hold(lib):
+    """The prefill form's MMA operands are fp16 copies of the bf16 expert
+    input and h: an input of magnitude 65536 or more sets COLI_FLAG_RANGE
+    (the call's outputs are undefined); the next call is clean."""
+    shape = _small_shape(tokens=40, n_shared=1)
+    layer = device_layer(shape, seed=16)
+    li = synth.LayerInputs(shape, seed=16)
+    x = synth.normal_bf16(16, 5, synth.X_IN, (40, shape.hidden))
+    big = x.copy()
+    big[3, 17] = 0x47C3          # bf16 99840
+    g = run_gpu_layer(lib, layer, big, flags=PREFILL)
+    assert g["flags"] & lib._lib.COLI_FLAG_RANGE
+    check_layer(lib, shape, layer, oracle_weights(shape, seed=16), x, rw=li.router_w(), flags=PREFILL)
+    g = run_gpu_layer(lib, layer, big)          # the decode form holds it
+    assert g["flags"] == 0
+
+
 def test_both_form_flags_are_rejected(lib):
     shape = _small_shape(tokens=40)
     layer = device_layer(shape, seed=9)
