@@ -54,6 +54,31 @@ def test_prefill_form_hot_expert_and_prenorm(lib):
                 flags=PREFILL | lib._lib.COLI_LAYER_PRENORM, max_ambiguous=3)
 
 
+def _dist_to_exact(lib, shape, layer, W, x, flags):
+    """Largest |GPU output - unrounded float64 oracle sum| over max|sum|, with
+    the GPU's own routing fed to the oracle (the FFN arithmetic alone)."""
+    g = run_gpu_layer(lib, layer, x, flags=flags)
+    assert g["flags"] == 0
+    _, acc = oracle.moe_ffn_combine(W, x, g["ids"], g["w"], shape.n_experts, shape.n_shared, return_f64=True)
+    return np.abs(oracle.bf16_bits_to_f64(g["out"]) - acc).max() / np.abs(acc).max()
+
+
+def test_prefill_form_arithmetic_error(lib):
+    """Distance of each form's output to the oracle's unrounded float64 sum.
+    Rounding the output to bf16 alone costs up to 2^-8 of a value (half an ulp
+    of an 8-bit significand); the rest is the form's arithmetic, allowed 1e-3
+    here.  The prefill form's fp16 operands (each weight q * s rounded once at
+    11 bits) keep it at the decode form's level."""
+    shape = _small_shape(tokens=96, hidden=1024, inter=512, n_experts=8, top_k=2, n_shared=1)
+    layer = device_layer(shape, seed=17)
+    W = oracle_weights(shape, seed=17)
+    x = synth.normal_bf16(17, 5, synth.X_IN, (96, shape.hidden))
+    dp = _dist_to_exact(lib, shape, layer, W, x, PREFILL)
+    dd = _dist_to_exact(lib, shape, layer, W, x, DECODE)
+    print(f"distance to the unrounded oracle: prefill form {dp:.3e}, decode form {dd:.3e} (2^-8 = {2.0 ** -8:.3e})")
+    assert dp <= 2.0 ** -8 + 1e-3 and dd <= 2.0 ** -8 + 1e-3
+
+
 def test_prefill_form_flags_inputs_fp16_cannot_hold(lib):
     """The prefill form's MMA operands are fp16 copies of the bf16 expert
     input and h: an input of magnitude 65536 or more sets COLI_FLAG_RANGE
