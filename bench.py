@@ -68,23 +68,47 @@ def parse():
     return a
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture
-# of the same kernel build: (workload, FFN form) -> bytes.  The batch-1 capture
-# ran on the 16-expert variant of the layer, which moves the same 9 experts per
-# step (profiles/ffn_splitk_kernel_glm52_layer_decode_b1_e16.md).  The prefill capture ran on the 32-expert, 512-token variant (same tile
-# shapes): there DRAM traffic was 1.063x the algorithmic bytes of the gate/up
-# launch (profiles/ffn_prefill_kernel_glm52_layer_prefill_512_e32.md); the
-# 4096-token figure is that ratio times its own algorithmic bytes (257 experts'
-# gate+up codes and scales, 36,864 gathered rows, h written).
-_PF_RATIO = (532.542208e6 + 16.592384e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
-TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.724544e6 + 3.525376e6,
-           ("glm52_layer_decode_b1_e16", "decode"): 191.724544e6 + 3.525376e6,
-           ("glm52_layer_prefill_512_e32", "prefill"): 532.542208e6 + 16.592384e6,
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture, with a digest of the kernel sources that capture ran on:
+# (workload, FFN form) -> bytes.  While the sources differ from that digest
+# (a kernel changed since the counters were taken) the line reports null.
+# The batch-1 capture ran on the 16-expert variant of the layer, which moves
+# the same 9 experts per step; the prefill capture on the 32-expert, 512-token
+# variant (same tile shapes), where DRAM traffic was 1.064x the algorithmic
+# bytes of the gate/up launch; the 4096-token figure is that ratio times its
+# own algorithmic bytes (257 experts' gate+up codes and scales, 36,864
+# gathered rows, h written).
+TRAFFIC_SOURCES = "47033e5dc090e639"
+_PF_RATIO = (532.682752e6 + 16.870912e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
+TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.315200e6 + 4.964096e6,
+           ("glm52_layer_decode_b1_e16", "decode"): 191.315200e6 + 4.964096e6,
+           ("glm52_layer_prefill_512_e32", "prefill"): 532.682752e6 + 16.870912e6,
            ("glm52_layer_prefill_4096", "prefill"):
                _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2),
            # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
            ("glm52_layer_prefill_4096_router", "prefill"):
                _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)}
+
+
+def kernel_sources_digest() -> str:
+    """First 16 hex digits of the sha256 over the library's kernel sources
+    (file name, then contents, in name order)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "int4_routed_expert_renorm_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str, form: str):
+    """The captured DRAM bytes per launch, or None when there is no capture of
+    the current kernel sources."""
+    if kernel_sources_digest() != TRAFFIC_SOURCES:
+        return None
+    return TRAFFIC.get((workload, form))
 
 
 def splitk_form(shape) -> bool:
@@ -504,7 +528,7 @@ def main():
                                "+ x read + h write/read + y write" + (" + y read + out write" if fused_combine else ""),
                 "peak_kind": f"{src} HBM copy"}
 
-    roof["traffic"] = TRAFFIC.get((shape.name, form))
+    roof["traffic"] = traffic_for(shape.name, form)
     # the same figure against the nominal spec (8 TB/s HBM3e; 2.25 PFLOP/s dense bf16), for context
     spec = 8000.0 if roof["unit"] == "GB/s" else 2250.0
     roof["frac_of_spec"] = roof["achieved"] / spec
