@@ -42,8 +42,11 @@
  *
  * Conventions for every call:
  *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
- *     The library allocates no memory, keeps no per-call state and does not
- *     retain pointers after the call returns.
+ *     The library allocates no memory at run time, keeps no per-call state
+ *     and does not retain pointers after the call returns.  Its only device
+ *     memory is file-scope: a status word per device and the fixed scratch
+ *     array of coli_moe_layer_noalloc (COLI_NOALLOC_SCRATCH_BYTES), which
+ *     exist once the library is loaded.
  *   - bf16 / fp16 tensors are passed as uint16_t bit patterns.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
  *     enqueue work on it: they never synchronise, never allocate, and can be
