@@ -124,7 +124,10 @@ typedef struct {
 } coli_moe_weights;
 
 /*
- * Route: top-k selection and renormalised softmax weights per token.
+ * Route: top-k selection and renormalised softmax weights per token
+ * (Colibri README, "L'idea": the router picks k experts per token and per
+ * layer; the renormalised softmax over the selected logits is the layer
+ * statement's reading, the README gives no formula).
  *   logits   fp32 [T][E]   router logits (device)
  *   bias     fp32 [E]      additive per-expert bias, or NULL
  *   topk_ids int32 [T][k]  out: selected experts, slot order = selection order
@@ -136,7 +139,9 @@ coli_status coli_moe_route(const float *logits, const float *bias, int T, int E,
                            int32_t *topk_ids, float *topk_w, void *stream);
 
 /*
- * Union: batch-union of the selected experts, without atomics.
+ * Union: batch-union of the selected experts, without atomics (Colibri README,
+ * "Mai aspettare il disco due volte": a batch reads each expert its tokens
+ * selected once, however many of them selected it).
  *   topk_ids  int32 [T][k]        in
  *   unique_ids int32 [min(E,T*k)] out: experts used by the batch, ascending
  *   n_unique  int32 [1]           out: U (stays on the device)
@@ -153,7 +158,10 @@ coli_status coli_moe_union(const int32_t *topk_ids, int T, int k, int E,
                            int32_t *perm, int32_t *pair_pos, void *stream);
 
 /*
- * Expert FFN + combine for an already routed and unioned batch.
+ * Expert FFN + combine for an already routed and unioned batch (Colibri
+ * README, "L'idea": int4 routed experts with group scales; each unique expert
+ * runs once over its tokens, SwiGLU, then the routing-weighted sum back into
+ * token order).
  *   x         bf16 [T][H]   expert input
  *   topk_ids, topk_w, unique_ids, n_unique, seg_off, perm, pair_pos:
  *             as produced by coli_moe_route / coli_moe_union
@@ -173,7 +181,9 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims *dims, const coli_moe_weight
                                 void *stream);
 
 /*
- * One whole MoE layer: [pre-norm] -> logits -> Route -> Union -> FFN -> combine.
+ * One whole MoE layer: [pre-norm] -> logits -> Route -> Union -> FFN -> combine
+ * (the per-token path of the Colibri README, "L'idea" and "Mai aspettare il
+ * disco due volte", with every expert resident: "Una gerarchia di memoria").
  *   x          bf16 [T][H]
  *   logits_in  fp32 [T][E] or NULL: when given, replaces x . W_r^T
  *   residual   bf16 [T][H] or NULL
