@@ -200,6 +200,38 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
                            void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * One expert-parallel rank's share of coli_moe_layer.  The pages' fastest
+ * runs spread full expert residence over several GPUs (Colibri README, "Cosa
+ * ottiene"); here G ranks each hold a contiguous range of the E experts, the
+ * router and the union are replicated, and the ranks' partial outputs are
+ * summed by an all-reduce.  The call routes every token over all E experts
+ * (router_w, router_bias: the full [E][H] / [E]; or logits_in), builds the
+ * union of the whole batch, and computes
+ *   out_partial[t] = sum over slots j with expert_begin <= id[t][j] < expert_end
+ *                    of w[t][j] * y_id(x_t)
+ *                  + (with_shared ? sum_s y_{E+s}(x_t) : 0) + (residual ? residual[t] : 0)
+ * in fp32, unrounded.  The sum of the ranks' partials (pass the residual on one
+ * rank only), rounded once to bf16 (coli_moe_partial_to_bf16), is the layer's
+ * output up to the order of that fp32 sum.
+ *   w            expert tensors of this rank only: routed experts
+ *                [expert_begin, expert_end) at indices 0.., then, when
+ *                with_shared != 0, the S shared experts; same layouts as above
+ *   out_partial  fp32 [T][H] (16-byte aligned; must not alias x)
+ *   logits_out, topk_ids_out, topk_w_out, ws, ws_bytes, flags: as coli_moe_layer
+ * Runs in the split-K decode form only: other batches (T > 8, I not a multiple
+ * of 256, COLI_PATH_PREFILL) return COLI_ERR_UNSUPPORTED;
+ * 0 <= expert_begin < expert_end <= E, else COLI_ERR_INVALID_ARG.
+ */
+coli_status coli_moe_layer_ep(const coli_moe_dims *dims, const coli_moe_weights *w, int expert_begin,
+                              int expert_end, int with_shared, const uint16_t *x, int T, const float *logits_in,
+                              const uint16_t *residual, uint32_t flags, float *out_partial, float *logits_out,
+                              int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+
+/* out[i] = bf16(partial[i]) for i < n (n a multiple of 4; partial 16-byte and
+ * out 8-byte aligned): the rounding step after the ranks' all-reduce. */
+coli_status coli_moe_partial_to_bf16(const float *partial, uint16_t *out, size_t n, void *stream);
+
+/*
  * coli_moe_layer without a caller-provided workspace.  The pages describe no
  * such call; it exists for callers that cannot allocate device memory when
  * they run the layer: code embedded in a host runtime that owns every device

@@ -24,7 +24,7 @@ COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
            "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form",
-           "coli_moe_union_offsets", "coli_moe_test_wait_timeout")
+           "coli_moe_union_offsets", "coli_moe_test_wait_timeout", "coli_moe_layer_ep", "coli_moe_partial_to_bf16")
 COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -67,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_ffn_form": (I, [D, I, U32, ctypes.POINTER(I)]),
         "coli_moe_union_offsets": (I, [D, I, ctypes.POINTER(Z)]),
         "coli_moe_test_wait_timeout": (I, [U64, P, P]),
+        "coli_moe_layer_ep": (I, [D, W, I, I, I, P, I, P, P, U32, P, P, P, P, P, Z, P]),
+        "coli_moe_partial_to_bf16": (I, [P, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -214,6 +216,26 @@ def coli_moe_layer_noalloc(dims, weights, x, out, logits_in=None, residual=None,
     _check(_lib.coli_moe_layer_noalloc(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
                                        _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
                                        _ptr(topk_w_out), _stream(stream)), "coli_moe_layer_noalloc")
+
+
+def coli_moe_layer_ep(dims, weights, expert_begin: int, expert_end: int, with_shared: bool, x, out_partial, ws,
+                      logits_in=None, residual=None, flags=0, logits_out=None, topk_ids_out=None, topk_w_out=None,
+                      stream=None):
+    """One expert-parallel rank's fp32 partial output (see the header)."""
+    T = _tokens(x, dims.hidden)
+    _layer_sizes(dims, T, None, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
+    _need(out_partial, T * dims.hidden, 4, "out_partial")
+    _check(_lib.coli_moe_layer_ep(ctypes.byref(dims), ctypes.byref(weights), expert_begin, expert_end,
+                                  1 if with_shared else 0, _ptr(x), T, _ptr(logits_in), _ptr(residual), flags,
+                                  _ptr(out_partial), _ptr(logits_out), _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "coli_moe_layer_ep")
+
+
+def coli_moe_partial_to_bf16(partial, out, stream=None):
+    """out = bf16(partial), elementwise (out: bf16 bits, int16 tensor)."""
+    n = partial.numel()
+    _need(out, n, 2, "out")
+    _check(_lib.coli_moe_partial_to_bf16(_ptr(partial), _ptr(out), n, _stream(stream)), "coli_moe_partial_to_bf16")
 
 
 def coli_moe_union_offsets(dims, T: int) -> list[int]:

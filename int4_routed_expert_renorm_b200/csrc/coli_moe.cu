@@ -427,12 +427,14 @@ bool launch_route(const float* lg, const float* bias, int T, int E, int k, int32
 // Route + union + plan in one CTA (T <= kFusedRouteMaxT); one warp does the
 // union when T*k <= kWarpUnionMaxP.
 bool launch_route_union(const float* lg, const float* bias, int T, int E, int k, int S, int tokb, int n_rb,
-                        int32_t* ids, float* w, const Ws& ws, uint32_t* status, cudaStream_t st) {
+                        int32_t* ids, float* w, const Ws& ws, uint32_t* status, cudaStream_t st, int eb = 0,
+                        int ee = -1) {
+  if (ee < 0) ee = E;
   if (T * k <= kWarpUnionMaxP) {
     const dim3 g(1), b(32 * (T < 8 ? T : 8));
 #define COLI_RUS(NV)                                                                                             \
   launch(route_union_small_kernel<NV>, g, b, 0, st, lg, bias, T, E, k, ids, w, ws.unique, ws.n_unique, ws.seg_off, \
-         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb)
+         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb, eb, ee)
     switch (route_nv(E)) {
       case 1: return COLI_RUS(1);
       case 2: return COLI_RUS(2);
@@ -599,14 +601,27 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
 
 // The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer;
 // the tile plan (ws.plan) must already be on the stream.
+// The experts one call computes: all of them, or an expert-parallel rank's
+// share (routed experts [begin, end), the shared ones when shared != 0), whose
+// weights then hold only those experts, and whose output is the unrounded
+// fp32 partial sum `out_f32`.
+struct EpRange {
+  bool on = false;
+  int begin = 0, end = 0, shared = 0;
+  const int32_t* ids = nullptr;
+  float* out_f32 = nullptr;
+};
+
 coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
                     const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
                     const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
-                    cudaStream_t st, const StageRecorder& rec) {
-  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
+                    cudaStream_t st, const StageRecorder& rec, const EpRange& ep = EpRange()) {
+  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k;
+  const int S = ep.on ? ep.shared : d->n_shared;
+  const int E_w = ep.on ? ep.end - ep.begin : E;   // routed experts held by the weights
   const int P = T * k;
-  const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
-  const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
+  const uint64_t rows_gu = static_cast<uint64_t>(E_w + S) * I;
+  const uint64_t rows_dn = static_cast<uint64_t>(E_w + S) * H;
   const int tokb = tok_block(T);
 
   // upper bound on tiles: every segment contributes ceil(cnt/64) <= cnt/64 + 1 blocks
@@ -650,6 +665,11 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   a.E = E;
   a.S = S;
   a.P = P;
+  a.e_off = ep.on ? ep.begin : 0;
+  a.e_end = ep.on ? ep.end : E;
+  a.e_shared = E_w;
+  a.topk_ids = ep.on ? ep.ids : nullptr;
+  a.out_f32 = ep.on ? ep.out_f32 : nullptr;
   if (use_splitk(d, T)) {
     // down maps of the split-K form: codes in boxes of 128 rows x one
     // 128-wide K slice (64 bytes, 64B swizzle; int8: 128 bytes, 128B
@@ -854,23 +874,31 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   return run_ffn(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di, s, rec);
 }
 
-coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
-                           const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
-                           float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
-                           void* stream) {
+namespace {
+
+coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
+                       const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
+                       float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                       void* stream, EpRange ep) {
   coli_status st = check_dims(dims);
   if (st != COLI_OK) return st;
   if (T < 0) return COLI_ERR_INVALID_ARG;
   if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
+  if (ep.on && (ep.begin < 0 || ep.end > dims->n_experts || ep.begin >= ep.end)) return COLI_ERR_INVALID_ARG;
   if ((st = check_weights(w, logits_in == nullptr)) != COLI_OK) return st;
   if (T == 0) return COLI_OK;
-  if (!x || !out || !ws) return COLI_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || !aligned(ws, 256))
+  if (!x || !ws || (ep.on ? !ep.out_f32 : !out)) return COLI_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (out && !aligned(out, 16)) || (ep.out_f32 && !aligned(ep.out_f32, 16)) ||
+      (residual && !aligned(residual, 16)) || !aligned(ws, 256))
     return COLI_ERR_INVALID_ARG;
-  if (x == out) return COLI_ERR_INVALID_ARG;
+  if (x == out || x == reinterpret_cast<const void*>(ep.out_f32)) return COLI_ERR_INVALID_ARG;
   const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
+  // an expert-parallel share runs in the split-K decode form only
+  if (ep.on && !(form == Form::kDecode && use_splitk(dims, T) && T <= kFusedRouteMaxT &&
+                 T * dims->top_k <= kWarpUnionMaxP))
+    return COLI_ERR_UNSUPPORTED;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
   DevInfo di;
@@ -926,7 +954,8 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   int32_t* ids = topk_ids_out ? topk_ids_out : lay.ids;
   float* tw = topk_w_out ? topk_w_out : lay.w;
   if (T <= kFusedRouteMaxT) {
-    if (!launch_route_union(lg, w->router_bias, T, E, k, S, tokb, H / kRowBlock, ids, tw, lay, di.status, s))
+    if (!launch_route_union(lg, w->router_bias, T, E, k, ep.on ? ep.shared : S, tokb, H / kRowBlock, ids, tw, lay,
+                            di.status, s, ep.on ? ep.begin : 0, ep.on ? ep.end : E))
       return COLI_ERR_CUDA;
     rec.mark_through(3, 5);
   } else {
@@ -955,8 +984,66 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w,
   if (form == Form::kPrefill)
     return run_ffn_prefill(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual,
                            out, lay, di, s, rec);
+  ep.ids = ids;
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
-                 di, s, rec);
+                 di, s, rec, ep);
+}
+
+}  // namespace
+
+coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
+                           const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
+                           float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  return layer_impl(dims, w, x, T, logits_in, residual, flags, out, logits_out, topk_ids_out, topk_w_out, ws,
+                    ws_bytes, stream, EpRange());
+}
+
+coli_status coli_moe_layer_ep(const coli_moe_dims* dims, const coli_moe_weights* w, int expert_begin,
+                              int expert_end, int with_shared, const uint16_t* x, int T, const float* logits_in,
+                              const uint16_t* residual, uint32_t flags, float* out_partial, float* logits_out,
+                              int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  EpRange ep;
+  ep.on = true;
+  ep.begin = expert_begin;
+  ep.end = expert_end;
+  ep.shared = with_shared ? (dims ? dims->n_shared : 0) : 0;
+  ep.out_f32 = out_partial;
+  return layer_impl(dims, w, x, T, logits_in, residual, flags, nullptr, logits_out, topk_ids_out, topk_w_out, ws,
+                    ws_bytes, stream, ep);
+}
+
+namespace {
+
+// out = bf16(in), four values per thread.
+__global__ void __launch_bounds__(256) partial_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
+                                                             size_t n4) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = in[i];
+    uint2 o;
+    o.x = float_to_bf16_bits(v.x) | (static_cast<uint32_t>(float_to_bf16_bits(v.y)) << 16);
+    o.y = float_to_bf16_bits(v.z) | (static_cast<uint32_t>(float_to_bf16_bits(v.w)) << 16);
+    out[i] = o;
+  }
+}
+
+}  // namespace
+
+coli_status coli_moe_partial_to_bf16(const float* partial, uint16_t* out, size_t n, void* stream) {
+  if (n == 0) return COLI_OK;
+  if (!partial || !out || n % 4 != 0 || !aligned(partial, 16) || !aligned(out, 8)) return COLI_ERR_INVALID_ARG;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  const size_t n4 = n / 4;
+  size_t blocks = (n4 + 255) / 256;
+  if (blocks > static_cast<size_t>(4) * di.sms) blocks = static_cast<size_t>(4) * di.sms;
+  return launch(partial_to_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, as_stream(stream),
+                reinterpret_cast<const float4*>(partial), reinterpret_cast<uint2*>(out), n4)
+             ? COLI_OK
+             : COLI_ERR_CUDA;
 }
 
 coli_status coli_moe_layer_noalloc(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,

@@ -70,6 +70,14 @@ struct FfnArgs {
   uint16_t* out;
   uint32_t* status;
   int H, I, T, k, E, S, P;
+  // expert-parallel rank (split-K form): the weights hold routed experts
+  // [e_off, e_off + n) at rows 0.. and the S shared ones from expert e_shared
+  // on; pairs whose expert (topk_ids) is not among them add nothing; with
+  // out_f32 the output is the unrounded fp32 partial sum (else e_off = 0,
+  // e_shared = E, topk_ids and out_f32 NULL)
+  int e_off, e_end, e_shared;
+  const int32_t* topk_ids;
+  float* out_f32;
 };
 
 // Shared-memory layout constants.  KC elements of K per stage; NT n-tiles of 8
@@ -272,12 +280,12 @@ __device__ __forceinline__ TileInfo decode_tile(const FfnArgs& a, const Meta& m,
   if (lo >= m.S) {
     const int u = lo - m.S;
     ti.routed = true;
-    ti.e = m.unique[u];
+    ti.e = m.unique[u] - a.e_off;
     ti.base = m.seg_off[u];
     ti.cnt = m.seg_off[u + 1] - ti.base;
   } else {
     ti.routed = false;
-    ti.e = a.E + lo;
+    ti.e = a.e_shared + lo;
     ti.base = a.P + lo * a.T;
     ti.cnt = a.T;
   }

@@ -643,7 +643,13 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* 
       const int row = j < a.k ? pos[t * a.k + j] : a.P + (j - a.k) * a.T + t;
       const float* src = a.ypart + static_cast<size_t>(row) * nsl * a.H + r;
       float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < nsl; s0 += 16) {
+      // an expert-parallel rank adds only the pairs of its own experts
+      bool here = true;
+      if (a.topk_ids && j < a.k) {
+        const int e = __ldg(a.topk_ids + t * a.k + j);
+        here = e >= a.e_off && e < a.e_end;
+      }
+      for (int s0 = 0; here && s0 < nsl; s0 += 16) {
         float4 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -689,6 +695,10 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* 
         acc.y += __uint_as_float(rv.x & 0xffff0000u);
         acc.z += __uint_as_float(rv.y << 16);
         acc.w += __uint_as_float(rv.y & 0xffff0000u);
+      }
+      if (a.out_f32) {
+        *reinterpret_cast<float4*>(a.out_f32 + static_cast<size_t>(t) * a.H + r) = acc;
+        continue;
       }
       uint2 o;
       o.x = float_to_bf16_bits(acc.x) | (static_cast<uint32_t>(float_to_bf16_bits(acc.y)) << 16);
@@ -780,7 +790,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     if (static_cast<int>(blockIdx.x) < a.S * nrb_gu) {
       const int nkc = a.H / F::D::KCG;
       pre = nkc < NS ? nkc : NS;
-      const int row0 = (a.E + static_cast<int>(blockIdx.x) / nrb_gu) * a.I + (blockIdx.x % nrb_gu) * kRowBlock;
+      const int row0 = (a.e_shared + static_cast<int>(blockIdx.x) / nrb_gu) * a.I + (blockIdx.x % nrb_gu) * kRowBlock;
       if (lane == 0) {
         const uint64_t cpol = l2_policy_evict_first();
         for (int kc = 0; kc < pre; ++kc)

@@ -430,7 +430,7 @@ __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, in
                                                 int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
                                                 int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status,
                                                 int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
-                                                int32_t* __restrict__ rb_done, int n_rb, int lane) {
+                                                int32_t* __restrict__ rb_done, int n_rb, int lane, int eb, int ee) {
   int key[4];
   bool bad = false;
 #pragma unroll
@@ -498,9 +498,12 @@ __device__ __forceinline__ void warp_union_plan(const int* ids, int P, int E, in
     if (sidx < S) {
       v = (T + tokb - 1) / tokb;
     } else if (sidx < S + U) {
+      // routed segments of experts outside [eb, ee) get no blocks (an expert-parallel
+      // rank computes its own experts only)
       const int uu = sidx - S;
       const int c = ((uu + 1 < U) ? seg_off[uu + 1] : Pv) - seg_off[uu];
-      v = (c + tokb - 1) / tokb;
+      const int eid = unique_ids[uu];
+      v = (eid >= eb && eid < ee) ? (c + tokb - 1) / tokb : 0;
     }
     nb[q] = v;
     lsum += v;
@@ -539,7 +542,7 @@ __device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, 
                                                   int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
                                                   int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status,
                                                   int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
-                                                  int32_t* __restrict__ rb_done, int n_rb, int lane) {
+                                                  int32_t* __restrict__ rb_done, int n_rb, int lane, int eb, int ee) {
   int key = 0x7fffffff;
   bool bad = false;
   if (lane < P) {
@@ -580,7 +583,8 @@ __device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, 
   }
   // plan: S shared segments of T tokens, then the U routed ones in order
   const int nb_shared = (T + tokb - 1) / tokb;
-  int nb = start ? (cnt + tokb - 1) / tokb : 0;
+  // (routed segments of experts outside [eb, ee) get no blocks)
+  int nb = (start && (key >> 8) >= eb && (key >> 8) < ee) ? (cnt + tokb - 1) / tokb : 0;
   int incl = nb;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -606,14 +610,17 @@ __device__ __forceinline__ void warp_union_plan32(const int* ids, int P, int E, 
 }
 
 // Route + union + plan for T*k <= 128: warp w routes tokens w, w + nwarps, ...;
-// then warp 0 alone builds the union and the plan.
+// then warp 0 alone builds the union and the plan.  The union covers every
+// selected expert; the plan gives blocks to the S shared segments and to the
+// routed experts in [eb, ee) only (the whole range [0, E) except on an
+// expert-parallel rank).
 template <int NV>
 __global__ void __launch_bounds__(256) route_union_small_kernel(
     const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
     int32_t* __restrict__ ids_out, float* __restrict__ w_out, int32_t* __restrict__ unique_ids,
     int32_t* __restrict__ n_unique, int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
     int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status, int S, int tokb, int32_t* __restrict__ plan,
-    int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done, int n_rb) {
+    int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done, int n_rb, int eb, int ee) {
   __shared__ int ids_s[kWarpUnionMaxP];
   pdl_wait();
   pdl_trigger();
@@ -634,10 +641,10 @@ __global__ void __launch_bounds__(256) route_union_small_kernel(
   if (warp == 0) {
     if (T * k <= 32)
       warp_union_plan32(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan,
-                        tb_done, rb_done, n_rb, lane);
+                        tb_done, rb_done, n_rb, lane, eb, ee);
     else
       warp_union_plan(ids_s, T * k, E, T, S, tokb, unique_ids, n_unique, seg_off, perm, pair_pos, status, plan,
-                      tb_done, rb_done, n_rb, lane);
+                      tb_done, rb_done, n_rb, lane, eb, ee);
   }
 }
 
