@@ -449,7 +449,7 @@ bool launch_route_union(const float* lg, const float* bias, int T, int E, int k,
   const dim3 g(1), b(kUnionThreads);
 #define COLI_RU(NV)                                                                                            \
   launch(route_union_kernel<NV>, g, b, smem, st, lg, bias, T, E, k, ids, w, ws.unique, ws.n_unique, ws.seg_off, \
-         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb)
+         ws.perm, ws.pair_pos, status, S, tokb, ws.plan, ws.tb_done, ws.rb_done, n_rb, eb, ee)
   switch (route_nv(E)) {
     case 1: return COLI_RU(1);
     case 2: return COLI_RU(2);
@@ -592,7 +592,8 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
     long blocks = (work + 255) / 256;
     if (blocks > 4L * di.sms) blocks = 4L * di.sms;
     if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
-                pair_pos, topk_w, residual, T, k, S, H, out))
+                pair_pos, topk_w, residual, T, k, S, H, out, static_cast<const int32_t*>(nullptr), 0, E,
+                static_cast<float*>(nullptr)))
       return COLI_ERR_CUDA;
   }
   rec.mark(8);
@@ -719,7 +720,8 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
     long blocks = (work + 255) / 256;
     if (blocks > 4L * di.sms) blocks = 4L * di.sms;
     if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
-                pair_pos, topk_w, residual, T, k, S, H, out))
+                pair_pos, topk_w, residual, T, k, S, H, out, ep.on ? ep.ids : static_cast<const int32_t*>(nullptr),
+                ep.on ? ep.begin : 0, ep.on ? ep.end : E, ep.on ? ep.out_f32 : static_cast<float*>(nullptr)))
       return COLI_ERR_CUDA;
   }
   rec.mark(8);
@@ -895,9 +897,10 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
-  // an expert-parallel share runs in the split-K decode form only
-  if (ep.on && !(form == Form::kDecode && use_splitk(dims, T) && T <= kFusedRouteMaxT &&
-                 T * dims->top_k <= kWarpUnionMaxP))
+  // an expert-parallel share runs in the decode forms, with route, union and
+  // plan in one kernel (T <= 128), and not through the two-phase kernel's
+  // own combine (T <= 4 with I = 128)
+  if (ep.on && !(form == Form::kDecode && T <= kFusedRouteMaxT && (use_splitk(dims, T) || T > kFusedCombineMaxT)))
     return COLI_ERR_UNSUPPORTED;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;

@@ -750,12 +750,16 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
 }
 
 // out[t, n] = bf16( sum_{j<k} w[t,j] * y[pair_pos[t*k+j], n] + sum_s y[P + s*T + t, n]
-//                   + residual[t, n] ), fp32, in exactly this order.
+//                   + residual[t, n] ), fp32, in exactly this order.  With ids (an
+// expert-parallel rank) only the slots whose expert is in [eb, ee) are added;
+// with out_f32 the fp32 sum is written there, unrounded, instead of out.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ ypair,
                                                       const int32_t* __restrict__ pair_pos,
                                                       const float* __restrict__ w,
                                                       const uint16_t* __restrict__ residual, int T, int k,
-                                                      int S, int H, uint16_t* __restrict__ out) {
+                                                      int S, int H, uint16_t* __restrict__ out,
+                                                      const int32_t* __restrict__ ids, int eb, int ee,
+                                                      float* __restrict__ out_f32) {
   pdl_wait();
   pdl_trigger();
   const int per_tok = H / 4;
@@ -776,6 +780,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         const int j = j0 + q;
         pp[q] = j < k ? __ldg(pair_pos + t * k + j) : -1;
         wt[q] = j < k ? __ldg(w + t * k + j) : 0.f;
+        if (ids && j < k) {
+          // an expert-parallel rank adds only the pairs of its own experts
+          const int e = __ldg(ids + t * k + j);
+          if (e < eb || e >= ee) pp[q] = -1;
+        }
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -805,6 +814,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       acc.y += __uint_as_float(r.x & 0xffff0000u);
       acc.z += __uint_as_float(r.y << 16);
       acc.w += __uint_as_float(r.y & 0xffff0000u);
+    }
+    if (out_f32) {
+      *reinterpret_cast<float4*>(out_f32 + static_cast<size_t>(t) * H + n) = acc;
+      continue;
     }
     uint2 o;
     o.x = float_to_bf16_bits(acc.x) | (static_cast<uint32_t>(float_to_bf16_bits(acc.y)) << 16);

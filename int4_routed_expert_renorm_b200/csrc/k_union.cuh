@@ -130,7 +130,7 @@ __device__ __forceinline__ int block_union(const int32_t* ids, int P, int E, int
 // rb_done per output row block) for this call.
 __device__ __forceinline__ void block_plan(int U, const int* seg_cnt, int T, int S, int tokb, int* scratch,
                                            int32_t* __restrict__ plan, int32_t* __restrict__ tb_done,
-                                           int32_t* __restrict__ rb_done, int n_rb) {
+                                           int32_t* __restrict__ rb_done, int n_rb, const int32_t* unique_ids = nullptr, int eb = 0, int ee = 0x7fffffff) {
   __shared__ int carry;
   const int n_seg = U + S;
   if (threadIdx.x == 0) carry = 0;
@@ -139,7 +139,11 @@ __device__ __forceinline__ void block_plan(int U, const int* seg_cnt, int T, int
     const int u = u0 + threadIdx.x;
     int nb = 0;
     if (u < S) nb = (T + tokb - 1) / tokb;
-    else if (u < n_seg) nb = (seg_cnt[u - S] + tokb - 1) / tokb;
+    else if (u < n_seg) {
+      // routed segments of experts outside [eb, ee) get no blocks (expert-parallel rank)
+      const int eid = unique_ids ? unique_ids[u - S] : eb;
+      nb = (eid >= eb && eid < ee) ? (seg_cnt[u - S] + tokb - 1) / tokb : 0;
+    }
     int tot = 0;
     const int ex = block_exclusive_scan(nb, scratch, &tot);
     const int c = carry;
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
                        int32_t* __restrict__ n_unique, int32_t* __restrict__ seg_off, int32_t* __restrict__ perm,
                        int32_t* __restrict__ pair_pos, uint32_t* __restrict__ status, int S, int tokb,
                        int32_t* __restrict__ plan, int32_t* __restrict__ tb_done, int32_t* __restrict__ rb_done,
-                       int n_rb) {
+                       int n_rb, int eb, int ee) {
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   int* ids_s = smem_i + kUnionWarps * E;
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kUnionThreads, 1)
   __syncthreads();
   const int U = block_union(ids_s, T * k, E, hist, scratch, seg_cnt, unique_ids, n_unique, seg_off, perm, pair_pos,
                             status);
-  block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb);
+  block_plan(U, seg_cnt, T, S, tokb, scratch, plan, tb_done, rb_done, n_rb, unique_ids, eb, ee);
 }
 
 // ---------------------------------------------------------------------------
