@@ -70,33 +70,39 @@ def parse():
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture, with a digest of the kernel sources that capture ran on:
-# (workload, FFN form) -> bytes.  While the sources differ from that digest
-# (a kernel changed since the counters were taken) the line reports null.
-# The batch-1 capture ran on the 16-expert variant of the layer, which moves
-# the same 9 experts per step; the prefill capture on the 32-expert, 512-token
-# variant (same tile shapes), where DRAM traffic was 1.064x the algorithmic
-# bytes of the gate/up launch; the 4096-token figure is that ratio times its
-# own algorithmic bytes (257 experts' gate+up codes and scales, 36,864
-# gathered rows, h written).
-TRAFFIC_SOURCES = "47033e5dc090e639"
-_PF_RATIO = (532.682752e6 + 16.870912e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
-TRAFFIC = {("glm52_layer_decode_b1", "decode"): 191.315200e6 + 4.964096e6,
-           ("glm52_layer_decode_b1_e16", "decode"): 191.315200e6 + 4.964096e6,
-           ("glm52_layer_prefill_512_e32", "prefill"): 532.682752e6 + 16.870912e6,
-           ("glm52_layer_prefill_4096", "prefill"):
-               _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2),
+# (workload, FFN form) -> (bytes, digest).  While the sources differ from that
+# digest (a kernel changed since the counters were taken) the line reports
+# null.  The batch-1 capture ran on the 16-expert variant of the layer, which
+# moves the same 9 experts per step; the prefill capture on the 32-expert,
+# 512-token variant (same tile shapes), where DRAM traffic was 1.062x the
+# algorithmic bytes of the gate/up launch; the 4096-token figure is that ratio
+# times its own algorithmic bytes (257 experts' gate+up codes and scales,
+# 36,864 gathered rows, h written).
+_SK_SOURCES = "9c400c5040a29e13"
+_PF_SOURCES = "552c12e296d31c08"
+_PF_RATIO = (532.615680e6 + 16.172544e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
+_PF_4096 = _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)
+TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.344896e6 + 5.110528e6, _SK_SOURCES),
+           ("glm52_layer_decode_b1_e16", "decode"): (191.344896e6 + 5.110528e6, _SK_SOURCES),
+           ("glm52_layer_prefill_512_e32", "prefill"): (532.615680e6 + 16.172544e6, _PF_SOURCES),
+           ("glm52_layer_prefill_4096", "prefill"): (_PF_4096, _PF_SOURCES),
            # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
-           ("glm52_layer_prefill_4096_router", "prefill"):
-               _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)}
+           ("glm52_layer_prefill_4096_router", "prefill"): (_PF_4096, _PF_SOURCES)}
+# the sources each captured kernel is built from
+_KERNEL_FILES = {"decode": ("common.cuh", "k_ffn_decode.cuh", "k_ffn_splitk.cuh"),
+                 "prefill": ("common.cuh", "k_ffn_decode.cuh", "k_ffn_prefill.cuh")}
 
 
-def kernel_sources_digest() -> str:
-    """First 16 hex digits of the sha256 over the library's kernel sources
-    (file name, then contents, in name order)."""
+def kernel_sources_digest(files=None) -> str:
+    """First 16 hex digits of the sha256 over the named kernel sources (all of
+    them by default): file name, then contents, in name order."""
     import glob
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "int4_routed_expert_renorm_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "int4_routed_expert_renorm_b200", "csrc")
+    paths = sorted(glob.glob(os.path.join(csrc, "*"))) if files is None else sorted(
+        os.path.join(csrc, f) for f in files)
+    for f in paths:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
@@ -105,10 +111,11 @@ def kernel_sources_digest() -> str:
 
 def traffic_for(workload: str, form: str):
     """The captured DRAM bytes per launch, or None when there is no capture of
-    the current kernel sources."""
-    if kernel_sources_digest() != TRAFFIC_SOURCES:
+    the current sources of that kernel."""
+    entry = TRAFFIC.get((workload, form))
+    if entry is None or kernel_sources_digest(_KERNEL_FILES[form]) != entry[1]:
         return None
-    return TRAFFIC.get((workload, form))
+    return entry[0]
 
 
 def splitk_form(shape) -> bool:

@@ -115,3 +115,23 @@ def test_expert_parallel_glm_shape(lib, T, world):
     assert err <= OUT_REL_TOL
     del full
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("kw", [dict(tokens=4, group=64), dict(tokens=40, group=64), dict(tokens=6, bits=8)],
+                         ids=["gs64-splitk", "gs64-two-phase", "int8"])
+def test_expert_parallel_containers(lib, kw):
+    """The gs64 and int8 containers through the expert-parallel share."""
+    shape = _small_shape(hidden=512, inter=512, n_experts=12, top_k=3, n_shared=1, **kw)
+    T = shape.tokens
+    full = sg.expert_tensors(shape, 24)
+    li = synth.LayerInputs(shape, 24)
+    x = synth.normal_bf16(24, 5, synth.X_IN, (T, 512))
+    out, _, routing = _ep_run(lib, shape, full, li, x, 3, x)
+    ref_out, ref_routing = _whole(lib, shape, full, li, x, x)
+    for lg, ids, w in routing:
+        assert np.array_equal(ids, ref_routing[1]) and np.array_equal(w, ref_routing[2])
+    W = oracle_weights(shape, seed=24)
+    ref = oracle.moe_ffn_combine(W, x, ref_routing[1], ref_routing[2], shape.n_experts, shape.n_shared, x)
+    err = _rel(out, ref)
+    print(f"expert-parallel {kw}: vs oracle {err:.3e}, vs the whole layer {_rel(out, ref_out):.3e}")
+    assert err <= OUT_REL_TOL and _rel(out, ref_out) <= OUT_REL_TOL
