@@ -127,8 +127,10 @@ coli_status dev_info(DevInfo* out) {
     COLI_SET_PF_SMEM(2, 64, false)
     COLI_SET_PF_SMEM(2, 64, true)
 #undef COLI_SET_PF_SMEM
-#define COLI_SET_SK_SMEM(NT, GR, B)                                                                        \
-  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<NT, GR, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define COLI_SET_SK_SMEM(NT, GR, B)                                                                           \
+  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<NT, GR, B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(SkCfg<GR, B>::SMEM)) == cudaSuccess;                           \
+  ok &= cudaFuncSetAttribute(ffn_splitk_kernel<NT, GR, B, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                              static_cast<int>(SkCfg<GR, B>::SMEM)) == cudaSuccess;
     COLI_SET_SK_SMEM(1, 32, 4)
     COLI_SET_SK_SMEM(2, 32, 4)
@@ -613,10 +615,30 @@ struct EpRange {
   float* out_f32 = nullptr;
 };
 
+// The split-K kernel's own routing (logits not NULL): the batch's router
+// logits and bias, and where the ids and weights go; the union and the plan
+// go to the workspace arrays as a routing kernel would write them.
+struct InRoute {
+  const float* logits = nullptr;
+  const float* bias = nullptr;
+  int32_t* ids = nullptr;
+  float* w = nullptr;
+};
+
+// The split-K kernel routes the batch itself for 2 to 8 tokens when one warp
+// can sort the pairs and route a token (T*k <= 128, E <= 256).  A single token
+// is routed by its own kernel: measured on the GLM-5.2-shaped layer, the
+// in-kernel routing made the batch-1 step slower (about 2 us of 65) and the
+// 4-token stack faster (about 3 %).
+inline bool splitk_routes(const coli_moe_dims* d, int T) {
+  return T >= 2 && use_splitk(d, T) && T * d->top_k <= kWarpUnionMaxP && d->n_experts <= 256;
+}
+
 coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
                     const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
                     const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
-                    cudaStream_t st, const StageRecorder& rec, const EpRange& ep = EpRange()) {
+                    cudaStream_t st, const StageRecorder& rec, const EpRange& ep = EpRange(),
+                    const InRoute& ir = InRoute()) {
   const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k;
   const int S = ep.on ? ep.shared : d->n_shared;
   const int E_w = ep.on ? ep.end - ep.begin : E;   // routed experts held by the weights
@@ -671,6 +693,19 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
   a.e_shared = E_w;
   a.topk_ids = ep.on ? ep.ids : nullptr;
   a.out_f32 = ep.on ? ep.out_f32 : nullptr;
+  a.tokb = tokb;
+  if (ir.logits) {
+    a.r_logits = ir.logits;
+    a.r_bias = ir.bias;
+    a.r_ids = ir.ids;
+    a.r_w = ir.w;
+    a.r_unique = ws.unique;
+    a.r_n_unique = ws.n_unique;
+    a.r_seg_off = ws.seg_off;
+    a.r_perm = ws.perm;
+    a.r_pair_pos = ws.pair_pos;
+    a.r_plan = ws.plan;
+  }
   if (use_splitk(d, T)) {
     // down maps of the split-K form: codes in boxes of 128 rows x one
     // 128-wide K slice (64 bytes, 64B swizzle; int8: 128 bytes, 128B
@@ -690,15 +725,15 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
     const bool nt2 = T > 4;
     FfnKernel k;
     size_t smem;
+#define COLI_SK(NT, GR, B) (ir.logits ? ffn_splitk_kernel<NT, GR, B, true> : ffn_splitk_kernel<NT, GR, B, false>)
     if (B == 4) {
-      k = nt2 ? (G == 32 ? ffn_splitk_kernel<2, 32, 4> : ffn_splitk_kernel<2, 64, 4>)
-              : (G == 32 ? ffn_splitk_kernel<1, 32, 4> : ffn_splitk_kernel<1, 64, 4>);
+      k = nt2 ? (G == 32 ? COLI_SK(2, 32, 4) : COLI_SK(2, 64, 4)) : (G == 32 ? COLI_SK(1, 32, 4) : COLI_SK(1, 64, 4));
       smem = G == 32 ? SkCfg<32, 4>::SMEM : SkCfg<64, 4>::SMEM;
     } else {
-      k = nt2 ? (G == 32 ? ffn_splitk_kernel<2, 32, 8> : ffn_splitk_kernel<2, 64, 8>)
-              : (G == 32 ? ffn_splitk_kernel<1, 32, 8> : ffn_splitk_kernel<1, 64, 8>);
+      k = nt2 ? (G == 32 ? COLI_SK(2, 32, 8) : COLI_SK(2, 64, 8)) : (G == 32 ? COLI_SK(1, 32, 8) : COLI_SK(1, 64, 8));
       smem = G == 32 ? SkCfg<32, 8>::SMEM : SkCfg<64, 8>::SMEM;
     }
+#undef COLI_SK
     if (!launch_splitk(k, smem, maps, a, grid, di.sms, st)) return COLI_ERR_CUDA;
     rec.mark_through(6, 7);
     rec.mark(8);
@@ -912,6 +947,8 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const StageRecorder rec(s);
   rec.mark(0);
   const int S = dims->n_shared, tokb = tok_block(T);
+  // the split-K kernel routes the batch itself: no routing kernel runs
+  const bool inroute = form == Form::kDecode && splitk_routes(dims, T);
 
   // 1. expert input (fragment order, optional pre-norm) and router logits
   float* lo = logits_out ? logits_out : lay.logits;
@@ -921,7 +958,7 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
     const float* wr = logits_in ? nullptr : w->router_w;
     const int grid = (logits_in ? 0 : E) + T;
     if (!launch(front_kernel, dim3(grid), dim3(256), 0, s, x, wr, T, E, H, prenorm ? 1 : 0, lo, lay.xn, lay.xq,
-                lay.xp, lay.xe, form == Form::kPrefill ? 1 : 0, di.status))
+                lay.xp, lay.xe, form == Form::kPrefill ? 1 : 0, di.status, inroute ? lay.rb_done : nullptr))
       return COLI_ERR_CUDA;
     rec.mark_through(1, 2);
     if (!logits_in) lg = lo;
@@ -956,7 +993,9 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   // 2. route, union and the FFN tile plan
   int32_t* ids = topk_ids_out ? topk_ids_out : lay.ids;
   float* tw = topk_w_out ? topk_w_out : lay.w;
-  if (T <= kFusedRouteMaxT) {
+  if (inroute) {
+    rec.mark_through(3, 5);
+  } else if (T <= kFusedRouteMaxT) {
     if (!launch_route_union(lg, w->router_bias, T, E, k, ep.on ? ep.shared : S, tokb, H / kRowBlock, ids, tw, lay,
                             di.status, s, ep.on ? ep.begin : 0, ep.on ? ep.end : E))
       return COLI_ERR_CUDA;
@@ -988,8 +1027,15 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
     return run_ffn_prefill(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual,
                            out, lay, di, s, rec);
   ep.ids = ids;
+  InRoute ir;
+  if (inroute) {
+    ir.logits = lg;
+    ir.bias = w->router_bias;
+    ir.ids = ids;
+    ir.w = tw;
+  }
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
-                 di, s, rec, ep);
+                 di, s, rec, ep, ir);
 }
 
 }  // namespace

@@ -78,6 +78,23 @@ struct FfnArgs {
   int e_off, e_end, e_shared;
   const int32_t* topk_ids;
   float* out_f32;
+  // split-K form with the routing in the kernel (r_logits not NULL; T*k <=
+  // 128 and E <= 256): the batch's router logits [T][E] and bias; every CTA
+  // routes the batch and builds the union and the tile plan (tokb tokens per
+  // block) in shared memory, and CTA 0 also writes them, the ids and the
+  // weights to the arrays below.  With r_logits NULL they come from an
+  // earlier kernel through the const pointers above.
+  const float* r_logits;
+  const float* r_bias;
+  int32_t* r_ids;
+  float* r_w;
+  int32_t* r_unique;
+  int32_t* r_n_unique;
+  int32_t* r_seg_off;
+  int32_t* r_perm;
+  int32_t* r_pair_pos;
+  int32_t* r_plan;
+  int tokb;
 };
 
 // Shared-memory layout constants.  KC elements of K per stage; NT n-tiles of 8

@@ -90,7 +90,7 @@ struct SkCfg {
   static constexpr int H_BYTES = kSkMaxT * kSkHRow;                    // h slice, bf16, natural order
   static constexpr int HP_BYTES = kSkMaxT * kSkHGroups * kPlaneRec;    // its plane records
   static constexpr int HMAX_BYTES = kRowWarps * kSkMaxT * 4 + kSkMaxT * 4;
-  static constexpr int ROUTE_BYTES = 3 * kSkMaxP * 4 + 16;   // routing weights, perm, pair_pos; U
+  static constexpr int ROUTE_BYTES = 4 * kSkMaxP * 4 + 16;   // routing weights, perm, pair_pos, ids; U
   static constexpr int NBAR = 64;
   static constexpr int FIXED =
       RED_BYTES + META_BYTES + H_BYTES + HP_BYTES + HMAX_BYTES + ROUTE_BYTES + 1024 + NBAR * 8 + 64;
@@ -105,6 +105,8 @@ struct SkCfg {
   static_assert(META_BYTES % 16 == 0 && H_BYTES % 16 == 0 && HP_BYTES % 16 == 0, "shared regions stay aligned");
   // the combine stages its pairs' y (k + S <= 36 per 4-row unit) in the stage ring
   static_assert(NS * STAGE >= 36 * 16, "combine staging");
+  // the in-kernel routing stages the router bias (E <= 256) in red
+  static_assert(RED_BYTES >= 256 * 4, "bias staging");
 };
 
 // Integer MMA of one 32-wide group: d = A * B + C with C = {c_lo, c_hi} in
@@ -622,8 +624,8 @@ __device__ __forceinline__ bool wait_counter(const int32_t* cnt, int target, vol
 // topk_w.  `cbar` (count: consumer warps) separates the passes; returns
 // false on a timeout.
 __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* pos, const float* w,
-                                               uint8_t* ring, int ring_bytes, uint64_t* cbar, uint32_t& cph,
-                                               volatile int* abort_flag, int warp, int lane) {
+                                               const int32_t* ids, uint8_t* ring, int ring_bytes, uint64_t* cbar,
+                                               uint32_t& cph, volatile int* abort_flag, int warp, int lane) {
   const int tid = warp * 32 + lane;
   const int nthr = kFfnConsumerWarps * 32;
   const int q4 = a.H / 4;
@@ -646,7 +648,7 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* 
       // an expert-parallel rank adds only the pairs of its own experts
       bool here = true;
       if (a.topk_ids && j < a.k) {
-        const int e = __ldg(a.topk_ids + t * a.k + j);
+        const int e = ids ? ids[t * a.k + j] : __ldg(a.topk_ids + t * a.k + j);
         here = e >= a.e_off && e < a.e_end;
       }
       for (int s0 = 0; here && s0 < nsl; s0 += 16) {
@@ -714,12 +716,46 @@ __device__ __forceinline__ bool splitk_combine(const FfnArgs& a, const int32_t* 
   return true;
 }
 
+// The split-K kernel's own routing (a.r_logits not NULL), kept out of line so
+// that it does not change the code of the kernel's main loops.  Warp t routes
+// token t (top-k, lowest index on ties, renormalised softmax); then warp 0
+// sorts the pairs into the union and lays out the plan, all in shared memory.
+// Every CTA computes the same from the same logits.
+__device__ __noinline__ void splitk_route(const FfnArgs& a, const float* bias_s, int32_t* ids_s, float* w_s,
+                                          int32_t* muniq, int32_t* n_unique_s, int32_t* mseg, int32_t* perm_s,
+                                          int32_t* pos_s, int32_t* mplan, int warp, int lane) {
+  const int P = a.T * a.k;
+  __syncthreads();
+  if (warp < a.T) {
+    int id;
+    float wt;
+    const bool bad = route_token<8, true>(a.r_logits + static_cast<size_t>(warp) * a.E, a.r_bias ? bias_s : nullptr, a.E,
+                                    a.k, lane, &id, &wt);
+    if (lane < a.k) {
+      ids_s[warp * a.k + lane] = id;
+      w_s[warp * a.k + lane] = wt;
+    }
+    if (bad && blockIdx.x == 0 && lane == 0) atomicOr(a.status, COLI_FLAG_NONFINITE);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t* st = blockIdx.x == 0 ? a.status : nullptr;
+    if (P <= 32)
+      warp_union_plan32(ids_s, P, a.E, a.T, a.S, a.tokb, muniq, n_unique_s, mseg, perm_s, pos_s, st, mplan, nullptr,
+                        nullptr, 0, lane, a.e_off, a.e_end);
+    else
+      warp_union_plan(ids_s, P, a.E, a.T, a.S, a.tokb, muniq, n_unique_s, mseg, perm_s, pos_s, st, mplan, nullptr,
+                      nullptr, 0, lane, a.e_off, a.e_end);
+  }
+}
+
 // The split-K FFN kernel.  At most one CTA per SM, all resident (the final
 // grid-wide wait needs that); a.rb_done[0] is the zeroed arrival counter.  NT: MMA
-// n-tiles of four tokens (1 for T <= 4, 2 for T <= 8).  The union, the tile
-// plan, the routing weights and the pair positions come from earlier kernels
-// and are copied into shared memory.
-template <int NT, int GROUP, int BITS>
+// n-tiles of four tokens (1 for T <= 4, 2 for T <= 8).  INROUTE: every CTA
+// routes the batch from the router logits (a.r_logits) and builds the union and
+// the tile plan itself; otherwise they come from earlier kernels.  Either way
+// they are kept in shared memory.
+template <int NT, int GROUP, int BITS, bool INROUTE>
 __global__ void __launch_bounds__(kFfnThreads, 1)
     ffn_splitk_kernel(const __grid_constant__ CUtensorMap gq, const __grid_constant__ CUtensorMap uq,
                       const __grid_constant__ CUtensorMap gs, const __grid_constant__ CUtensorMap us,
@@ -740,7 +776,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   float* w_s = reinterpret_cast<float*>(hb.hp + F::HP_BYTES + F::HMAX_BYTES);
   int32_t* perm_s = reinterpret_cast<int32_t*>(w_s + kSkMaxP);
   int32_t* pos_s = perm_s + kSkMaxP;
-  int32_t* n_unique_s = pos_s + kSkMaxP;
+  int32_t* ids_s = pos_s + kSkMaxP;
+  int32_t* n_unique_s = ids_s + kSkMaxP;
   uint64_t* full = reinterpret_cast<uint64_t*>(hb.hp + F::HP_BYTES + F::HMAX_BYTES + F::ROUTE_BYTES);
   uint64_t* empty = full + NS;
   uint64_t* red_full = empty + NS;
@@ -799,13 +836,19 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       }
     }
   }
+  const int P = a.T * a.k;
+  // the router bias is no output of an earlier kernel: staged before the wait
+  float* bias_s = red;
+  if (INROUTE && a.r_bias)
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) bias_s[i] = __ldg(a.r_bias + i);
   pdl_wait();
   pdl_trigger();
-  {
+  if constexpr (INROUTE) {
+    splitk_route(a, bias_s, ids_s, w_s, muniq, n_unique_s, mseg, perm_s, pos_s, mplan, warp, lane);
+  } else {
     // every array in one round of loads, up to its allocated size (the union
     // of P pairs has at most Umax = min(E, P) experts), not to the sizes the
     // routing kernel reports, so no load waits on another
-    const int P = a.T * a.k;
     const int Umax = P < a.E ? P : a.E;
     if (threadIdx.x == 0) *n_unique_s = __ldg(a.n_unique);
     for (int i = threadIdx.x; i < Umax + a.S + 3; i += blockDim.x) mplan[i] = __ldg(a.plan + i);
@@ -860,6 +903,21 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   }
 
   // ---------------- consumers ----------------
+  if (INROUTE && blockIdx.x == 0) {
+    // publish the union and the plan this CTA built (plain stores: nothing
+    // in this kernel reads them back)
+    const int tid = threadIdx.x, nthr = kFfnConsumerWarps * 32;
+    for (int i = tid; i < m.U; i += nthr) a.r_unique[i] = muniq[i];
+    for (int i = tid; i <= m.U; i += nthr) a.r_seg_off[i] = mseg[i];
+    for (int i = tid; i < m.n_seg + 3; i += nthr) a.r_plan[i] = mplan[i];
+    for (int i = tid; i < P; i += nthr) {
+      a.r_perm[i] = perm_s[i];
+      a.r_pair_pos[i] = pos_s[i];
+      a.r_ids[i] = ids_s[i];
+      a.r_w[i] = w_s[i];
+    }
+    if (tid == 0) *a.r_n_unique = m.U;
+  }
   int s = 0;
   uint32_t ph = 0, rph = 0, lu = 0;
   for (int t = blockIdx.x; t < m.tiles_gu; t += gridDim.x, ++lu) {
@@ -886,7 +944,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   if (!mbar_wait(gbar, 0, abort_flag, a.status)) return;
   // (the combine's CTA barriers are cbar's next phases)
   uint32_t cph = 1;
-  splitk_combine(a, pos_s, w_s, smem, NS * STAGE, cbar, cph, abort_flag, warp, lane);
+  splitk_combine(a, pos_s, w_s, INROUTE ? ids_s : nullptr, smem, NS * STAGE, cbar, cph, abort_flag, warp, lane);
 }
 
 }  // namespace coli

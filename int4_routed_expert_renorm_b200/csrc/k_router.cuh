@@ -392,14 +392,17 @@ __global__ void __launch_bounds__(256) logits_mma_kernel(const uint16_t* __restr
 // grid exponent), so that no block does both.  With
 // prenorm every block normalises its tokens itself (n = bf16(x * r) with
 // r = 1/sqrt(mean(x^2) + 1e-6) summed in the same order as prep_kernel), so
-// the logits see exactly the normalised input the experts see.
+// the logits see exactly the normalised input the experts see.  Block 0
+// zeroes *zero_ctr when it is not NULL (the arrival counter of a split-K FFN
+// kernel that routes the batch itself, so that no routing kernel runs between).
 __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                                                     int T, int E, int H, int prenorm, float* __restrict__ logits,
                                                     uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
                                                     uint8_t* __restrict__ xp, int32_t* __restrict__ xe, int xq_f16,
-                                                    uint32_t* __restrict__ status) {
+                                                    uint32_t* __restrict__ status, int32_t* __restrict__ zero_ctr) {
   pdl_wait();
   pdl_trigger();
+  if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
   const int nlog = wr ? E : 0;   // blocks [0, nlog): logits of expert b; then one block per token
   __shared__ float red[8][8];
   __shared__ float rs[64];
@@ -557,10 +560,21 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
 // w_j = exp(l_j - l_max) / sum_{i<k} exp(l_i - l_max), summed in slot order.
 // NaN ranks as -inf; NaN or +inf anywhere, or a selected -inf, returns bad.
 // Lane j < k gets slot j in *id / *w.
-template <int NV>
+// PRELOAD: every logit and bias load is issued before any arithmetic (the
+// split-K kernel's own routing, where the logits come from L2); the same
+// values and decisions either way.
+template <int NV, bool PRELOAD = false>
 __device__ __forceinline__ bool route_token(const float* __restrict__ lr, const float* __restrict__ bias, int E,
                                             int k, int lane, int* id, float* w) {
-  float v[NV];
+  float v[NV], bq[NV];
+  if constexpr (PRELOAD) {
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = e < E ? lr[e] : 0.f;
+      bq[q] = (bias && e < E) ? bias[e] : 0.f;
+    }
+  }
   uint32_t taken = 0;
   bool bad = false;
 #pragma unroll
@@ -568,8 +582,8 @@ __device__ __forceinline__ bool route_token(const float* __restrict__ lr, const 
     const int e = lane + 32 * q;
     float val = -INFINITY;
     if (e < E) {
-      val = lr[e];
-      if (bias) val = val + bias[e];
+      val = PRELOAD ? v[q] : lr[e];
+      if (bias) val = val + (PRELOAD ? bq[q] : bias[e]);
       if (isnan(val)) {
         bad = true;
         val = -INFINITY;

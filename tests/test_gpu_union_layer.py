@@ -1,9 +1,12 @@
 """Bit-exact parity of the batch-union that coli_moe_layer itself computes.
 
-The layer does not call coli_moe_union: small batches route and unite in one
-warp (T*k <= 32 and <= 128 take two different sorts), batches up to 128
-tokens in one CTA, larger decode batches in the route + union kernels, and
-prefill batches in a many-CTA counting sort.  Each of these leaves its
+The layer does not call coli_moe_union: batches of 2 to 8 tokens (T*k <=
+128, E <= 256) are routed and united by every CTA of the split-K kernel
+itself (CTA 0 writes the results out), other small batches in one warp of a
+routing kernel (T*k <= 32 and <= 128 take two different sorts), batches up
+to 128 tokens in one CTA, larger decode batches in the route + union
+kernels, and prefill batches in a many-CTA counting sort.  Each of these
+leaves its
 unique ids, segment offsets, permutation and inverse in the call's workspace
 (coli_moe_union_offsets says where); they are compared element by element
 with the oracle's union of the ids the layer selected, and those ids with
@@ -33,8 +36,13 @@ def _shape(T, E, k, H=256, I=256, S=1):
 
 # (T, E, k, logits kind, the union code the layer runs for it)
 CASES = [
-    (1, 256, 8, "normal", "one warp, T*k <= 32"),
-    (4, 256, 8, "normal", "one warp, T*k <= 32"),
+    (1, 256, 8, "normal", "routing kernel, one warp, T*k <= 32"),
+    (4, 256, 8, "normal", "split-K kernel's own routing, T*k <= 32"),
+    (8, 256, 8, "zipf", "split-K kernel's own routing, T*k <= 128"),
+    (3, 16, 2, "ties", "split-K kernel's own routing, tie-dense logits"),
+    (6, 200, 4, "normal", "split-K kernel's own routing, E not a multiple of 32"),
+    (4, 512, 8, "normal", "routing kernel for E > 256, split-K form"),
+    (8, 64, 32, "ties", "one CTA for T*k > 128, split-K form"),
     (16, 256, 8, "zipf", "one warp, T*k <= 128"),
     (11, 16, 2, "ties", "one warp, T*k <= 32, tie-dense logits"),
     (17, 256, 8, "normal", "one CTA, T <= 128"),
@@ -96,3 +104,24 @@ def test_union_offsets_lie_inside_the_workspace(lib):
         assert all(o % 4 == 0 for o in off)
         assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
         assert spans[-1][1] <= lib.coli_moe_workspace_bytes(dims, T)
+
+
+@pytest.mark.parametrize("T", [1, 6], ids=["routing-kernel", "split-K-own-routing"])
+def test_layer_nonfinite_logits_flagged(lib, T):
+    """NaN and +inf logits set COLI_FLAG_NONFINITE on the layer path too, and
+    the selection stays the oracle's (NaN ranks as -inf)."""
+    E, k = 32, 4
+    shape = _shape(T, E, k)
+    layer = device_layer(shape, seed=22)
+    l32 = np.random.default_rng(5 + T).standard_normal((T, E)).astype(np.float32)
+    l32[0, 5] = np.nan
+    l32[T - 1, 0] = np.inf
+    x = synth.normal_bf16(22, 5, synth.X_IN, (T, shape.hidden))
+    xd = to_dev_bits(x)
+    out = torch.empty_like(xd)
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    lib.coli_moe_get_status()                      # clears the flags
+    layer.forward(xd, out, layer.workspace(T), logits_in=torch.from_numpy(l32).cuda(), topk_ids_out=ids)
+    st, flags = lib.coli_moe_get_status()
+    assert flags & lib._lib.COLI_FLAG_NONFINITE
+    assert np.array_equal(ids.cpu().numpy(), oracle.route(l32, k)[0])
