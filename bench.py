@@ -74,17 +74,17 @@ def parse():
 # digest (a kernel changed since the counters were taken) the line reports
 # null.  The batch-1 capture ran on the 16-expert variant of the layer, which
 # moves the same 9 experts per step; the prefill capture on the 32-expert,
-# 512-token variant (same tile shapes), where DRAM traffic was 1.062x the
+# 512-token variant (same tile shapes), where DRAM traffic was 1.063x the
 # algorithmic bytes of the gate/up launch; the 4096-token figure is that ratio
 # times its own algorithmic bytes (257 experts' gate+up codes and scales,
 # 36,864 gathered rows, h written).
-_SK_SOURCES = "9c400c5040a29e13"
-_PF_SOURCES = "552c12e296d31c08"
-_PF_RATIO = (532.615680e6 + 16.172544e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
+_SK_SOURCES = "30261d98ff90c3f0"
+_PF_SOURCES = "64537c0e6dc7cceb"
+_PF_RATIO = (532.914432e6 + 16.164864e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
 _PF_4096 = _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)
-TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.344896e6 + 5.110528e6, _SK_SOURCES),
-           ("glm52_layer_decode_b1_e16", "decode"): (191.344896e6 + 5.110528e6, _SK_SOURCES),
-           ("glm52_layer_prefill_512_e32", "prefill"): (532.615680e6 + 16.172544e6, _PF_SOURCES),
+TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
+           ("glm52_layer_decode_b1_e16", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
+           ("glm52_layer_prefill_512_e32", "prefill"): (532.914432e6 + 16.164864e6, _PF_SOURCES),
            ("glm52_layer_prefill_4096", "prefill"): (_PF_4096, _PF_SOURCES),
            # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
            ("glm52_layer_prefill_4096_router", "prefill"): (_PF_4096, _PF_SOURCES)}
