@@ -400,10 +400,25 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
                                                     uint16_t* __restrict__ xn, uint16_t* __restrict__ xq,
                                                     uint8_t* __restrict__ xp, int32_t* __restrict__ xe, int xq_f16,
                                                     uint32_t* __restrict__ status, int32_t* __restrict__ zero_ctr) {
+  const int nlog = wr ? E : 0;   // blocks [0, nlog): logits of expert b; then one block per token
+  // a logits block's first W_r loads (warp w: range [w H/8, (w+1) H/8), lane l:
+  // elements 4 l + 128 it) do not depend on the previous kernel
+  constexpr int kIt = 8;                       // float4 per lane per pass (1024 elements per warp)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hw = H >> 3;
+  const int h0 = warp * hw, h1 = h0 + hw;
+  const float* wrow = wr + static_cast<size_t>(static_cast<int>(blockIdx.x) < nlog ? blockIdx.x : 0) * H;
+  float4 w0[kIt];
+  if (static_cast<int>(blockIdx.x) < nlog) {
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      const int h = h0 + lane * 4 + it * 128;
+      w0[it] = h < h1 ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   pdl_wait();
   pdl_trigger();
   if (zero_ctr && blockIdx.x == 0 && threadIdx.x == 0) *zero_ctr = 0;
-  const int nlog = wr ? E : 0;   // blocks [0, nlog): logits of expert b; then one block per token
   __shared__ float red[8][8];
   __shared__ float rs[64];
   const int e = blockIdx.x;
@@ -488,13 +503,9 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
   if (static_cast<int>(blockIdx.x) >= nlog) return;
   // logits of expert e for every token, 8 tokens at a time.  Each lane issues
   // all its W_r loads (and a token's x loads) before any arithmetic, so the
-  // DRAM round trips overlap instead of following one another.
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hw = H >> 3;
-  const int h0 = warp * hw, h1 = h0 + hw;
-  const float* wrow = wr + static_cast<size_t>(e) * H;
+  // DRAM round trips overlap instead of following one another; the first
+  // pass's W_r values are w0, loaded before the wait.
   __shared__ float part[8][8];
-  constexpr int kIt = 8;                       // float4 per lane per pass (1024 elements per warp)
   for (int t0 = 0; t0 < T; t0 += 8) {
     const int nt = min(8, T - t0);
     float acc[8];
@@ -502,10 +513,12 @@ __global__ void __launch_bounds__(256) front_kernel(const uint16_t* __restrict__
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
     for (int hb = h0 + lane * 4; hb < h1; hb += 128 * kIt) {
       float4 w[kIt];
+      const bool first = hb == h0 + lane * 4;
 #pragma unroll
       for (int it = 0; it < kIt; ++it)
-        w[it] = (hb + it * 128 < h1) ? __ldg(reinterpret_cast<const float4*>(wrow + hb + it * 128))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        w[it] = first ? w0[it]
+                      : (hb + it * 128 < h1) ? __ldg(reinterpret_cast<const float4*>(wrow + hb + it * 128))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (q < nt) {
