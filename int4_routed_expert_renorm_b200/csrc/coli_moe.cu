@@ -592,7 +592,9 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   {
     const long work = static_cast<long>(T) * (H / 4);
     long blocks = (work + 255) / 256;
-    if (blocks > 4L * di.sms) blocks = 4L * di.sms;
+    // enough blocks in flight for the combine to stream its 4 (k + S) H bytes
+    // per token at the memory's rate (4 x SMs left it ~10 % short at 4096 tokens)
+    if (blocks > 16L * di.sms) blocks = 16L * di.sms;
     if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
                 pair_pos, topk_w, residual, T, k, S, H, out, static_cast<const int32_t*>(nullptr), 0, E,
                 static_cast<float*>(nullptr)))
