@@ -381,16 +381,22 @@ def main():
     flags = cm._lib.COLI_LAYER_PRENORM if shape.prenorm else 0
     flags |= {"auto": 0, "decode": cm._lib.COLI_PATH_DECODE, "prefill": cm._lib.COLI_PATH_PREFILL}[a.form]
 
-    def step(bi, x=None, out=None):
+    def step(bi, x=None, out=None, host=False):
+        # host: x (and the first layer's residual) and out are page-locked host
+        # buffers, read and written by the library's own kernels
         x = xs[bi] if x is None else x
+        hx = cm._lib.COLI_LAYER_HOST_X if host else 0
+        ho = cm._lib.COLI_LAYER_HOST_OUT if host else 0
         if shape.layers == 1:
             o = outs[0] if out is None else out
-            layers[0].forward(x, o, ws, logits_in=lgs[bi], flags=flags)
+            layers[0].forward(x, o, ws, logits_in=lgs[bi], flags=flags | hx | ho)
             return o
         h = x
         for li_, lay in enumerate(layers):
-            o = outs[li_ % 2] if (out is None or li_ < len(layers) - 1) else out
-            lay.forward(h, o, ws, residual=h if shape.prenorm else None, flags=flags)
+            last = li_ == len(layers) - 1
+            o = outs[li_ % 2] if (out is None or not last) else out
+            f = flags | (hx if li_ == 0 else 0) | (ho if last else 0)
+            lay.forward(h, o, ws, residual=h if shape.prenorm else None, flags=f)
             h = o
         return h
 
@@ -599,11 +605,56 @@ def main():
         return job_throughput(world, T, K2, ms)
 
     io = {"h2d_bytes_per_step": T * H * 2 + (T * E * 4 if shape.logits_in else 0), "d2h_bytes_per_step": T * H * 2}
-    e2e = {"value": e2e_run(g_e2e), "unit": UNIT, **io,
-           "how": "CUDA graph of the layer call(s) replayed each step" if g_e2e is not None else "eager calls"}
+    e2e_copies = {"value": e2e_run(g_e2e), "unit": UNIT, **io,
+                  "how": ("cudaMemcpyAsync of x in and out back around a CUDA graph of the layer call(s)"
+                          if g_e2e is not None else "cudaMemcpyAsync around eager calls")}
+
+    # the same with the input and the output in page-locked host memory, read
+    # and written by the library's kernels (COLI_LAYER_HOST_X | _HOST_OUT):
+    # the transfers are inside the layer call, no copy engine involved
+    def e2e_host_step(bi):
+        if ld is not None:
+            lgs_save = lgs[bi]
+            lgs[bi] = ld
+        step(bi, x=xh[bi], out=oh, host=True)
+        if ld is not None:
+            lgs[bi] = lgs_save
+
+    g_host = None
+    if use_graph:   # one graph per rotating batch: each reads its own host rows
+        for bi in range(NB):
+            e2e_host_step(bi)
+        torch.cuda.synchronize()
+        g_host = []
+        for bi in range(NB):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                e2e_host_step(bi)
+            g_host.append(g)
+
+    def e2e_host_run(graphs):
+        for i in range(K2):
+            bi = i % NB
+            flush_l2()
+            es[i].record()
+            if ld is not None:
+                ld.copy_(lh[bi], non_blocking=True)
+            if graphs is not None:
+                graphs[bi].replay()
+            else:
+                e2e_host_step(bi)
+            ee[i].record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(sum(es[i].elapsed_time(ee[i]) for i in range(K2)), world, "cuda")
+        return job_throughput(world, T, K2, ms)
+
+    e2e = {"value": e2e_host_run(g_host), "unit": UNIT, **io,
+           "how": ("CUDA graph of the layer call(s) with x read from and out written to page-locked host memory "
+                   "by the library's kernels" if g_host is not None else "eager calls, host-memory x and out")}
     # the same through eager calls: the host side of every call (argument
     # checks, tensor-map encoding, launches) inside the timed region
-    e2e_eager = {"value": e2e_run(None), "unit": UNIT, **io, "how": "eager calls"} if g_e2e is not None else None
+    e2e_eager = ({"value": e2e_host_run(None), "unit": UNIT, **io, "how": "eager calls, host-memory x and out"}
+                 if g_host is not None else None)
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -618,7 +669,8 @@ def main():
             "config": workload_config(shape, NB), "union_per_batch": U, "union_per_layer": u_stack or None,
             "int4_bytes_per_step": bytes_step, "int4_gbs": int4_gbs, "int4_frac_of_hbm": int4_gbs / hbm,
             "roofline": roof, "stage_ms": stage_ms,
-            "cpu_baseline": cpu, "e2e": e2e, "e2e_eager": e2e_eager, "gpu_launches": launches, "clocks": clocks,
+            "cpu_baseline": cpu, "e2e": e2e, "e2e_eager": e2e_eager, "e2e_copies": e2e_copies,
+            "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -95,6 +95,16 @@ typedef enum {
 
 /* Layer flags (coli_moe_layer / coli_moe_expert_ffn). */
 #define COLI_LAYER_PRENORM       0x1u  /* route and run the experts on n = bf16(x * rsqrt(mean(x^2) + 1e-6)) */
+#define COLI_LAYER_HOST_X        0x2u  /* coli_moe_layer / _noalloc: x (and the residual, if given) are in
+                                        * page-locked host memory mapped into the device's address space
+                                        * (cudaHostAlloc, cudaHostRegister with cudaHostRegisterMapped);
+                                        * one kernel copies the rows into the workspace before use */
+#define COLI_LAYER_HOST_OUT      0x4u  /* coli_moe_layer / _noalloc: out is in such host memory; the
+                                        * call's last kernel writes the bf16 rows there directly */
+/* With either HOST flag, a pointer the device cannot reach (pageable host
+ * memory) returns COLI_ERR_INVALID_ARG; the expert-parallel entry returns
+ * COLI_ERR_UNSUPPORTED.  For small decode batches these replace two
+ * cudaMemcpyAsync calls and their latency. */
 #define COLI_PATH_DECODE         0x10u /* force the decode FFN form (weights streamed once, mma.sync) */
 #define COLI_PATH_PREFILL        0x20u /* force the prefill FFN form (tcgen05 grouped GEMM) */
 /* With neither flag the prefill form is taken when T >= 32 and T*k >= 32*min(E, T*k)

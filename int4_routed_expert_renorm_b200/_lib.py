@@ -19,6 +19,7 @@ COLI_OK, COLI_ERR_INVALID_ARG, COLI_ERR_UNSUPPORTED, COLI_ERR_WORKSPACE = 0, 1, 
 COLI_ERR_CUDA, COLI_ERR_NONFINITE, COLI_ERR_DEVICE = 4, 5, 6
 COLI_FLAG_NONFINITE, COLI_FLAG_BAD_ID, COLI_FLAG_TIMEOUT, COLI_FLAG_RANGE = 0x1, 0x2, 0x4, 0x8
 COLI_LAYER_PRENORM, COLI_PATH_DECODE, COLI_PATH_PREFILL = 0x1, 0x10, 0x20
+COLI_LAYER_HOST_X, COLI_LAYER_HOST_OUT = 0x2, 0x4
 COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
@@ -94,6 +95,18 @@ def _ptr(t):
         raise ValueError("tensor arguments must be contiguous (dense, row-major)")
     if t.device.type != "cuda":
         raise ValueError(f"tensor arguments must be in device memory, got a tensor on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t, name: str):
+    """Host address of a page-locked CPU tensor (COLI_LAYER_HOST_X / _OUT);
+    the library maps it to its device address and refuses any other."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (dense, row-major)")
+    if t.device.type != "cpu" or not t.is_pinned():
+        raise ValueError(f"{name}: the HOST flag needs a page-locked CPU tensor, got one on {t.device}")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -197,14 +210,22 @@ def coli_moe_expert_ffn(dims, weights, x, topk_ids, topk_w, unique_ids, n_unique
                                     ws.numel() * ws.element_size(), _stream(stream)), "coli_moe_expert_ffn")
 
 
+def _io_ptrs(flags, x, residual, out):
+    """x, residual, out: device tensors, or page-locked CPU tensors under the
+    COLI_LAYER_HOST_X (x, residual) and COLI_LAYER_HOST_OUT (out) flags."""
+    hx, ho = flags & COLI_LAYER_HOST_X, flags & COLI_LAYER_HOST_OUT
+    return ((_host_ptr(x, "x") if hx else _ptr(x)), (_host_ptr(residual, "residual") if hx else _ptr(residual)),
+            (_host_ptr(out, "out") if ho else _ptr(out)))
+
+
 def coli_moe_layer(dims, weights, x, out, ws, logits_in=None, residual=None, flags=0, logits_out=None,
                    topk_ids_out=None, topk_w_out=None, stream=None):
     T = _tokens(x, dims.hidden)
     _layer_sizes(dims, T, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
-    _check(_lib.coli_moe_layer(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
-                               _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
-                               _ptr(topk_w_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
-           "coli_moe_layer")
+    px, pr, po = _io_ptrs(flags, x, residual, out)
+    _check(_lib.coli_moe_layer(ctypes.byref(dims), ctypes.byref(weights), px, T, _ptr(logits_in), pr, flags, po,
+                               _ptr(logits_out), _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "coli_moe_layer")
 
 
 def coli_moe_layer_noalloc(dims, weights, x, out, logits_in=None, residual=None, flags=0, logits_out=None,
@@ -213,9 +234,10 @@ def coli_moe_layer_noalloc(dims, weights, x, out, logits_in=None, residual=None,
     tensor, for callers that cannot allocate device memory (see the header)."""
     T = _tokens(x, dims.hidden)
     _layer_sizes(dims, T, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
-    _check(_lib.coli_moe_layer_noalloc(ctypes.byref(dims), ctypes.byref(weights), _ptr(x), T, _ptr(logits_in),
-                                       _ptr(residual), flags, _ptr(out), _ptr(logits_out), _ptr(topk_ids_out),
-                                       _ptr(topk_w_out), _stream(stream)), "coli_moe_layer_noalloc")
+    px, pr, po = _io_ptrs(flags, x, residual, out)
+    _check(_lib.coli_moe_layer_noalloc(ctypes.byref(dims), ctypes.byref(weights), px, T, _ptr(logits_in), pr, flags,
+                                       po, _ptr(logits_out), _ptr(topk_ids_out), _ptr(topk_w_out),
+                                       _stream(stream)), "coli_moe_layer_noalloc")
 
 
 def coli_moe_layer_ep(dims, weights, expert_begin: int, expert_end: int, with_shared: bool, x, out_partial, ws,

@@ -244,6 +244,8 @@ struct Ws {
   int32_t* rb_done;  // [H/128] down completion per output row block
   uint16_t* hq;      // [P+S*T][I]
   float* ypair;      // [P+S*T][H]
+  uint16_t* xin;     // [T][H] the input rows copied from host memory (COLI_LAYER_HOST_X)
+  uint16_t* rin;     // [T][H] the residual rows copied from host memory
   size_t bytes;
 };
 
@@ -316,6 +318,8 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
     const size_t yb = rows * H * 4, pb = use_splitk(d, T) ? rows * (I / 128) * H * 4 : 0;
     ws.ypair = static_cast<float*>(take(yb > pb ? yb : pb));
   }
+  ws.xin = static_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
+  ws.rin = static_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
   ws.bytes = o;
   return ws;
 }
@@ -883,6 +887,7 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   if (T < 0) return COLI_ERR_INVALID_ARG;
   if (static_cast<int64_t>(T) * dims->top_k > (int64_t(1) << 24)) return COLI_ERR_UNSUPPORTED;
   if ((st = check_weights(w, false)) != COLI_OK) return st;
+  if (flags & (COLI_LAYER_HOST_X | COLI_LAYER_HOST_OUT)) return COLI_ERR_UNSUPPORTED;   // device buffers only
   if (T == 0) return COLI_OK;
   if (!x || !topk_ids || !topk_w || !unique_ids || !n_unique || !seg_off || !perm || !pair_pos || !out || !ws)
     return COLI_ERR_INVALID_ARG;
@@ -915,6 +920,17 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
 
 namespace {
 
+// The device address of page-locked, mapped host memory, or NULL for any
+// other pointer (device memory, or host memory the device cannot reach).
+const void* host_mapped(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
                        const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
                        float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
@@ -934,6 +950,21 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
+  // host-memory input and output: page-locked and mapped, used through their
+  // device addresses (an expert-parallel share writes an fp32 partial instead)
+  const bool host_x = (flags & COLI_LAYER_HOST_X) != 0, host_out = (flags & COLI_LAYER_HOST_OUT) != 0;
+  if ((host_x || host_out) && ep.on) return COLI_ERR_UNSUPPORTED;
+  const uint16_t* xh = nullptr;
+  const uint16_t* rh = nullptr;
+  if (host_x) {
+    xh = static_cast<const uint16_t*>(host_mapped(x));
+    rh = residual ? static_cast<const uint16_t*>(host_mapped(residual)) : nullptr;
+    if (!xh || (residual && !rh)) return COLI_ERR_INVALID_ARG;
+  }
+  if (host_out) {
+    out = static_cast<uint16_t*>(const_cast<void*>(host_mapped(out)));
+    if (!out) return COLI_ERR_INVALID_ARG;
+  }
   // an expert-parallel share runs in the decode forms, with route, union and
   // plan in one kernel (T <= 128), and not through the two-phase kernel's
   // own combine (T <= 4 with I = 128)
@@ -948,6 +979,19 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const bool prenorm = (flags & COLI_LAYER_PRENORM) != 0;
   const StageRecorder rec(s);
   rec.mark(0);
+  if (host_x) {
+    // the rows into the workspace (a residual that is x itself is copied once)
+    const bool rsep = rh && rh != xh;
+    const long n16 = static_cast<long>(T) * H / 8;
+    long blocks = (n16 + 255) / 256;
+    if (blocks > 4L * di.sms) blocks = 4L * di.sms;
+    if (!launch(stage_rows_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s, reinterpret_cast<const uint4*>(xh),
+                reinterpret_cast<uint4*>(lay.xin), rsep ? reinterpret_cast<const uint4*>(rh) : nullptr,
+                rsep ? reinterpret_cast<uint4*>(lay.rin) : nullptr, n16))
+      return COLI_ERR_CUDA;
+    x = lay.xin;
+    residual = rh ? (rsep ? lay.rin : lay.xin) : nullptr;
+  }
   const int S = dims->n_shared, tokb = tok_block(T);
   // the split-K kernel routes the batch itself: no routing kernel runs
   const bool inroute = form == Form::kDecode && splitk_routes(dims, T);

@@ -385,6 +385,23 @@ __global__ void __launch_bounds__(256) logits_mma_kernel(const uint16_t* __restr
       }
 }
 
+// COLI_LAYER_HOST_X: the input rows (and, when b is not NULL, the residual
+// rows) from page-locked host memory into the workspace, n 16-byte chunks
+// each.  It waits for the previous kernel first, which may still read the
+// staging buffers of an earlier call.
+__global__ void __launch_bounds__(256) stage_rows_kernel(const uint4* __restrict__ a, uint4* __restrict__ da,
+                                                         const uint4* __restrict__ b, uint4* __restrict__ db,
+                                                         long n) {
+  pdl_wait();
+  pdl_trigger();
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const uint4 v = a[i];
+    if (b) db[i] = b[i];
+    da[i] = v;
+  }
+}
+
 // Small-batch front end (T <= 8), one launch of E + T blocks (T when the
 // logits are given, wr == NULL): block e < E computes the router logits of
 // expert e for every token; block E + t writes token t's fragment-ordered

@@ -121,6 +121,9 @@ def test_layer_argument_checks(colimoe):
     assert L(d, w, x, 0, ws, 0) == m._lib.COLI_OK                                # T = 0: no-op
     nw = m.coli_moe_weights(*[ctypes.c_void_p(0x100000 + i * 0x1000) for i in range(6)], None, None)
     assert L(d, nw, x, 4, ws, need) == m._lib.COLI_ERR_INVALID_ARG              # no router, no logits_in
+    # host-memory flags: pointers the device cannot reach as host memory are refused
+    assert L(d, w, x, 4, ws, need, m._lib.COLI_LAYER_HOST_X) == m._lib.COLI_ERR_INVALID_ARG
+    assert L(d, w, x, 4, ws, need, m._lib.COLI_LAYER_HOST_OUT) == m._lib.COLI_ERR_INVALID_ARG
 
 
 def test_expert_ffn_argument_checks(colimoe):
@@ -133,6 +136,21 @@ def test_expert_ffn_argument_checks(colimoe):
     assert F(4, need - 256) == m._lib.COLI_ERR_WORKSPACE
     assert F(4, need, x=_fake(0x600000)) == m._lib.COLI_ERR_INVALID_ARG   # out aliases x
     assert F(0, 0) == m._lib.COLI_OK
+    for hf in (m._lib.COLI_LAYER_HOST_X, m._lib.COLI_LAYER_HOST_OUT):         # device buffers only
+        assert lib.coli_moe_expert_ffn(ctypes.byref(d), ctypes.byref(w), f, 4, f, f, f, f, f, f, f, None,
+                                       _fake(0x600000), hf, _fake(0x700000), need, None) == m._lib.COLI_ERR_UNSUPPORTED
+
+
+def test_binding_host_flags_need_page_locked_tensors(colimoe):
+    """Under COLI_LAYER_HOST_X the binding passes x (and the residual) only as
+    page-locked CPU tensors; anything else is refused before the library."""
+    import torch
+    m = colimoe
+    d, w = _dims(m), _weights(m)
+    x = torch.zeros(2, d.hidden, dtype=torch.int16)            # CPU, not page-locked
+    with pytest.raises(ValueError, match="page-locked"):
+        m._lib.coli_moe_layer(d, w, x, torch.zeros_like(x), torch.empty(16, dtype=torch.uint8),
+                              flags=m._lib.COLI_LAYER_HOST_X)
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
