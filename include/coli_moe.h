@@ -256,7 +256,7 @@ coli_status coli_moe_partial_to_bf16(const float *partial, uint16_t *out, size_t
  *   - Arguments and results are those of coli_moe_layer, without ws/ws_bytes.
  *   - Batches whose coli_moe_workspace_bytes(dims, T) exceeds
  *     COLI_NOALLOC_SCRATCH_BYTES are rejected with COLI_ERR_WORKSPACE before
- *     anything is launched (up to 87 tokens for H=6144, I=2048, E=256, k=8, S=1).
+ *     anything is launched (up to 82 tokens for H=6144, I=2048, E=256, k=8, S=1).
  *   - The first call on a device looks up the array's device address (one
  *     cudaGetSymbolAddress with that device current); make that first call
  *     before capturing a stream.  No call allocates or frees device memory.
