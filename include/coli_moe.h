@@ -327,6 +327,75 @@ coli_status coli_moe_get_status(void *stream, uint32_t *flags);
  * COLI_FLAG_TIMEOUT). */
 coli_status coli_moe_test_wait_timeout(uint64_t limit_ns, uint64_t *elapsed_ns, void *stream);
 
+/*
+ * Host-RAM expert tier: Place, Overlap and Learn (Colibri README, "Una
+ * gerarchia di memoria, non un requisito di memoria" and "Mai aspettare il
+ * disco due volte"; getting-started guide, "トークンごとの処理経路", steps 3-5).
+ * Every routed expert lives in page-locked host memory; the device holds C of
+ * them at a time in slots.  A tiered layer call routes and unites the batch as
+ * coli_moe_layer does, then places the union on the device: experts already in
+ * a slot are hits; each miss takes the slot, not used by this batch, that
+ * holds the expert routed least often so far (empty slots first, then the
+ * least recently used, then the lowest index), and its three matrices are
+ * copied from host memory into that slot by the library's kernels.  The FFN
+ * then runs on the slots; placement changes neither the routing nor the
+ * arithmetic, so the output equals coli_moe_layer's bit for bit.  Learn: the
+ * tier counts the routed pairs of every expert over all calls, and the
+ * eviction order keeps the most used experts resident.  Overlap: a caller
+ * that predicts the next layer's experts (for example with that layer's
+ * router on the current input) places them with coli_moe_tier_prefetch on
+ * another stream while the current layer computes.
+ *
+ * coli_moe_tier (per layer):
+ *   gate_q .. down_s  every routed expert's codes and scales, laid out as in
+ *                     coli_moe_weights (E experts, no shared ones), in
+ *                     page-locked host memory mapped into the device's address
+ *                     space (cudaHostAlloc, cudaHostRegister with
+ *                     cudaHostRegisterMapped); the library reads it only
+ *   n_slots           C, routed experts held on the device, 1 <= C <= E
+ *   state             device memory of coli_moe_tier_state_bytes(dims, C)
+ *                     bytes, 256-byte aligned, owned by the caller, set up by
+ *                     coli_moe_tier_reset before first use; its layout (int32
+ *                     unless noted): slot_of[E] (slot of expert e, or -1),
+ *                     owner[C] (expert in slot c, or -1), usage[E] (uint32,
+ *                     routed pairs per expert), last[C] (uint32, the call count
+ *                     at the slot's last use), calls, hits, misses, fills
+ *                     (uint32 counters), then scratch
+ * The weights passed with a tier (`slots`) are device arrays of C routed
+ * experts followed by the S shared ones, with the router weight and bias as in
+ * coli_moe_weights; their contents follow the tier (reset leaves them unused).
+ */
+typedef struct {
+  const uint8_t *gate_q, *up_q, *down_q;
+  const uint16_t *gate_s, *up_s, *down_s;
+  int32_t n_slots;
+  void *state;
+} coli_moe_tier;
+
+/* Device bytes of a tier's state; 0 for invalid arguments. */
+size_t coli_moe_tier_state_bytes(const coli_moe_dims *dims, int32_t n_slots);
+
+/* Empties every slot and clears the counters (enqueued on `stream`). */
+coli_status coli_moe_tier_reset(const coli_moe_dims *dims, const coli_moe_tier *tier, void *stream);
+
+/* coli_moe_layer through a tier: arguments as coli_moe_layer's, with `slots`
+ * in place of the weights.  Decode form only (COLI_PATH_PREFILL, or an
+ * automatic choice of the prefill form, returns COLI_ERR_UNSUPPORTED), and a
+ * batch must fit the slots: min(E, T*k) <= C, else COLI_ERR_UNSUPPORTED.
+ * Workspace: coli_moe_workspace_bytes(dims, T). */
+coli_status coli_moe_layer_tiered(const coli_moe_dims *dims, const coli_moe_weights *slots,
+                                  const coli_moe_tier *tier, const uint16_t *x, int T, const float *logits_in,
+                                  const uint16_t *residual, uint32_t flags, uint16_t *out, float *logits_out,
+                                  int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                                  void *stream);
+
+/* Places experts ids[0..n) (device int32, any order, repeats allowed, n <= C)
+ * as a tiered call would, without counting them as routed: the copies of the
+ * misses are enqueued on `stream`.  Calls on one tier must be ordered (one
+ * stream, or events); tiers of different layers are independent. */
+coli_status coli_moe_tier_prefetch(const coli_moe_dims *dims, const coli_moe_weights *slots,
+                                   const coli_moe_tier *tier, const int32_t *ids, int32_t n, void *stream);
+
 /* Static description of a status code. */
 const char *coli_status_str(coli_status s);
 

@@ -25,7 +25,8 @@ COLI_FORM_DECODE_SPLITK, COLI_FORM_DECODE_TWOPHASE, COLI_FORM_PREFILL = 1, 2, 3
 EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_layer",
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
            "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form",
-           "coli_moe_union_offsets", "coli_moe_test_wait_timeout", "coli_moe_layer_ep", "coli_moe_partial_to_bf16")
+           "coli_moe_union_offsets", "coli_moe_test_wait_timeout", "coli_moe_layer_ep", "coli_moe_partial_to_bf16",
+           "coli_moe_tier_state_bytes", "coli_moe_tier_reset", "coli_moe_layer_tiered", "coli_moe_tier_prefetch")
 COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -47,12 +48,19 @@ class coli_moe_weights(ctypes.Structure):
                 ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p)]
 
 
+class coli_moe_tier(ctypes.Structure):
+    _fields_ = [("gate_q", ctypes.c_void_p), ("up_q", ctypes.c_void_p), ("down_q", ctypes.c_void_p),
+                ("gate_s", ctypes.c_void_p), ("up_s", ctypes.c_void_p), ("down_s", ctypes.c_void_p),
+                ("n_slots", ctypes.c_int32), ("state", ctypes.c_void_p)]
+
+
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(f"{path} is not built; run `python -m int4_routed_expert_renorm_b200.build`")
     lib = ctypes.CDLL(path)
     P, I, Z, U32, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_uint64
     D, W = ctypes.POINTER(coli_moe_dims), ctypes.POINTER(coli_moe_weights)
+    TR = ctypes.POINTER(coli_moe_tier)
     sig = {
         "coli_moe_route": (I, [P, P, I, I, I, P, P, P]),
         "coli_moe_union": (I, [P, I, I, I, P, P, P, P, P, P]),
@@ -70,6 +78,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_test_wait_timeout": (I, [U64, P, P]),
         "coli_moe_layer_ep": (I, [D, W, I, I, I, P, I, P, P, U32, P, P, P, P, P, Z, P]),
         "coli_moe_partial_to_bf16": (I, [P, P, Z, P]),
+        "coli_moe_tier_state_bytes": (Z, [D, I]),
+        "coli_moe_tier_reset": (I, [D, TR, P]),
+        "coli_moe_layer_tiered": (I, [D, W, TR, P, I, P, P, U32, P, P, P, P, P, Z, P]),
+        "coli_moe_tier_prefetch": (I, [D, W, TR, P, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -251,6 +263,34 @@ def coli_moe_layer_ep(dims, weights, expert_begin: int, expert_end: int, with_sh
                                   1 if with_shared else 0, _ptr(x), T, _ptr(logits_in), _ptr(residual), flags,
                                   _ptr(out_partial), _ptr(logits_out), _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "coli_moe_layer_ep")
+
+
+def coli_moe_tier_state_bytes(dims, n_slots: int) -> int:
+    return _lib.coli_moe_tier_state_bytes(ctypes.byref(dims), n_slots)
+
+
+def coli_moe_tier_reset(dims, tier, stream=None):
+    _check(_lib.coli_moe_tier_reset(ctypes.byref(dims), ctypes.byref(tier), _stream(stream)), "coli_moe_tier_reset")
+
+
+def coli_moe_layer_tiered(dims, slots, tier, x, out, ws, logits_in=None, residual=None, flags=0, logits_out=None,
+                          topk_ids_out=None, topk_w_out=None, stream=None):
+    """coli_moe_layer through a host-RAM expert tier (see the header)."""
+    T = _tokens(x, dims.hidden)
+    _layer_sizes(dims, T, out, residual, logits_in, logits_out, topk_ids_out, topk_w_out)
+    px, pr, po = _io_ptrs(flags, x, residual, out)
+    _check(_lib.coli_moe_layer_tiered(ctypes.byref(dims), ctypes.byref(slots), ctypes.byref(tier), px, T,
+                                      _ptr(logits_in), pr, flags, po, _ptr(logits_out), _ptr(topk_ids_out),
+                                      _ptr(topk_w_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "coli_moe_layer_tiered")
+
+
+def coli_moe_tier_prefetch(dims, slots, tier, ids, stream=None):
+    """Places experts ids (device int32, at most n_slots of them) in the tier."""
+    if ids.dtype.itemsize != 4:
+        raise ValueError("ids: int32 expert ids")
+    _check(_lib.coli_moe_tier_prefetch(ctypes.byref(dims), ctypes.byref(slots), ctypes.byref(tier), _ptr(ids),
+                                       ids.numel(), _stream(stream)), "coli_moe_tier_prefetch")
 
 
 def coli_moe_partial_to_bf16(partial, out, stream=None):

@@ -7,6 +7,7 @@
 // or synchronises, except coli_moe_get_status.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -17,6 +18,7 @@
 #include "k_ffn_prefill.cuh"
 #include "k_ffn_splitk.cuh"
 #include "k_router.cuh"
+#include "k_tier.cuh"
 #include "k_union.cuh"
 
 using namespace coli;
@@ -246,6 +248,7 @@ struct Ws {
   float* ypair;      // [P+S*T][H]
   uint16_t* xin;     // [T][H] the input rows copied from host memory (COLI_LAYER_HOST_X)
   uint16_t* rin;     // [T][H] the residual rows copied from host memory
+  int32_t* sunique;  // [min(E,P)] device slot of each unique expert (host-RAM tier)
   size_t bytes;
 };
 
@@ -320,6 +323,7 @@ Ws layout(const coli_moe_dims* d, int T, void* base) {
   }
   ws.xin = static_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
   ws.rin = static_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
+  ws.sunique = static_cast<int32_t*>(take(Umax * 4));
   ws.bytes = o;
   return ws;
 }
@@ -644,10 +648,12 @@ coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, co
                     const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
                     const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
                     cudaStream_t st, const StageRecorder& rec, const EpRange& ep = EpRange(),
-                    const InRoute& ir = InRoute()) {
+                    const InRoute& ir = InRoute(), int slots = 0) {
   const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k;
   const int S = ep.on ? ep.shared : d->n_shared;
-  const int E_w = ep.on ? ep.end - ep.begin : E;   // routed experts held by the weights
+  // routed experts held by the weights: all, an expert-parallel rank's range,
+  // or the slots of a host-RAM tier (the union then holds slot numbers)
+  const int E_w = slots > 0 ? slots : ep.on ? ep.end - ep.begin : E;
   const int P = T * k;
   const uint64_t rows_gu = static_cast<uint64_t>(E_w + S) * I;
   const uint64_t rows_dn = static_cast<uint64_t>(E_w + S) * H;
@@ -918,6 +924,14 @@ coli_status coli_moe_expert_ffn(const coli_moe_dims* dims, const coli_moe_weight
   return run_ffn(dims, w, T, unique_ids, n_unique, seg_off, perm, pair_pos, topk_w, residual, out, lay, di, s, rec);
 }
 
+// A host-RAM tier as the kernels see it: the slot count, the device state and
+// the copy description (host sources through their device addresses).
+struct TierArgs {
+  int slots;
+  void* state;
+  TierCopy cp;
+};
+
 namespace {
 
 // The device address of page-locked, mapped host memory, or NULL for any
@@ -934,7 +948,7 @@ const void* host_mapped(const void* p) {
 coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, const uint16_t* x, int T,
                        const float* logits_in, const uint16_t* residual, uint32_t flags, uint16_t* out,
                        float* logits_out, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
-                       void* stream, EpRange ep) {
+                       void* stream, EpRange ep, const TierArgs* tier = nullptr) {
   coli_status st = check_dims(dims);
   if (st != COLI_OK) return st;
   if (T < 0) return COLI_ERR_INVALID_ARG;
@@ -950,6 +964,11 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
+  // a host-RAM tier: decode form, no expert-parallel share, and every batch's
+  // union must fit the slots
+  if (tier && (form != Form::kDecode || ep.on ||
+               std::min<int64_t>(dims->n_experts, static_cast<int64_t>(T) * dims->top_k) > tier->slots))
+    return COLI_ERR_UNSUPPORTED;
   // host-memory input and output: page-locked and mapped, used through their
   // device addresses (an expert-parallel share writes an fp32 partial instead)
   const bool host_x = (flags & COLI_LAYER_HOST_X) != 0, host_out = (flags & COLI_LAYER_HOST_OUT) != 0;
@@ -994,7 +1013,7 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   }
   const int S = dims->n_shared, tokb = tok_block(T);
   // the split-K kernel routes the batch itself: no routing kernel runs
-  const bool inroute = form == Form::kDecode && splitk_routes(dims, T);
+  const bool inroute = form == Form::kDecode && splitk_routes(dims, T) && !tier;
 
   // 1. expert input (fragment order, optional pre-norm) and router logits
   float* lo = logits_out ? logits_out : lay.logits;
@@ -1080,6 +1099,17 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
     ir.ids = ids;
     ir.w = tw;
   }
+  if (tier) {
+    // Place (and Learn): the union's experts into slots, the misses copied in
+    // from host memory; the FFN then reads the slots
+    if (!launch(tier_place_kernel, dim3(1), dim3(256), 0, s, static_cast<const int32_t*>(lay.unique), 0,
+                static_cast<const int32_t*>(lay.n_unique), static_cast<const int32_t*>(lay.seg_off), E, tier->slots,
+                tier->state, lay.sunique, di.status) ||
+        !launch(tier_fill_kernel, dim3(4 * di.sms), dim3(256), 0, s, tier->cp, tier->state, E, tier->slots))
+      return COLI_ERR_CUDA;
+    return run_ffn(dims, w, T, lay.sunique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out,
+                   lay, di, s, rec, ep, ir, tier->slots);
+  }
   return run_ffn(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out, lay,
                  di, s, rec, ep, ir);
 }
@@ -1164,6 +1194,87 @@ coli_status coli_moe_layer_noalloc(const coli_moe_dims* dims, const coli_moe_wei
   }
   return coli_moe_layer(dims, w, x, T, logits_in, residual, flags, out, logits_out, topk_ids_out, topk_w_out, ptr,
                         COLI_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+namespace {
+
+// Checks a tier against the dims (and, with `slots`, the device slot arrays)
+// and fills the kernels' view of it.
+coli_status tier_args(const coli_moe_dims* d, const coli_moe_tier* t, const coli_moe_weights* slots,
+                      TierArgs* out) {
+  coli_status st = check_dims(d);
+  if (st != COLI_OK) return st;
+  if (!t || !t->state || !aligned(t->state, 256)) return COLI_ERR_INVALID_ARG;
+  if (t->n_slots < 1 || t->n_slots > d->n_experts) return COLI_ERR_INVALID_ARG;
+  *out = TierArgs{};
+  out->slots = t->n_slots;
+  out->state = t->state;
+  if (!slots) return COLI_OK;
+  const size_t H = d->hidden, I = d->inter, G = d->group, B = code_bits(d);
+  const size_t qg = I * H * B / 8, qd = H * I * B / 8, sg = I * (H / G) * 2, sd = H * (I / G) * 2;
+  const void* hs[6] = {t->gate_q, t->up_q, t->down_q, t->gate_s, t->up_s, t->down_s};
+  const void* ds[6] = {slots->gate_q, slots->up_q, slots->down_q, slots->gate_s, slots->up_s, slots->down_s};
+  const size_t per[6] = {qg, qg, qd, sg, sg, sd};
+  for (int m = 0; m < 6; ++m) {
+    if (per[m] % 16) return COLI_ERR_UNSUPPORTED;
+    if (!hs[m] || !ds[m] || !aligned(hs[m], 16) || !aligned(ds[m], 16)) return COLI_ERR_INVALID_ARG;
+    const void* dev = host_mapped(hs[m]);
+    if (!dev) return COLI_ERR_INVALID_ARG;
+    out->cp.src[m] = static_cast<const uint4*>(dev);
+    out->cp.dst[m] = static_cast<uint4*>(const_cast<void*>(ds[m]));
+    out->cp.per[m] = static_cast<long>(per[m] / 16);
+  }
+  return COLI_OK;
+}
+
+}  // namespace
+
+size_t coli_moe_tier_state_bytes(const coli_moe_dims* dims, int32_t n_slots) {
+  if (check_dims(dims) != COLI_OK || n_slots < 1 || n_slots > dims->n_experts) return 0;
+  return align256(tier_state_words(dims->n_experts, n_slots) * 4);
+}
+
+coli_status coli_moe_tier_reset(const coli_moe_dims* dims, const coli_moe_tier* tier, void* stream) {
+  TierArgs ta;
+  coli_status st = tier_args(dims, tier, nullptr, &ta);
+  if (st != COLI_OK) return st;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  const int n = std::max(dims->n_experts, ta.slots);
+  return launch(tier_reset_kernel, dim3((n + 255) / 256), dim3(256), 0, as_stream(stream), ta.state,
+                dims->n_experts, ta.slots)
+             ? COLI_OK
+             : COLI_ERR_CUDA;
+}
+
+coli_status coli_moe_layer_tiered(const coli_moe_dims* dims, const coli_moe_weights* slots, const coli_moe_tier* tier,
+                                  const uint16_t* x, int T, const float* logits_in, const uint16_t* residual,
+                                  uint32_t flags, uint16_t* out, float* logits_out, int32_t* topk_ids_out,
+                                  float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  TierArgs ta;
+  coli_status st = tier_args(dims, tier, slots, &ta);
+  if (st != COLI_OK) return st;
+  return layer_impl(dims, slots, x, T, logits_in, residual, flags, out, logits_out, topk_ids_out, topk_w_out, ws,
+                    ws_bytes, stream, EpRange(), &ta);
+}
+
+coli_status coli_moe_tier_prefetch(const coli_moe_dims* dims, const coli_moe_weights* slots,
+                                   const coli_moe_tier* tier, const int32_t* ids, int32_t n, void* stream) {
+  TierArgs ta;
+  coli_status st = tier_args(dims, tier, slots, &ta);
+  if (st != COLI_OK) return st;
+  if (n < 0 || n > ta.slots || (n > 0 && (!ids || !aligned(ids, 4)))) return COLI_ERR_INVALID_ARG;
+  if (n == 0) return COLI_OK;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  return launch(tier_place_kernel, dim3(1), dim3(256), 0, s, ids, static_cast<int>(n),
+                static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr), dims->n_experts,
+                ta.slots, ta.state, static_cast<int32_t*>(nullptr), di.status) &&
+                 launch(tier_fill_kernel, dim3(4 * di.sms), dim3(256), 0, s, ta.cp, ta.state, dims->n_experts,
+                        ta.slots)
+             ? COLI_OK
+             : COLI_ERR_CUDA;
 }
 
 coli_status coli_moe_test_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns, void* stream) {

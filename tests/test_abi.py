@@ -141,6 +141,33 @@ def test_expert_ffn_argument_checks(colimoe):
                                        _fake(0x600000), hf, _fake(0x700000), need, None) == m._lib.COLI_ERR_UNSUPPORTED
 
 
+def test_tier_state_bytes_and_argument_checks(colimoe):
+    """The tier's state size (int32 words: 2 E + 4 C + 5, 256-byte aligned)
+    and the checks that need no GPU."""
+    m = colimoe
+    lib = m._lib._lib
+    d = _dims(m)
+    E = d.n_experts
+    for C in (1, 7, E):
+        assert m.coli_moe_tier_state_bytes(d, C) == -(-(4 * (2 * E + 4 * C + 5)) // 256) * 256
+    assert m.coli_moe_tier_state_bytes(d, 0) == 0 and m.coli_moe_tier_state_bytes(d, E + 1) == 0
+    f = ctypes.c_void_p(0x10000)
+    t = m.coli_moe_tier(f, f, f, f, f, f, 4, ctypes.c_void_p(0x20000))
+    assert lib.coli_moe_tier_reset(ctypes.byref(d), ctypes.byref(m.coli_moe_tier(f, f, f, f, f, f, 0, f)),
+                                   None) == m._lib.COLI_ERR_INVALID_ARG       # no slots
+    assert lib.coli_moe_tier_reset(ctypes.byref(d), ctypes.byref(m.coli_moe_tier(f, f, f, f, f, f, 4,
+                                                                                 ctypes.c_void_p(0x20010))),
+                                   None) == m._lib.COLI_ERR_INVALID_ARG       # state not 256-byte aligned
+    w = _weights(m)
+    # host arrays the device cannot reach as host memory are refused
+    assert lib.coli_moe_tier_prefetch(ctypes.byref(d), ctypes.byref(w), ctypes.byref(t), f, 2,
+                                      None) == m._lib.COLI_ERR_INVALID_ARG
+    x, out, ws = _fake(0x200000), _fake(0x300000), _fake(0x400000)
+    assert lib.coli_moe_layer_tiered(ctypes.byref(d), ctypes.byref(w), ctypes.byref(t), x, 1, None, None, 0, out,
+                                     None, None, None, ws, m.coli_moe_workspace_bytes(d, 1),
+                                     None) == m._lib.COLI_ERR_INVALID_ARG
+
+
 def test_binding_host_flags_need_page_locked_tensors(colimoe):
     """Under COLI_LAYER_HOST_X the binding passes x (and the residual) only as
     page-locked CPU tensors; anything else is refused before the library."""
