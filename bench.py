@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--batches", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tier", type=int, default=0,
+                    help="run a one-layer decode workload through a host-RAM expert tier with this many device "
+                         "slots (the routed experts in page-locked host memory)")
     ap.add_argument("--form", choices=["auto", "decode", "prefill"], default="auto",
                     help="FFN form (COLI_PATH_*); auto lets the library choose")
     ap.add_argument("--graph", choices=["on", "off"], default="on",
@@ -359,7 +362,16 @@ def main():
         li = synth.LayerInputs(shape, 0, l)
         rw = None if shape.logits_in else torch.from_numpy(li.router_w()).cuda()
         b = li.bias()
-        layers.append(cm.MoELayer(dims, sg.expert_tensors(shape, 0, l), rw, None if b is None else torch.from_numpy(b).cuda()))
+        bias = None if b is None else torch.from_numpy(b).cuda()
+        if a.tier:
+            if shape.layers != 1:
+                raise SystemExit("--tier runs one-layer workloads")
+            full = sg.expert_tensors(shape, 0, l)
+            layers.append(cm.tier.TieredLayer(dims, full, a.tier, rw, bias))
+            del full
+            torch.cuda.empty_cache()
+        else:
+            layers.append(cm.MoELayer(dims, sg.expert_tensors(shape, 0, l), rw, bias))
     NB = a.batches
     xs = [torch.from_numpy(synth.activations(shape, 0, bi).view(np.int16)).cuda() for bi in rank_batches(rank, NB)]
     lgs = [None] * NB
@@ -457,6 +469,7 @@ def main():
     torch.cuda.synchronize()
     sampler = ClockSampler(local) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
+    tier0 = layers[0].state_arrays() if a.tier else None
     cm.coli_moe_launch_count(reset=True)
     t_wall0 = time.time()
     for i in range(K):
@@ -482,6 +495,16 @@ def main():
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
     total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     value = job_throughput(world, T, K, total_ms)
+    tier = None
+    if a.tier:
+        # the timed steps' placement: hits, misses, and the expert bytes the
+        # misses copied over the host link
+        t1 = layers[0].state_arrays()
+        hits, misses = t1["hits"] - tier0["hits"], t1["misses"] - tier0["misses"]
+        fill_b = (t1["fills"] - tier0["fills"]) * shape.expert_bytes() / K
+        tier = {"slots": a.tier, "experts": E, "hit_rate": hits / max(1, hits + misses), "hits_per_step": hits / K,
+                "misses_per_step": misses / K, "fill_bytes_per_step": fill_b,
+                "fill_gbs_over_the_step": fill_b / (total_ms / K / 1e3) / 1e9}
 
     # dominant kernel, timed live on the launching stream (stage 5 -> 6): the
     # decode form's one persistent FFN launch (gate/up, down and, for T <= 4,
@@ -666,10 +689,11 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": a.warmup,
             "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "ffn_form": form, "cuda_graph": use_graph,
-            "config": workload_config(shape, NB), "union_per_batch": U, "union_per_layer": u_stack or None,
+            "config": dict(workload_config(shape, NB), **({"tier_slots": a.tier} if a.tier else {})),
+            "union_per_batch": U, "union_per_layer": u_stack or None,
             "int4_bytes_per_step": bytes_step, "int4_gbs": int4_gbs, "int4_frac_of_hbm": int4_gbs / hbm,
             "roofline": roof, "stage_ms": stage_ms,
-            "cpu_baseline": cpu, "e2e": e2e, "e2e_eager": e2e_eager, "e2e_copies": e2e_copies,
+            "cpu_baseline": cpu, "e2e": e2e, "e2e_eager": e2e_eager, "e2e_copies": e2e_copies, "tier": tier,
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

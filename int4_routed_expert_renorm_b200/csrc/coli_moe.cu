@@ -1107,6 +1107,7 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
                 tier->state, lay.sunique, di.status) ||
         !launch(tier_fill_kernel, dim3(4 * di.sms), dim3(256), 0, s, tier->cp, tier->state, E, tier->slots))
       return COLI_ERR_CUDA;
+    rec.mark(5);   // the stage before the FFN ends after the copies
     return run_ffn(dims, w, T, lay.sunique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual, out,
                    lay, di, s, rec, ep, ir, tier->slots);
   }

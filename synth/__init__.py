@@ -174,6 +174,9 @@ DECODE_B1_E16 = LayerShape("glm52_layer_decode_b1_e16", 6144, 2048, 16, 8, 1, 1)
 # 0.7 GB resident): split-K units of the same shape as DECODE_B64's, for
 # profiler captures.
 DECODE_B64_E32 = LayerShape("glm52_layer_decode_b64_zipf_e32", 6144, 2048, 32, 8, 1, 64, zipf_bias=True)
+# Batch-1 decode with the Zipf router bias of DECODE_B64: a workload whose hot
+# experts recur, for the host-RAM expert tier.
+DECODE_B1_ZIPF = LayerShape("glm52_layer_decode_b1_zipf", 6144, 2048, 256, 8, 1, 1, zipf_bias=True)
 # Prefill tiles of the same shape as PREFILL_4096 (~128 tokens on every expert;
 # 32 routed + 1 shared expert resident, 0.7 GB): for profiler captures.
 PREFILL_512_E32 = LayerShape("glm52_layer_prefill_512_e32", 6144, 2048, 32, 8, 1, 512, logits_in=True)
@@ -191,7 +194,7 @@ DECODE_B1_INT8 = LayerShape("glm52_layer_int8_decode_b1", 6144, 2048, 256, 8, 1,
 PREFILL_4096_ROUTER = LayerShape("glm52_layer_prefill_4096_router", 6144, 2048, 256, 8, 1, 4096)
 WORKLOADS = {s.name: s for s in (TINY, DECODE_B1, DECODE_B64, PREFILL_4096, STACK16_B4, DECODE_B1_E16,
                                  DECODE_B64_E32, PREFILL_512_E32, DECODE_B1_GS64, PREFILL_4096_GS64, DECODE_B1_INT8,
-                                 PREFILL_4096_ROUTER)}
+                                 PREFILL_4096_ROUTER, DECODE_B1_ZIPF)}
 
 
 class LayerInputs:
