@@ -67,6 +67,29 @@ class TieredLayer:
         """Place experts `ids` (device int32, at most n_slots) ahead of use."""
         coli_moe_tier_prefetch(self.dims, self.weights, self.tier, ids.contiguous(), stream)
 
+    # ---- Learn: the usage counts, kept across runs ----------------------------
+    def usage(self) -> np.ndarray:
+        """Routed pairs per expert over every call since the last reset."""
+        return self.state_arrays()["usage"]
+
+    def warm_from_usage(self, usage, stream=None):
+        """Start from a saved usage profile (for example a previous run's
+        ``usage()``): the counts are written into the tier's state and its
+        ``n_slots`` most used experts (ties to the lower index) are placed, so
+        that the hottest experts are resident before the first call."""
+        E = self.dims.n_experts
+        u = np.asarray(usage, dtype=np.int64).reshape(-1)
+        if u.size != E or (u < 0).any():
+            raise ValueError(f"usage: {u.size} non-negative counts needed, one per expert ({E})")
+        u = np.minimum(u, 0xFFFFFFFF).astype(np.uint32)
+        words = torch.from_numpy(u.view(np.int32).copy()).to(self.state.device)
+        C = self.n_slots
+        off = 4 * (E + C)                                   # usage[E] follows slot_of[E] and owner[C]
+        torch.cuda.synchronize()
+        self.state[off:off + 4 * E].copy_(words.view(torch.uint8))
+        hot = np.lexsort((np.arange(E), -u.astype(np.int64)))[:C].astype(np.int32)
+        self.prefetch(torch.from_numpy(hot).to(self.state.device), stream)
+
     # ---- the state, read back (synchronises) ------------------------------
     def _words(self) -> np.ndarray:
         torch.cuda.synchronize()

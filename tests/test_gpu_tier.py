@@ -180,3 +180,32 @@ def test_tier_refuses_what_it_cannot_hold(m):
     assert st_ == 0 and fl == 0
     del full, resident, tl
     torch.cuda.empty_cache()
+
+
+def test_tier_warm_start_from_a_usage_profile(m):
+    """Learn across runs: a saved usage profile makes its most used experts
+    resident before the first call (the pages' pinned hot experts), and the
+    counts carry on from it."""
+    E, k, C = 32, 2, 6
+    shape, full, resident, tl = _setup(m, 2, E, k, C, seed=44)
+    profile = np.zeros(E, np.int64)
+    profile[[3, 9, 10, 21, 30, 31, 7]] = [50, 40, 40, 30, 20, 20, 20]   # 31 and 7 tie with 30: lower index wins
+    tl.warm_from_usage(profile)
+    st = tl.state_arrays()
+    assert sorted(st["owner"].tolist()) == [3, 7, 9, 10, 21, 30]
+    assert np.array_equal(st["usage"], profile.astype(np.uint32))
+    # a call that routes to two of them hits and adds its pairs to the profile
+    T = 1
+    l32 = np.full((T, E), -5.0, np.float32)
+    l32[0, 9], l32[0, 21] = 2.0, 1.0
+    x = synth.normal_bf16(44, 5, synth.X_IN, (T, 512))
+    xd, lg = to_dev_bits(x), torch.from_numpy(l32).cuda()
+    o_t, o_r = torch.empty_like(xd), torch.empty_like(xd)
+    tl.forward(xd, o_t, tl.workspace(T), logits_in=lg)
+    resident.forward(xd, o_r, resident.workspace(T), logits_in=lg)
+    st = tl.state_arrays()
+    assert st["hits"] == 2 and st["misses"] == 0
+    assert st["usage"][9] == 41 and st["usage"][21] == 31
+    assert np.array_equal(bits(o_t), bits(o_r))
+    del full, resident, tl
+    torch.cuda.empty_cache()
