@@ -392,11 +392,12 @@ bool launch_cooperative(FfnKernel kernel, size_t smem, const CUtensorMap* m, con
 // The split-K kernel as a plain launch with programmatic dependent launch:
 // its grid is at most one CTA per SM and its shared memory admits one CTA
 // per SM, so every CTA becomes resident without a cooperative launch (a CTA
-// that finds its SM still busy with the routing kernel's one CTA starts when
-// that CTA ends; the routing kernel waits on nothing of this kernel).  The
-// plain launch lets the CTAs start their prologue and the shared experts'
-// weight stream while the routing kernel still runs, which a cooperative
-// launch does not.  Every wait in the kernel is bounded.
+// that finds its SM still busy with the preceding kernel's CTAs -- the routing
+// kernel's one CTA, the front kernel's, or a tier's copies -- starts when they
+// end; none of them waits on anything of this kernel).  The plain launch lets
+// the CTAs start their prologue and the shared experts' weight stream while
+// the preceding kernel still runs, which a cooperative launch does not.  Every
+// wait in the kernel is bounded.
 bool launch_splitk(FfnKernel kernel, size_t smem, const CUtensorMap* m, const FfnArgs& a, int grid, int sms,
                    cudaStream_t st) {
   if (grid > sms) return false;
