@@ -228,11 +228,12 @@ coli_status coli_moe_layer(const coli_moe_dims *dims, const coli_moe_weights *w,
  *                with_shared != 0, the S shared experts; same layouts as above
  *   out_partial  fp32 [T][H] (16-byte aligned; must not alias x)
  *   logits_out, topk_ids_out, topk_w_out, ws, ws_bytes, flags: as coli_moe_layer
- * Runs in the decode forms for T <= 128 (the split-K form up to 8 tokens, the
- * two-phase form above; with I = 128 not for T <= 4, whose two-phase kernel
- * combines in place); other batches and COLI_PATH_PREFILL return
+ * Runs in the prefill form (any batch; the tile plan covers the rank's
+ * experts only) and in the decode forms for T <= 128 (the split-K form up to 8
+ * tokens, the two-phase form above; with I = 128 not for T <= 4, whose
+ * two-phase kernel combines in place); decode batches above 128 tokens return
  * COLI_ERR_UNSUPPORTED; 0 <= expert_begin < expert_end <= E, else
- * COLI_ERR_INVALID_ARG.
+ * COLI_ERR_INVALID_ARG.  Host-memory flags are not accepted here.
  */
 coli_status coli_moe_layer_ep(const coli_moe_dims *dims, const coli_moe_weights *w, int expert_begin,
                               int expert_end, int with_shared, const uint16_t *x, int T, const float *logits_in,

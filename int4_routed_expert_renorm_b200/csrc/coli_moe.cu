@@ -526,16 +526,30 @@ bool launch_prefill(const CUtensorMap* m, const PfArgs& a, int grid, cudaStream_
          cudaSuccess;
 }
 
+// The experts one call computes: all of them, or an expert-parallel rank's
+// share (routed experts [begin, end), the shared ones when shared != 0), whose
+// weights then hold only those experts, and whose output is the unrounded
+// fp32 partial sum `out_f32`.
+struct EpRange {
+  bool on = false;
+  int begin = 0, end = 0, shared = 0;
+  const int32_t* ids = nullptr;
+  float* out_f32 = nullptr;
+};
+
 // Prefill form: gather the expert input into pair order, plan the token
 // blocks, gate/up GEMM (h), down GEMM (y), combine.
 coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
                             const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm,
                             const int32_t* pair_pos, const float* topk_w, const uint16_t* residual, uint16_t* out,
-                            const Ws& ws, const DevInfo& di, cudaStream_t st, const StageRecorder& rec) {
-  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k, S = d->n_shared;
+                            const Ws& ws, const DevInfo& di, cudaStream_t st, const StageRecorder& rec,
+                            const EpRange& ep = EpRange()) {
+  const int H = d->hidden, I = d->inter, E = d->n_experts, k = d->top_k;
+  const int S = ep.on ? ep.shared : d->n_shared;
+  const int E_w = ep.on ? ep.end - ep.begin : E;   // routed experts held by the weights
   const int P = T * k;
-  const uint64_t rows_gu = static_cast<uint64_t>(E + S) * I;
-  const uint64_t rows_dn = static_cast<uint64_t>(E + S) * H;
+  const uint64_t rows_gu = static_cast<uint64_t>(E_w + S) * I;
+  const uint64_t rows_dn = static_cast<uint64_t>(E_w + S) * H;
   CUtensorMap mg[8], md[8];   // q0, q1, s0, s1, token rows in boxes of 128, 64, 32, 16 rows
   const int G = d->group;
   if (!pf_weight_maps(w->gate_q, w->gate_s, rows_gu, H, G, &mg[0], &mg[2]) ||
@@ -561,7 +575,9 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
                 static_cast<const uint16_t*>(ws.xq), perm, k, P, H, ws.xg))
       return COLI_ERR_CUDA;
   }
-  if (!launch(pf_plan_kernel, dim3(1), dim3(1024), 0, st, n_unique, seg_off, T, S, ws.plan)) return COLI_ERR_CUDA;
+  if (!launch(pf_plan_kernel, dim3(1), dim3(1024), 0, st, n_unique, seg_off, T, S, ws.plan,
+              ep.on ? unique : static_cast<const int32_t*>(nullptr), ep.on ? ep.begin : 0, ep.on ? ep.end : E))
+    return COLI_ERR_CUDA;
   rec.mark(5);
 
   PfArgs a{};
@@ -579,6 +595,8 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
   a.E = E;
   a.S = S;
   a.P = P;
+  a.e_off = ep.on ? ep.begin : 0;
+  a.e_shared = E_w;
   const int Umax = P < E ? P : E;
   const long blocks_ub = static_cast<long>(Umax) + P / kPfMaxN + static_cast<long>(S) * (T / kPfMaxN + 1);
   auto grid_for = [&](int mb) {
@@ -605,26 +623,13 @@ coli_status run_ffn_prefill(const coli_moe_dims* d, const coli_moe_weights* w, i
     // per token at the memory's rate (4 x SMs left it ~10 % short at 4096 tokens)
     if (blocks > 16L * di.sms) blocks = 16L * di.sms;
     if (!launch(combine_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, st, static_cast<const float*>(ws.ypair),
-                pair_pos, topk_w, residual, T, k, S, H, out, static_cast<const int32_t*>(nullptr), 0, E,
-                static_cast<float*>(nullptr)))
+                pair_pos, topk_w, residual, T, k, S, H, out, ep.on ? ep.ids : static_cast<const int32_t*>(nullptr),
+                ep.on ? ep.begin : 0, ep.on ? ep.end : E, ep.on ? ep.out_f32 : static_cast<float*>(nullptr)))
       return COLI_ERR_CUDA;
   }
   rec.mark(8);
   return COLI_OK;
 }
-
-// The FFN + combine part shared by coli_moe_expert_ffn and coli_moe_layer;
-// the tile plan (ws.plan) must already be on the stream.
-// The experts one call computes: all of them, or an expert-parallel rank's
-// share (routed experts [begin, end), the shared ones when shared != 0), whose
-// weights then hold only those experts, and whose output is the unrounded
-// fp32 partial sum `out_f32`.
-struct EpRange {
-  bool on = false;
-  int begin = 0, end = 0, shared = 0;
-  const int32_t* ids = nullptr;
-  float* out_f32 = nullptr;
-};
 
 // The split-K kernel's own routing (logits not NULL): the batch's router
 // logits and bias, and where the ids and weights go; the union and the plan
@@ -645,6 +650,8 @@ inline bool splitk_routes(const coli_moe_dims* d, int T) {
   return T >= 2 && use_splitk(d, T) && T * d->top_k <= kWarpUnionMaxP && d->n_experts <= 256;
 }
 
+// The decode-form FFN + combine part shared by coli_moe_expert_ffn and
+// coli_moe_layer; the tile plan (ws.plan) must already be on the stream.
 coli_status run_ffn(const coli_moe_dims* d, const coli_moe_weights* w, int T, const int32_t* unique,
                     const int32_t* n_unique, const int32_t* seg_off, const int32_t* perm, const int32_t* pair_pos,
                     const float* topk_w, const uint16_t* residual, uint16_t* out, const Ws& ws, const DevInfo& di,
@@ -985,10 +992,11 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
     out = static_cast<uint16_t*>(const_cast<void*>(host_mapped(out)));
     if (!out) return COLI_ERR_INVALID_ARG;
   }
-  // an expert-parallel share runs in the decode forms, with route, union and
-  // plan in one kernel (T <= 128), and not through the two-phase kernel's
-  // own combine (T <= 4 with I = 128)
-  if (ep.on && !(form == Form::kDecode && T <= kFusedRouteMaxT && (use_splitk(dims, T) || T > kFusedCombineMaxT)))
+  // an expert-parallel share runs in the prefill form, or in the decode forms
+  // with route, union and plan in one kernel (T <= 128) and not through the
+  // two-phase kernel's own combine (T <= 4 with I = 128)
+  if (ep.on && !(form == Form::kPrefill || (form == Form::kDecode && T <= kFusedRouteMaxT &&
+                                            (use_splitk(dims, T) || T > kFusedCombineMaxT))))
     return COLI_ERR_UNSUPPORTED;
   const Ws lay = layout(dims, T, ws);
   if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
@@ -1089,10 +1097,10 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
     rec.mark_through(4, 5);
   }
   // 3. expert FFN and combine
+  ep.ids = ids;
   if (form == Form::kPrefill)
     return run_ffn_prefill(dims, w, T, lay.unique, lay.n_unique, lay.seg_off, lay.perm, lay.pair_pos, tw, residual,
-                           out, lay, di, s, rec);
-  ep.ids = ids;
+                           out, lay, di, s, rec, ep);
   InRoute ir;
   if (inroute) {
     ir.logits = lg;

@@ -58,6 +58,9 @@ struct PfArgs {
   float* ypair;               // down output: y [P+S*T][H]
   uint32_t* status;
   int H, I, T, k, E, S, P;
+  // expert-parallel rank: the weights hold routed experts [e_off, ...) at rows
+  // 0.. and the S shared ones from expert e_shared on (else 0 and E)
+  int e_off, e_shared;
 };
 
 // Shared-memory / TMEM plan of one launch.  NMAT weight blocks per tile share
@@ -203,12 +206,12 @@ __device__ __forceinline__ PfTile pf_decode(const PfArgs& a, const int32_t* blk_
   const int j = blk - blk_off[lo], nb = blk_off[lo + 1] - blk_off[lo];
   int cnt, sbase, obase;
   if (lo < U) {
-    ti.e = uniq[lo];
+    ti.e = uniq[lo] - a.e_off;
     sbase = seg[lo];
     cnt = seg[lo + 1] - sbase;
     obase = sbase;
   } else {
-    ti.e = a.E + (lo - U);
+    ti.e = a.e_shared + (lo - U);
     cnt = a.T;
     obase = a.P + (lo - U) * a.T;
     sbase = DOWN ? obase : a.P;   // gate/up: every shared segment reads the token-order rows
@@ -223,11 +226,14 @@ __device__ __forceinline__ PfTile pf_decode(const PfArgs& a, const int32_t* blk_
 }
 
 // Blocks of the prefill form: every segment (union experts, then shared
-// experts) split into ceil(cnt / 160) near-equal token blocks.
-// plan = [n_seg, total_blocks, blk_off[0..n_seg]].  One CTA of 1024 threads.
+// experts) split into ceil(cnt / 160) near-equal token blocks; with `uniq`
+// (an expert-parallel rank) routed segments of experts outside [eb, ee) get
+// none.  plan = [n_seg, total_blocks, blk_off[0..n_seg]].  One CTA of 1024
+// threads.
 __global__ void __launch_bounds__(1024) pf_plan_kernel(const int32_t* __restrict__ n_unique,
                                                        const int32_t* __restrict__ seg_off, int T, int S,
-                                                       int32_t* __restrict__ plan) {
+                                                       int32_t* __restrict__ plan, const int32_t* __restrict__ uniq,
+                                                       int eb, int ee) {
   pdl_wait();
   pdl_trigger();
   __shared__ int scratch[33];
@@ -235,6 +241,7 @@ __global__ void __launch_bounds__(1024) pf_plan_kernel(const int32_t* __restrict
   const int n_seg = U + S;
   auto nblk = [&](int s) -> int {
     if (s >= n_seg) return 0;
+    if (uniq && s < U && (uniq[s] < eb || uniq[s] >= ee)) return 0;
     const int cnt = s < U ? seg_off[s + 1] - seg_off[s] : T;
     return (cnt + kPfMaxN - 1) / kPfMaxN;
   };

@@ -65,7 +65,8 @@ def test_layer_ep_argument_checks():
     assert L(0, 128, 1, p=ctypes.c_void_p(0x300008)) == m._lib.COLI_ERR_INVALID_ARG   # partial not 16-byte aligned
     assert L(0, 128, 9) in (m._lib.COLI_OK, m._lib.COLI_ERR_CUDA)   # the two-phase form, T <= 128
     assert L(0, 128, 129) == m._lib.COLI_ERR_UNSUPPORTED      # route + union + plan in one kernel only
-    assert L(0, 128, 4, flags=0x20) == m._lib.COLI_ERR_UNSUPPORTED   # prefill form
+    assert L(0, 128, 4, flags=0x20) in (m._lib.COLI_OK, m._lib.COLI_ERR_CUDA)   # the prefill form
+    assert L(0, 128, 4, flags=0x2) == m._lib.COLI_ERR_UNSUPPORTED   # host-memory input
     assert L(0, 128, 0) == m._lib.COLI_OK                    # T = 0
     # past the checks a machine without a GPU stops at the device query
     assert L(0, 128, 4) in (m._lib.COLI_OK, m._lib.COLI_ERR_CUDA)

@@ -1,5 +1,5 @@
 """Expert parallelism on the GPU (split-K form up to 8 tokens, two-phase form
-up to 128), with the ranks emulated one after another
+up to 128, the prefill form at any size), with the ranks emulated one after another
 on one device (each rank's call is independent: nothing waits on another
 rank).  Each rank holds a contiguous range of the routed experts (rank 0 also
 the shared ones and the residual) and computes its fp32 share with
@@ -73,8 +73,12 @@ def _rel(a_bits, b_bits):
     return np.abs(a - b).max() / np.abs(b).max()
 
 
+PREFILL = 0x20
+
+
 @pytest.mark.parametrize("T,world,flags", [(1, 2, 0), (5, 3, 0), (8, 2, PRENORM), (3, 4, PRENORM),
-                                           (20, 3, 0), (64, 2, PRENORM), (100, 4, 0)])
+                                           (20, 3, 0), (64, 2, PRENORM), (100, 4, 0),
+                                           (40, 2, PREFILL), (300, 3, PREFILL | PRENORM), (200, 4, PREFILL)])
 def test_expert_parallel_small(lib, T, world, flags):
     shape = _small_shape(tokens=T, hidden=512, inter=256, n_experts=16, top_k=4, n_shared=1)
     full = sg.expert_tensors(shape, 23)
@@ -96,18 +100,18 @@ def test_expert_parallel_small(lib, T, world, flags):
     assert np.array_equal(out, oracle.f64_to_bf16_bits(total.astype(np.float64)))
 
 
-@pytest.mark.parametrize("T,world", [(1, 2), (4, 4), (24, 2)])
-def test_expert_parallel_glm_shape(lib, T, world):
+@pytest.mark.parametrize("T,world,form", [(1, 2, 0), (4, 4, 0), (24, 2, 0), (160, 2, PREFILL)])
+def test_expert_parallel_glm_shape(lib, T, world, form):
     """The GLM-5.2-shaped layer (H 6144, I 2048, top-8, one shared expert) with
     16 routed experts resident, spread over 2 and 4 ranks (24 tokens: the
-    two-phase form)."""
+    two-phase form; 160 tokens forced into the prefill form)."""
     base = synth.DECODE_B1_E16
     shape = synth.LayerShape(base.name, base.hidden, base.inter, base.n_experts, base.top_k, base.n_shared, T)
     full = sg.expert_tensors(shape, 0)
     li = synth.LayerInputs(shape, 0)
     x = np.concatenate([synth.activations(shape, 0, b)[:1] for b in range(T)])
-    out, _, routing = _ep_run(lib, shape, full, li, x, world, x, PRENORM)
-    ref_out, ref_routing = _whole(lib, shape, full, li, x, x, PRENORM)
+    out, _, routing = _ep_run(lib, shape, full, li, x, world, x, PRENORM | form)
+    ref_out, ref_routing = _whole(lib, shape, full, li, x, x, PRENORM | form)
     for lg, ids, w in routing:
         assert np.array_equal(ids, ref_routing[1]) and np.array_equal(w, ref_routing[2])
     err = _rel(out, ref_out)
