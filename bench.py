@@ -88,6 +88,8 @@ _PF_4096 = _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)
 TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
            ("glm52_layer_decode_b1_e16", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
            ("glm52_layer_prefill_512_e32", "prefill"): (532.914432e6 + 16.164864e6, _PF_SOURCES),
+           # the two-phase decode kernel (the same sources as the split-K one)
+           ("glm52_layer_decode_b64_zipf_e32", "decode"): (742.315776e6 + 16.262400e6, _SK_SOURCES),
            ("glm52_layer_prefill_4096", "prefill"): (_PF_4096, _PF_SOURCES),
            # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
            ("glm52_layer_prefill_4096_router", "prefill"): (_PF_4096, _PF_SOURCES)}
