@@ -82,12 +82,12 @@ def parse():
 # times its own algorithmic bytes (257 experts' gate+up codes and scales,
 # 36,864 gathered rows, h written).
 _SK_SOURCES = "30261d98ff90c3f0"
-_PF_SOURCES = "64537c0e6dc7cceb"
-_PF_RATIO = (532.914432e6 + 16.164864e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
+_PF_SOURCES = "f68518e319918e88"
+_PF_RATIO = (532.678912e6 + 16.509440e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
 _PF_4096 = _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)
 TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
            ("glm52_layer_decode_b1_e16", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
-           ("glm52_layer_prefill_512_e32", "prefill"): (532.914432e6 + 16.164864e6, _PF_SOURCES),
+           ("glm52_layer_prefill_512_e32", "prefill"): (532.678912e6 + 16.509440e6, _PF_SOURCES),
            # the two-phase decode kernel (the same sources as the split-K one)
            ("glm52_layer_decode_b64_zipf_e32", "decode"): (742.315776e6 + 16.262400e6, _SK_SOURCES),
            ("glm52_layer_prefill_4096", "prefill"): (_PF_4096, _PF_SOURCES),
