@@ -37,8 +37,11 @@
  *   int8 container (dims.code_bits == 8; the README requires the MTP head to
  *   be int8, "Decodifica speculativa, onestamente"): the same layout with one
  *   two's-complement byte per code, gate_q/up_q [E+S][I][H], down_q
- *   [E+S][H][I].  It runs in the decode form for T <= 8 (the MTP head's draft
- *   batches); other batches and the prefill form return COLI_ERR_UNSUPPORTED.
+ *   [E+S][H][I].  It runs in the split-K decode form (I a multiple of 256):
+ *   batches of up to 8 tokens (the MTP head's draft batches) in one pass,
+ *   larger ones in consecutive 8-token passes (each token's output is that of
+ *   its batch-1 call; the weights are read once per pass); COLI_PATH_PREFILL
+ *   returns COLI_ERR_UNSUPPORTED.
  *
  * Conventions for every call:
  *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
@@ -114,7 +117,8 @@ typedef enum {
  * also computes that tile's K slice of the down projection (fixed-order
  * partial sums; a token's output is the same bits in any batch of up to 8);
  * otherwise gate/up tiles and then down tiles, in blocks of 16 (T <= 64) or
- * 32 tokens.  int8 codes (dims.code_bits == 8) take the first only. */
+ * 32 tokens.  int8 codes (dims.code_bits == 8) take the first only, in 8-token
+ * passes above 8 tokens. */
 
 typedef struct {
   int32_t hidden;     /* H */

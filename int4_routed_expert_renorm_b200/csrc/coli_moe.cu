@@ -480,7 +480,8 @@ Form choose_form(uint32_t flags, int T, const coli_moe_dims* d) {
   const int E = d->n_experts, k = d->top_k;
   const bool fd = (flags & COLI_PATH_DECODE) != 0, fp = (flags & COLI_PATH_PREFILL) != 0;
   if (fd && fp) return Form::kInvalid;
-  if (code_bits(d) == 8) return (fp || !use_splitk(d, T)) ? Form::kUnsupported : Form::kDecode;
+  // int8 codes: the split-K decode form, batches above 8 tokens in 8-token passes
+  if (code_bits(d) == 8) return (fp || d->inter % 256 != 0) ? Form::kUnsupported : Form::kDecode;
   if (fd) return Form::kDecode;
   if (fp) return Form::kPrefill;
   const long P = static_cast<long>(T) * k;
@@ -837,7 +838,8 @@ coli_status coli_moe_union_offsets(const coli_moe_dims* dims, int T, size_t* off
   // the layout of a workspace based at address 0 gives the offsets (256-byte
   // aligned, so any workspace the calls accept has the same ones)
   uint8_t* const base = reinterpret_cast<uint8_t*>(uintptr_t(256));
-  const Ws w = layout(dims, T, base);
+  // int8 batches above 8 tokens run in 8-token passes: the last pass's union
+  const Ws w = layout(dims, code_bits(dims) == 8 && T > kSkMaxT ? kSkMaxT : T, base);
   auto rel = [&](const void* p) { return static_cast<size_t>(static_cast<const uint8_t*>(p) - base); };
   off[0] = rel(w.unique);
   off[1] = rel(w.n_unique);
@@ -859,7 +861,9 @@ coli_status coli_moe_ffn_form(const coli_moe_dims* dims, int T, uint32_t flags, 
     case Form::kInvalid: return COLI_ERR_INVALID_ARG;
     case Form::kUnsupported: return COLI_ERR_UNSUPPORTED;
     case Form::kPrefill: *form = COLI_FORM_PREFILL; return COLI_OK;
-    case Form::kDecode: *form = use_splitk(dims, T) ? COLI_FORM_DECODE_SPLITK : COLI_FORM_DECODE_TWOPHASE; return COLI_OK;
+    case Form::kDecode:
+      *form = (use_splitk(dims, T) || code_bits(dims) == 8) ? COLI_FORM_DECODE_SPLITK : COLI_FORM_DECODE_TWOPHASE;
+      return COLI_OK;
   }
   return COLI_ERR_INVALID_ARG;
 }
@@ -972,6 +976,24 @@ coli_status layer_impl(const coli_moe_dims* dims, const coli_moe_weights* w, con
   const Form form = choose_form(flags, T, dims);
   if (form == Form::kInvalid) return COLI_ERR_INVALID_ARG;
   if (form == Form::kUnsupported) return COLI_ERR_UNSUPPORTED;
+  // int8 codes above 8 tokens: consecutive passes of up to 8 tokens through
+  // the split-K form, each a whole layer call on its rows (every token's output
+  // is the bits of its batch-1 output; the weights are read once per pass)
+  if (code_bits(dims) == 8 && T > kSkMaxT) {
+    const int H = dims->hidden, E = dims->n_experts, k = dims->top_k;
+    for (int t0 = 0; t0 < T; t0 += kSkMaxT) {
+      const int tc = std::min(kSkMaxT, T - t0);
+      const size_t oh = static_cast<size_t>(t0) * H, oe = static_cast<size_t>(t0) * E, ok = static_cast<size_t>(t0) * k;
+      EpRange epc = ep;
+      if (ep.out_f32) epc.out_f32 = ep.out_f32 + oh;
+      const coli_status sc = layer_impl(dims, w, x + oh, tc, logits_in ? logits_in + oe : nullptr,
+                                        residual ? residual + oh : nullptr, flags, out ? out + oh : nullptr,
+                                        logits_out ? logits_out + oe : nullptr, topk_ids_out ? topk_ids_out + ok : nullptr,
+                                        topk_w_out ? topk_w_out + ok : nullptr, ws, ws_bytes, stream, epc, tier);
+      if (sc != COLI_OK) return sc;
+    }
+    return COLI_OK;
+  }
   // a host-RAM tier: decode form, no expert-parallel share, and every batch's
   // union must fit the slots
   if (tier && (form != Form::kDecode || ep.on ||

@@ -110,7 +110,10 @@ def test_layer_argument_checks(colimoe):
     assert L(d, w, x, 4, ws, need - 1) == m._lib.COLI_ERR_WORKSPACE
     assert L(_dims(m, group=16), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, group=64, inter=1280), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
-    assert L(_dims(m, code_bits=8), w, x, 9, ws, m.coli_moe_workspace_bytes(d, 9)) == m._lib.COLI_ERR_UNSUPPORTED
+    # int8 above 8 tokens: 8-token passes (past the checks a machine without a GPU stops at the device query)
+    assert L(_dims(m, code_bits=8), w, x, 9, ws, m.coli_moe_workspace_bytes(d, 9)) in (m._lib.COLI_OK,
+                                                                                      m._lib.COLI_ERR_CUDA)
+    assert L(_dims(m, code_bits=8), w, x, 9, ws, m.coli_moe_workspace_bytes(d, 8) - 256) == m._lib.COLI_ERR_WORKSPACE
     assert L(_dims(m, code_bits=8), w, x, 4, ws, need, 0x20) == m._lib.COLI_ERR_UNSUPPORTED   # forced prefill
     assert L(_dims(m, inter=384), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
     assert L(_dims(m, n_shared=9), w, x, 4, ws, need) == m._lib.COLI_ERR_UNSUPPORTED
@@ -209,8 +212,8 @@ def _form_rule(T, E, k, inter=2048, code_bits=4, flags=0):
     if fd and fp:
         return "invalid"
     splitk = T <= 8 and inter % 256 == 0
-    if code_bits == 8:
-        return 1 if (splitk and not fp) else "unsupported"
+    if code_bits == 8:   # the split-K form, batches above 8 tokens in 8-token passes
+        return 1 if (inter % 256 == 0 and not fp) else "unsupported"
     P = T * k
     prefill = fp or (not fd and T >= 32 and P >= 32 * min(E, P))
     return 3 if prefill else (1 if splitk else 2)
@@ -283,8 +286,8 @@ def test_gpu_tests_exercise_the_form_they_name(colimoe):
         for T in (9, 64, 65):
             shape = _small_shape(tokens=T, hidden=512, inter=inter, n_experts=8, top_k=2, n_shared=1)
             assert form(shape) == m._lib.COLI_FORM_DECODE_TWOPHASE, (inter, T)
-    with pytest.raises(m._lib.ColiError):
-        form(_small_shape(bits=8, tokens=9, inter=256))
+    # int8 batches above 8 tokens run the split-K form in 8-token passes
+    assert form(_small_shape(bits=8, tokens=9, inter=256)) == m._lib.COLI_FORM_DECODE_SPLITK
 
 
 @pytest.mark.parametrize("bits", [4, 8])

@@ -3,7 +3,8 @@
 The README requires the MTP head to be int8 ("Decodifica speculativa,
 onestamente"); the library takes the int4 container with one
 two's-complement byte per code (dims.code_bits = 8) through the split-K
-decode form, for the head's draft batches of up to 8 tokens.  Each code is
+decode form: the head's draft batches of up to 8 tokens in one pass, larger
+batches in consecutive 8-token passes.  Each code is
 split into a signed high nibble (decoded straight to 16 * hi) and an
 unsigned low nibble that meet the same activation fragment in the MMA.
 """
@@ -36,13 +37,29 @@ def test_int8_small_shapes(lib, kw):
     print(f"int8 {kw}: max rel err {err:.3e}")
 
 
-def test_int8_unsupported_batches_are_rejected(lib):
-    shape = _small_shape(bits=8, tokens=9, inter=256)
+@pytest.mark.parametrize("T", [9, 20])
+def test_int8_batches_above_8_tokens_run_in_passes(lib, T):
+    """int8 batches above 8 tokens run as consecutive 8-token split-K passes:
+    every token's output is the bits of its own batch-1 output, and the layer
+    matches the oracle; the prefill form stays unsupported for int8 codes."""
+    shape = _small_shape(bits=8, tokens=T, inter=256)
     layer = device_layer(shape, seed=42)
-    x = to_dev_bits(synth.normal_bf16(42, 5, synth.X_IN, (9, shape.hidden)))
-    with pytest.raises(lib.ColiError):
-        layer.forward(x, torch.empty_like(x), layer.workspace(9))
-    x4 = x[:4].contiguous()
+    li = synth.LayerInputs(shape, seed=42)
+    x = synth.normal_bf16(42, 5, synth.X_IN, (T, shape.hidden))
+    res = synth.normal_bf16(42, 6, synth.X_IN, (T, shape.hidden))
+    err, g = check_layer(lib, shape, layer, oracle_weights(shape, seed=42), x, rw=li.router_w(), residual_bits=res)
+    print(f"int8 T={T} in 8-token passes: max rel err {err:.3e}")
+    xd, rd = to_dev_bits(x), to_dev_bits(res)
+    whole = torch.empty_like(xd)
+    layer.forward(xd, whole, layer.workspace(T), residual=rd)
+    one = torch.empty_like(xd[:1])
+    ws1 = layer.workspace(1)
+    for t in range(T):
+        layer.forward(xd[t:t + 1].contiguous(), one, ws1, residual=rd[t:t + 1].contiguous())
+        assert torch.equal(one[0], whole[t]), t
+    st, fl = lib.coli_moe_get_status()
+    assert st == 0 and fl == 0
+    x4 = xd[:4].contiguous()
     with pytest.raises(lib.ColiError):
         layer.forward(x4, torch.empty_like(x4), layer.workspace(4), flags=0x20)   # COLI_PATH_PREFILL
 
