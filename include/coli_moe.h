@@ -401,6 +401,19 @@ coli_status coli_moe_layer_tiered(const coli_moe_dims *dims, const coli_moe_weig
 coli_status coli_moe_tier_prefetch(const coli_moe_dims *dims, const coli_moe_weights *slots,
                                    const coli_moe_tier *tier, const int32_t *ids, int32_t n, void *stream);
 
+/* Overlap, lookahead form (the pages' router lookahead: routing one layer
+ * ahead is largely predictable): routes x with the NEXT layer's router
+ * (`next`: that layer's slot arrays with its router weight and bias) and
+ * places the experts it selects in that layer's tier, as coli_moe_tier_prefetch
+ * would (nothing counted as routed).  Meant to run on another stream while the
+ * current layer computes.  x: bf16 [T][H] device rows (COLI_LAYER_PRENORM
+ * applies the next layer's pre-norm); min(E, T*k) <= C, else
+ * COLI_ERR_UNSUPPORTED; ws: a workspace of coli_moe_workspace_bytes(dims, T)
+ * bytes that no concurrent call uses (its routing arrays are overwritten). */
+coli_status coli_moe_tier_lookahead(const coli_moe_dims *dims, const coli_moe_weights *next,
+                                    const coli_moe_tier *next_tier, const uint16_t *x, int T, uint32_t flags,
+                                    void *ws, size_t ws_bytes, void *stream);
+
 /* Static description of a status code. */
 const char *coli_status_str(coli_status s);
 

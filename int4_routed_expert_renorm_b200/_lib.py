@@ -26,7 +26,8 @@ EXPORTS = ("coli_moe_route", "coli_moe_union", "coli_moe_expert_ffn", "coli_moe_
            "coli_moe_workspace_bytes", "coli_moe_get_status", "coli_status_str", "coli_moe_version",
            "coli_moe_launch_count", "coli_moe_set_stage_events", "coli_moe_layer_noalloc", "coli_moe_ffn_form",
            "coli_moe_union_offsets", "coli_moe_test_wait_timeout", "coli_moe_layer_ep", "coli_moe_partial_to_bf16",
-           "coli_moe_tier_state_bytes", "coli_moe_tier_reset", "coli_moe_layer_tiered", "coli_moe_tier_prefetch")
+           "coli_moe_tier_state_bytes", "coli_moe_tier_reset", "coli_moe_layer_tiered", "coli_moe_tier_prefetch",
+           "coli_moe_tier_lookahead")
 COLI_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -82,6 +83,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "coli_moe_tier_reset": (I, [D, TR, P]),
         "coli_moe_layer_tiered": (I, [D, W, TR, P, I, P, P, U32, P, P, P, P, P, Z, P]),
         "coli_moe_tier_prefetch": (I, [D, W, TR, P, I, P]),
+        "coli_moe_tier_lookahead": (I, [D, W, TR, P, I, U32, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -291,6 +293,15 @@ def coli_moe_tier_prefetch(dims, slots, tier, ids, stream=None):
         raise ValueError("ids: int32 expert ids")
     _check(_lib.coli_moe_tier_prefetch(ctypes.byref(dims), ctypes.byref(slots), ctypes.byref(tier), _ptr(ids),
                                        ids.numel(), _stream(stream)), "coli_moe_tier_prefetch")
+
+
+def coli_moe_tier_lookahead(dims, next_slots, next_tier, x, ws, flags=0, stream=None):
+    """Routes x with the next layer's router and places its experts in that
+    layer's tier (see the header)."""
+    T = _tokens(x, dims.hidden)
+    _check(_lib.coli_moe_tier_lookahead(ctypes.byref(dims), ctypes.byref(next_slots), ctypes.byref(next_tier),
+                                        _ptr(x), T, flags, _ptr(ws), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "coli_moe_tier_lookahead")
 
 
 def coli_moe_partial_to_bf16(partial, out, stream=None):

@@ -1309,6 +1309,56 @@ coli_status coli_moe_tier_prefetch(const coli_moe_dims* dims, const coli_moe_wei
              : COLI_ERR_CUDA;
 }
 
+coli_status coli_moe_tier_lookahead(const coli_moe_dims* dims, const coli_moe_weights* next,
+                                    const coli_moe_tier* next_tier, const uint16_t* x, int T, uint32_t flags,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  TierArgs ta;
+  coli_status st = tier_args(dims, next_tier, next, &ta);
+  if (st != COLI_OK) return st;
+  if ((st = check_weights(next, true)) != COLI_OK) return st;
+  if (T < 0) return COLI_ERR_INVALID_ARG;
+  if (T == 0) return COLI_OK;
+  const int H = dims->hidden, E = dims->n_experts, k = dims->top_k;
+  if (std::min<int64_t>(E, static_cast<int64_t>(T) * k) > ta.slots) return COLI_ERR_UNSUPPORTED;
+  if (!x || !ws || !aligned(x, 16) || !aligned(ws, 256)) return COLI_ERR_INVALID_ARG;
+  const Ws lay = layout(dims, T, ws);
+  if (ws_bytes < lay.bytes) return COLI_ERR_WORKSPACE;
+  DevInfo di;
+  if (dev_info(&di) != COLI_OK) return COLI_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int prenorm = (flags & COLI_LAYER_PRENORM) ? 1 : 0;
+  // the next layer's logits of x, as its own call would compute them
+  if (T <= 8) {
+    if (!launch(front_kernel, dim3(E + T), dim3(256), 0, s, x, next->router_w, T, E, H, prenorm, lay.logits, lay.xn,
+                lay.xq, static_cast<uint8_t*>(nullptr), static_cast<int32_t*>(nullptr), 0, di.status,
+                static_cast<int32_t*>(nullptr)))
+      return COLI_ERR_CUDA;
+  } else {
+    if (!launch(prep_kernel, dim3(T), dim3(256), 0, s, x, H, prenorm, lay.xn, lay.xq, static_cast<uint8_t*>(nullptr),
+                static_cast<int32_t*>(nullptr), 0, di.status))
+      return COLI_ERR_CUDA;
+    const uint16_t* xr = prenorm ? lay.xn : x;
+    if (T >= kLogitsMmaMinT) {
+      if (!launch(logits_mma_kernel, dim3((E + kLgBN - 1) / kLgBN, (T + kLgBM - 1) / kLgBM), dim3(256), 0, s, xr,
+                  next->router_w, T, E, H, lay.logits))
+        return COLI_ERR_CUDA;
+    } else {
+      const int tt = logits_tokens_per_block(H);
+      if (!launch(logits_tile_kernel, dim3((E + 7) / 8, (T + tt - 1) / tt), dim3(256), static_cast<size_t>(tt) * H * 2,
+                  s, xr, next->router_w, T, E, H, tt, lay.logits))
+        return COLI_ERR_CUDA;
+    }
+  }
+  // its top-k, then the selected experts placed (repeats are placed once)
+  if (!launch_route(lay.logits, next->router_bias, T, E, k, lay.ids, lay.w, di.status, s)) return COLI_ERR_CUDA;
+  return launch(tier_place_kernel, dim3(1), dim3(256), 0, s, static_cast<const int32_t*>(lay.ids), T * k,
+                static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr), E, ta.slots, ta.state,
+                static_cast<int32_t*>(nullptr), di.status) &&
+                 launch(tier_fill_kernel, dim3(4 * di.sms), dim3(256), 0, s, ta.cp, ta.state, E, ta.slots)
+             ? COLI_OK
+             : COLI_ERR_CUDA;
+}
+
 coli_status coli_moe_test_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns, void* stream) {
   if (limit_ns == 0 || limit_ns > kWaitLimitNs) return COLI_ERR_INVALID_ARG;
   if (elapsed_ns && !aligned(elapsed_ns, 8)) return COLI_ERR_INVALID_ARG;

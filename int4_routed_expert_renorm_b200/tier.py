@@ -11,8 +11,8 @@ import numpy as np
 import torch
 
 from ._lib import (COLI_ERR_INVALID_ARG, ColiError, coli_moe_dims, coli_moe_layer_tiered, coli_moe_tier,
-                   coli_moe_tier_prefetch, coli_moe_tier_reset, coli_moe_tier_state_bytes, coli_moe_weights,
-                   coli_moe_workspace_bytes)
+                   coli_moe_tier_lookahead, coli_moe_tier_prefetch, coli_moe_tier_reset, coli_moe_tier_state_bytes,
+                   coli_moe_weights, coli_moe_workspace_bytes)
 
 _NAMES = ("gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s")
 
@@ -66,6 +66,13 @@ class TieredLayer:
     def prefetch(self, ids: torch.Tensor, stream=None):
         """Place experts `ids` (device int32, at most n_slots) ahead of use."""
         coli_moe_tier_prefetch(self.dims, self.weights, self.tier, ids.contiguous(), stream)
+
+    def lookahead(self, x: torch.Tensor, ws: torch.Tensor, flags: int = 0, stream=None):
+        """Route x (the previous layer's input, on the device) with this
+        layer's router and place the experts it selects: run it on another
+        stream while the previous layer computes.  `ws` is a workspace of its
+        own (``workspace(T)``)."""
+        coli_moe_tier_lookahead(self.dims, self.weights, self.tier, x, ws, flags, stream)
 
     # ---- Learn: the usage counts, kept across runs ----------------------------
     def usage(self) -> np.ndarray:

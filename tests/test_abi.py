@@ -169,6 +169,11 @@ def test_tier_state_bytes_and_argument_checks(colimoe):
     assert lib.coli_moe_layer_tiered(ctypes.byref(d), ctypes.byref(w), ctypes.byref(t), x, 1, None, None, 0, out,
                                      None, None, None, ws, m.coli_moe_workspace_bytes(d, 1),
                                      None) == m._lib.COLI_ERR_INVALID_ARG
+    assert lib.coli_moe_tier_lookahead(ctypes.byref(d), ctypes.byref(w), ctypes.byref(t), x, 1, 0, ws,
+                                       m.coli_moe_workspace_bytes(d, 1), None) == m._lib.COLI_ERR_INVALID_ARG
+    assert lib.coli_moe_tier_lookahead(ctypes.byref(d), ctypes.byref(w),
+                                       ctypes.byref(m.coli_moe_tier(f, f, f, f, f, f, 0, f)), x, 1, 0, ws,
+                                       m.coli_moe_workspace_bytes(d, 1), None) == m._lib.COLI_ERR_INVALID_ARG
 
 
 def test_binding_host_flags_need_page_locked_tensors(colimoe):

@@ -209,3 +209,35 @@ def test_tier_warm_start_from_a_usage_profile(m):
     assert np.array_equal(bits(o_t), bits(o_r))
     del full, resident, tl
     torch.cuda.empty_cache()
+
+
+def test_tier_lookahead_places_the_next_layers_experts(m):
+    """Overlap: routing a layer's input with the next layer's router on a side
+    stream places that layer's experts while the current one runs; when the
+    next layer then sees the same rows it routes them identically and misses
+    nothing."""
+    E, k, C, T = 32, 2, 8, 3
+    shape, full, resident, cur = _setup(m, T, E, k, C, seed=45)
+    shape2, full2, resident2, nxt = _setup(m, T, E, k, C, seed=46)
+    x = synth.normal_bf16(45, 5, synth.X_IN, (T, 512))
+    xd = to_dev_bits(x)
+    o_cur = torch.empty_like(xd)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    ws_side = nxt.workspace(T)
+    with torch.cuda.stream(side):
+        nxt.lookahead(xd, ws_side, stream=side)
+    cur.forward(xd, o_cur, cur.workspace(T))           # the current layer meanwhile
+    torch.cuda.current_stream().wait_stream(side)
+    st = nxt.state_arrays()
+    assert st["fills"] > 0 and st["hits"] == 0 and st["misses"] == 0 and st["usage"].sum() == 0
+    o_t, o_r = torch.empty_like(xd), torch.empty_like(xd)
+    nxt.forward(xd, o_t, nxt.workspace(T))
+    resident2.forward(xd, o_r, resident2.workspace(T))
+    st = nxt.state_arrays()
+    assert st["misses"] == 0 and st["hits"] > 0
+    assert np.array_equal(bits(o_t), bits(o_r))
+    s_, fl = m.coli_moe_get_status()
+    assert s_ == 0 and fl == 0
+    del full, resident, cur, full2, resident2, nxt
+    torch.cuda.empty_cache()
