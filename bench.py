@@ -195,13 +195,14 @@ class ClockSampler:
 _KINDS = {"gate": (synth.GATE_Q, synth.GATE_S), "up": (synth.UP_Q, synth.UP_S), "down": (synth.DOWN_Q, synth.DOWN_S)}
 
 
-def _oracle_tokens(name: str, batch: int, toks: list[int]) -> tuple[float, int]:
+def _oracle_tokens(name: str, batch: int, toks: list[int], warm: int = 0) -> tuple[float, int]:
     """Time the plain-C oracle (oracle/c/moe_ref.c, -O2, one thread) on tokens
     `toks` of input batch `batch` of a workload, one token per call, each on
     the first layer of the workload: the weights of the experts a token
     selects are generated beforehand (untimed); the timed call is the C
     oracle's whole layer (logits or given logits, route, union, expert FFN,
-    combine; pre-norm for the stack).  Returns (seconds, calls)."""
+    combine; pre-norm for the stack).  The first `warm` calls run untimed
+    (warm-up).  Returns (seconds, timed calls)."""
     import oracle.cref as cr
     cr.build()
     shape = synth.WORKLOADS[name]
@@ -213,7 +214,7 @@ def _oracle_tokens(name: str, batch: int, toks: list[int]) -> tuple[float, int]:
     if shape.logits_in:
         lg = synth.normal_f32(0, 1000 + batch, synth.LOGITS_IN, (shape.tokens, shape.n_experts), 1.0)
     elapsed = 0.0
-    for t in toks:
+    for n_call, t in enumerate(toks):
         xt = x[t:t + 1]
         xin = cr.rms_norm(xt) if shape.prenorm else xt
         lt = None if lg is None else lg[t:t + 1]
@@ -227,8 +228,9 @@ def _oracle_tokens(name: str, batch: int, toks: list[int]) -> tuple[float, int]:
         cr.moe_layer_experts(lambda kind, e: held[(kind, e)], shape.hidden, shape.inter, xin, shape.n_experts,
                              shape.top_k, shape.n_shared, shape.group, shape.bits, router_w=rw, bias=bias,
                              logits_in=lt, residual_bits=xt if shape.prenorm else None, experts=need)
-        elapsed += time.perf_counter() - t0
-    return elapsed, len(toks)
+        if n_call >= warm:
+            elapsed += time.perf_counter() - t0
+    return elapsed, len(toks) - min(warm, len(toks))
 
 
 def cpu_model() -> str:
@@ -241,7 +243,7 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def oracle_sample(shape: synth.LayerShape, seconds: float):
+def oracle_sample(shape: synth.LayerShape, seconds: float, warm: int = 0):
     """Time the CPU oracle, as it stands, on a bounded sample of the workload.
 
     The plain-C oracle, one token per call.  Decode and stack workloads: one
@@ -250,7 +252,8 @@ def oracle_sample(shape: synth.LayerShape, seconds: float):
     process per host core (spawned, so no CUDA state is inherited), each
     timing its own share of tokens; throughput = all tokens over the longest
     worker's oracle time.  The stack times one layer per token and scales by
-    the layer count.  Returns (tokens/s, cores, calls, description)."""
+    the layer count.  `warm` untimed warm-up calls precede the timed ones
+    (in every process).  Returns (tokens/s, cores, timed calls, description)."""
     per_call = 4.0 if shape.hidden >= 4096 else 0.001      # rough C-oracle seconds per token (GLM shape)
     ncores = os.cpu_count() or 1
     parallel = shape.tokens >= 512 and ncores > 1
@@ -261,8 +264,10 @@ def oracle_sample(shape: synth.LayerShape, seconds: float):
             step = max(1, shape.tokens // max(1, n))
             toks = [(i // shape.tokens, (i * step) % shape.tokens) for i in range(n)]
         el, calls = 0.0, 0
-        for b in sorted({bt for bt, _ in toks}):
-            e, c = _oracle_tokens(shape.name, b, [t for bb, t in toks if bb == b])
+        for i, b in enumerate(sorted({bt for bt, _ in toks})):
+            tl = [t for bb, t in toks if bb == b]
+            w = warm if i == 0 else 0
+            e, c = _oracle_tokens(shape.name, b, tl[:1] * w + tl, w)
             el += e
             calls += c
         el *= shape.layers
@@ -275,14 +280,15 @@ def oracle_sample(shape: synth.LayerShape, seconds: float):
         tok_lists = [[(w * per_worker + i) * 131 % shape.tokens for i in range(per_worker)] for w in range(ncores)]
         ctx = mp.get_context("spawn")
         with ctx.Pool(ncores) as pool:
-            res = pool.starmap(_oracle_tokens, [(shape.name, 0, tl) for tl in tok_lists])
+            res = pool.starmap(_oracle_tokens, [(shape.name, 0, tl[:1] * warm + tl, warm) for tl in tok_lists])
         el = max(e for e, _ in res)
         calls = sum(c for _, c in res)
         cores = ncores
         desc = (f"{calls} calls of 1 token each of {shape.name}, {per_worker} per process on {ncores} processes "
                 f"(spawned), throughput = tokens / longest process; plain C oracle (gcc -O2, -ffp-contract=off)")
     desc += (f"{'; one layer timed, x' + str(shape.layers) + ' for the stack' if shape.layers > 1 else ''}"
-             f"; touched experts' weights generated untimed; host: {ncores} cores, {cpu_model()}")
+             f"; touched experts' weights generated untimed"
+             f"{f'; {warm} untimed warm-up call(s) first' if warm else ''}; host: {ncores} cores, {cpu_model()}")
     return calls / el, cores, calls, desc
 
 
@@ -323,10 +329,12 @@ def run_reference(a):
     if rank != 0:
         return 0
     shape = synth.WORKLOADS[a.workload]
-    v, cores, calls, desc = oracle_sample(shape, max(5.0, a.cpu_seconds))
+    # warm-up: up to 3 untimed oracle calls (each takes seconds at the GLM shape)
+    warm = max(1, min(a.warmup, 3))
+    v, cores, calls, desc = oracle_sample(shape, max(5.0, a.cpu_seconds), warm)
     # a step here is one timed oracle call (one token; for the stack, one
     # token through all layers)
-    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus, "steps": calls, "warmup": 0,
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus, "steps": calls, "warmup": warm,
             "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": workload_config(shape, a.batches),
