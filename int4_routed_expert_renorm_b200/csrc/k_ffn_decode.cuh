@@ -666,7 +666,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   using F = FusedCfg<NT, KCD, GROUP>;
   constexpr int NS = F::NS, STAGE = F::STAGE;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KiB-aligned start, as an offset from smem_raw so that the compiler
+  // keeps every pointer derived from it in the shared state space (ld.shared
+  // / st.shared rather than generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   float* red = reinterpret_cast<float*>(smem + NS * STAGE);
   int32_t* meta = reinterpret_cast<int32_t*>(smem + NS * STAGE + F::RED_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE + F::RED_BYTES + F::META_BYTES);

@@ -296,7 +296,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                        const __grid_constant__ CUtensorMap mb32, const __grid_constant__ CUtensorMap mb16, PfArgs a) {
   using C = PfCfg<NMAT>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KiB-aligned start, as an offset from smem_raw so that the compiler
+  // keeps every pointer derived from it in the shared state space (ld.shared
+  // / st.shared rather than generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* cst_base = smem;
   uint8_t* bst_base = smem + C::NSC * C::CSTAGE;
   int32_t* meta = reinterpret_cast<int32_t*>(bst_base + C::NSB * C::BSTAGE);

@@ -764,7 +764,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   using F = SkCfg<GROUP, BITS>;
   constexpr int NS = F::NS, STAGE = F::STAGE;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KiB-aligned start, as an offset from smem_raw so that the compiler
+  // keeps every pointer derived from it in the shared state space (ld.shared
+  // / st.shared rather than generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* fixed = smem + NS * STAGE;
   float* red = reinterpret_cast<float*>(fixed);
   int32_t* meta = reinterpret_cast<int32_t*>(fixed + F::RED_BYTES);
