@@ -77,19 +77,19 @@ def parse():
 # digest (a kernel changed since the counters were taken) the line reports
 # null.  The batch-1 capture ran on the 16-expert variant of the layer, which
 # moves the same 9 experts per step; the prefill capture on the 32-expert,
-# 512-token variant (same tile shapes), where DRAM traffic was 1.063x the
+# 512-token variant (same tile shapes), where DRAM traffic was 1.067x the
 # algorithmic bytes of the gate/up launch; the 4096-token figure is that ratio
 # times its own algorithmic bytes (257 experts' gate+up codes and scales,
 # 36,864 gathered rows, h written).
-_SK_SOURCES = "30261d98ff90c3f0"
-_PF_SOURCES = "f68518e319918e88"
-_PF_RATIO = (532.678912e6 + 16.509440e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
+_SK_SOURCES = "1b3dc4bd04b4489a"
+_PF_SOURCES = "70d5aa5efa5b0120"
+_PF_RATIO = (532.818432e6 + 18.652416e6) / (33 * 2 * 6684672 + 4608 * 6144 * 2 + 4608 * 2048 * 2)
 _PF_4096 = _PF_RATIO * (257 * 2 * 6684672 + 36864 * 6144 * 2 + 36864 * 2048 * 2)
-TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
-           ("glm52_layer_decode_b1_e16", "decode"): (191.316224e6 + 4.540160e6, _SK_SOURCES),
-           ("glm52_layer_prefill_512_e32", "prefill"): (532.678912e6 + 16.509440e6, _PF_SOURCES),
+TRAFFIC = {("glm52_layer_decode_b1", "decode"): (191.196416e6 + 5.173248e6, _SK_SOURCES),
+           ("glm52_layer_decode_b1_e16", "decode"): (191.196416e6 + 5.173248e6, _SK_SOURCES),
+           ("glm52_layer_prefill_512_e32", "prefill"): (532.818432e6 + 18.652416e6, _PF_SOURCES),
            # the two-phase decode kernel (the same sources as the split-K one)
-           ("glm52_layer_decode_b64_zipf_e32", "decode"): (742.315776e6 + 16.262400e6, _SK_SOURCES),
+           ("glm52_layer_decode_b64_zipf_e32", "decode"): (758.119168e6 + 16.141824e6, _SK_SOURCES),
            ("glm52_layer_prefill_4096", "prefill"): (_PF_4096, _PF_SOURCES),
            # same gate/up launch: all 256 routed experts and the shared one touched, 36,864 rows
            ("glm52_layer_prefill_4096_router", "prefill"): (_PF_4096, _PF_SOURCES)}
